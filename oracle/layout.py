@@ -55,7 +55,8 @@ def philox_stream(seed: int, i: int, h: int, count: int) -> list[int]:
     """First ``count`` raw 64-bit words of Philox4x64-10 for query block i, head h."""
     if count <= 0:
         return []
-    bg = np.random.Philox(key=[seed & 0xFFFFFFFFFFFFFFFF, 0], counter=[0, i, h, 0])
+    key = np.array([seed & 0xFFFFFFFFFFFFFFFF, 0], dtype=np.uint64)  # no float round trip
+    bg = np.random.Philox(key=key, counter=np.array([0, i, h, 0], dtype=np.uint64))
     return [int(x) for x in bg.random_raw(count)]
 
 
