@@ -1,0 +1,236 @@
+"""Thin ctypes binding of libbsa.so (the C ABI in include/bsa.h).
+
+Argument marshalling only: every step of the forward runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  If the
+shared library is missing this module raises at import; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbsa.so")
+
+BSA_OK = 0
+BSA_ERR_INVALID_ARG = -1
+BSA_ERR_UNSUPPORTED = -2
+BSA_ERR_CUDA = -3
+BSA_ERR_LAYOUT_MISMATCH = -4
+BSA_ERR_DEVICE_TIMEOUT = -5
+BSA_ERR_OOM = -6
+BSA_ERR_WORKSPACE = -7
+
+# name -> (restype, argtypes); mirrors include/bsa.h
+_SIGNATURES = {
+    "bsa_layout_build": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
+                                        ctypes.POINTER(ctypes.c_int32),
+                                        ctypes.POINTER(ctypes.c_void_p)]),
+    "bsa_layout_csr": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p),
+                                      ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int64),
+                                      ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+    "bsa_layout_globals": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p),
+                                          ctypes.POINTER(ctypes.c_int)]),
+    "bsa_layout_tiles": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p),
+                                        ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_void_p),
+                                        ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int64)]),
+    "bsa_layout_upload": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "bsa_layout_free": (None, [ctypes.c_void_p]),
+    "bsa_workspace_bytes": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_size_t)]),
+    "bsa_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "bsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "bsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "bsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p]),
+}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing; build it with "
+                          "`python -m block_sparse_attention_bigbird_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+LIB_PATH = _LIB_PATH
+
+
+class BsaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {bsa_strerror(code)} ({code})")
+        self.code = code
+
+
+def bsa_strerror(code: int) -> str:
+    return lib.bsa_strerror(int(code)).decode()
+
+
+def _check(code: int, what: str) -> None:
+    if code != BSA_OK:
+        raise BsaError(code, what)
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class Layout:
+    """Owner of a bsa_layout*; freed with the object."""
+
+    def __init__(self, handle: int, H: int, L: int):
+        self._h = ctypes.c_void_p(handle)
+        self.H = H
+        self.L = L
+        self._workspaces = {}
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        return self._h
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib.bsa_layout_free(h)
+            self._h = ctypes.c_void_p(0)
+
+
+def bsa_layout_build(H: int, L: int, block: int = 64, window: int = 1, n_global: int = 2,
+                     n_random: int = 3, seed: int = 0, globals=None) -> Layout:
+    out = ctypes.c_void_p()
+    gptr = None
+    if globals is not None:
+        g = np.ascontiguousarray(np.asarray(globals, dtype=np.int32))
+        n_global = int(g.size)
+        gptr = g.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    _check(lib.bsa_layout_build(H, L, block, window, n_global, n_random,
+                                ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), gptr, ctypes.byref(out)),
+           "bsa_layout_build")
+    return Layout(out.value, H, L)
+
+
+def bsa_layout_csr(layout: Layout):
+    """(row_ptr int32 [H*nb+1], col_idx int32 [nnz]) as numpy copies."""
+    rp, ci = ctypes.c_void_p(), ctypes.c_void_p()
+    nnz, nb, H = ctypes.c_int64(), ctypes.c_int(), ctypes.c_int()
+    _check(lib.bsa_layout_csr(layout.handle, ctypes.byref(rp), ctypes.byref(ci), ctypes.byref(nnz),
+                              ctypes.byref(nb), ctypes.byref(H)), "bsa_layout_csr")
+    n_rows = H.value * nb.value + 1
+    row_ptr = np.ctypeslib.as_array(ctypes.cast(rp, ctypes.POINTER(ctypes.c_int32)), (n_rows,)).copy()
+    col_idx = (np.ctypeslib.as_array(ctypes.cast(ci, ctypes.POINTER(ctypes.c_int32)), (nnz.value,)).copy()
+               if nnz.value else np.zeros(0, np.int32))
+    return row_ptr, col_idx
+
+
+def bsa_layout_globals(layout: Layout) -> np.ndarray:
+    gp, n = ctypes.c_void_p(), ctypes.c_int()
+    _check(lib.bsa_layout_globals(layout.handle, ctypes.byref(gp), ctypes.byref(n)), "bsa_layout_globals")
+    if n.value == 0:
+        return np.zeros(0, np.int32)
+    return np.ctypeslib.as_array(ctypes.cast(gp, ctypes.POINTER(ctypes.c_int32)), (n.value,)).copy()
+
+
+def bsa_layout_tiles(layout: Layout):
+    """(pair_q [n_pairs, 2], pair_ptr [H*n_pairs+1], pair_ent [n_ent] uint32) as numpy copies."""
+    pq, pp, pe = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+    n_pairs, n_ent = ctypes.c_int(), ctypes.c_int64()
+    _check(lib.bsa_layout_tiles(layout.handle, ctypes.byref(pq), ctypes.byref(n_pairs), ctypes.byref(pp),
+                                ctypes.byref(pe), ctypes.byref(n_ent)), "bsa_layout_tiles")
+    P = n_pairs.value
+    pair_q = np.ctypeslib.as_array(ctypes.cast(pq, ctypes.POINTER(ctypes.c_int32)), (2 * P,)).copy()
+    pair_ptr = np.ctypeslib.as_array(ctypes.cast(pp, ctypes.POINTER(ctypes.c_int32)),
+                                     (layout.H * P + 1,)).copy()
+    pair_ent = np.ctypeslib.as_array(ctypes.cast(pe, ctypes.POINTER(ctypes.c_uint32)), (n_ent.value,)).copy()
+    return pair_q.reshape(P, 2), pair_ptr, pair_ent
+
+
+def bsa_layout_upload(layout: Layout, stream=None) -> None:
+    _check(lib.bsa_layout_upload(layout.handle, ctypes.c_void_p(_stream_ptr(stream))), "bsa_layout_upload")
+    layout._workspaces.clear()
+
+
+def bsa_workspace_bytes(layout: Layout, B: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib.bsa_workspace_bytes(layout.handle, B, ctypes.byref(n)), "bsa_workspace_bytes")
+    return n.value
+
+
+def _workspace(layout: Layout, B: int, device):
+    import torch
+    key = (str(device), B)
+    ws = layout._workspaces.get(key)
+    if ws is None:
+        ws = torch.zeros(bsa_workspace_bytes(layout, B), dtype=torch.uint8, device=device)
+        layout._workspaces[key] = ws
+    return ws
+
+
+def bsa_forward(q, k, v, layout: Layout, key_mask=None, scale: Optional[float] = None, out=None,
+                lse=None, workspace=None, stream=None):
+    """O (bf16 [B,H,L,64]) and lse (fp32 [B,H,L]) of the block-sparse attention.
+
+    q, k, v: contiguous bf16 CUDA tensors [B, H, L, 64].  key_mask: optional
+    uint8 CUDA tensor [B, L] (1 = keep).  workspace: optional zero-initialised
+    uint8 CUDA tensor of at least bsa_workspace_bytes(layout, B) bytes; when
+    omitted a cached one of the layout is used (not safe for concurrent calls
+    on different streams with the same layout).
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [B, H, L, d]")
+    if q.shape != k.shape or q.shape != v.shape:
+        raise ValueError("q, k, v shapes differ")
+    B, H, L, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    if key_mask is not None:
+        if key_mask.dtype != torch.uint8 or tuple(key_mask.shape) != (B, L) or not key_mask.is_contiguous():
+            raise ValueError("key_mask must be a contiguous uint8 tensor [B, L]")
+    if workspace is None:
+        workspace = _workspace(layout, B, q.device)
+    code = lib.bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L, d, layout.handle,
+                           key_mask.data_ptr() if key_mask is not None else None,
+                           ctypes.c_float(scale if scale is not None else 0.0), out.data_ptr(),
+                           lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                           ctypes.c_void_p(_stream_ptr(stream)))
+    _check(code, "bsa_forward")
+    return out, lse
+
+
+def bsa_sync_status(stream=None) -> int:
+    """Synchronises the stream; returns (and clears) the device status word."""
+    return lib.bsa_sync_status(ctypes.c_void_p(_stream_ptr(stream)))
+
+
+def bsa_debug_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check(lib.bsa_debug_wait_timeout(ctypes.c_uint64(timeout_ns), ctypes.c_void_p(_stream_ptr(stream))),
+           "bsa_debug_wait_timeout")
+
+
+def header_symbols() -> list[str]:
+    """Function names declared in include/bsa.h (parsed from the header text)."""
+    import re
+    hdr = os.path.join(os.path.dirname(os.path.dirname(_LIB_PATH)), "include", "bsa.h")
+    with open(hdr) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:int|void|const char\*)\s+(bsa_\w+)\s*\(", text, re.M)))

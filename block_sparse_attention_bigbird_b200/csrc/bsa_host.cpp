@@ -1,0 +1,378 @@
+// Host side of the BigBird block-sparse attention library: the seeded layout
+// builder, the 128-row tile decomposition and the static work list.  Pure C++,
+// no GPU needed.  Every entry point validates its arguments and returns a
+// bsa_status; no exception crosses the C ABI.
+#include <algorithm>
+#include <cstring>
+#include <new>
+
+#include "bsa_internal.h"
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Philox4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy
+// as 1, 2, 3", SC'11): a counter-based generator.  Each of the ten rounds
+// multiplies counter words 0 and 2 by two fixed 64-bit constants, swaps the
+// halves across the words and xors in the round key; the key is bumped by two
+// Weyl constants (golden ratio and sqrt(3)-1 in 64-bit fixed point) between
+// rounds.  The stream here follows the convention of numpy's Philox bit
+// generator: the 256-bit counter is incremented BEFORE each 4-word block is
+// produced and the words of a block are handed out in order 0..3.
+// ---------------------------------------------------------------------------
+constexpr uint64_t kPhiloxM0 = 0xD2E7470EE14C6C93ull;
+constexpr uint64_t kPhiloxM1 = 0xCA5A826395121157ull;
+constexpr uint64_t kPhiloxW0 = 0x9E3779B97F4A7C15ull;
+constexpr uint64_t kPhiloxW1 = 0xBB67AE8584CAA73Bull;
+
+inline void mulhilo64(uint64_t a, uint64_t b, uint64_t* hi, uint64_t* lo) {
+  unsigned __int128 p = static_cast<unsigned __int128>(a) * b;
+  *hi = static_cast<uint64_t>(p >> 64);
+  *lo = static_cast<uint64_t>(p);
+}
+
+void philox4x64_10(const uint64_t in[4], const uint64_t key_in[2], uint64_t out[4]) {
+  uint64_t c0 = in[0], c1 = in[1], c2 = in[2], c3 = in[3];
+  uint64_t k0 = key_in[0], k1 = key_in[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += kPhiloxW0;
+      k1 += kPhiloxW1;
+    }
+    uint64_t hi0, lo0, hi1, lo1;
+    mulhilo64(kPhiloxM0, c0, &hi0, &lo0);
+    mulhilo64(kPhiloxM1, c2, &hi1, &lo1);
+    const uint64_t n0 = hi1 ^ c1 ^ k0;
+    const uint64_t n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  out[0] = c0;
+  out[1] = c1;
+  out[2] = c2;
+  out[3] = c3;
+}
+
+class PhiloxStream {
+ public:
+  PhiloxStream(uint64_t seed, uint64_t i, uint64_t h) {
+    ctr_[0] = 0;
+    ctr_[1] = i;
+    ctr_[2] = h;
+    ctr_[3] = 0;
+    key_[0] = seed;
+    key_[1] = 0;
+  }
+  uint64_t next() {
+    if (pos_ == 4) {
+      for (int w = 0; w < 4; ++w) {  // 256-bit little-endian increment
+        if (++ctr_[w] != 0) break;
+      }
+      philox4x64_10(ctr_, key_, buf_);
+      pos_ = 0;
+    }
+    return buf_[pos_++];
+  }
+
+ private:
+  uint64_t ctr_[4];
+  uint64_t key_[2];
+  uint64_t buf_[4] = {0, 0, 0, 0};
+  int pos_ = 4;
+};
+
+// k-th (0-based) block of [0, nb) that is not in the sorted list `excl`.
+inline int kth_free(int k, const std::vector<int>& excl) {
+  int v = k;
+  for (int e : excl) {
+    if (e <= v)
+      ++v;
+    else
+      break;
+  }
+  return v;
+}
+
+// One row of the layout (BigBird: window + globals + random, see bsa.h).
+void build_row(int h, int i, int nb, int window, const std::vector<int32_t>& globals,
+               const std::vector<uint8_t>& is_global, int n_random, uint64_t seed,
+               std::vector<int32_t>* row) {
+  row->clear();
+  if (is_global[i]) {
+    for (int j = 0; j < nb; ++j) row->push_back(j);
+    return;
+  }
+  const int lo = std::max(0, i - window);
+  const int hi = std::min(nb - 1, i + window);
+  // excluded = window U globals, sorted and distinct
+  std::vector<int> excl;
+  excl.reserve(static_cast<size_t>(hi - lo + 1) + globals.size());
+  for (int j = lo; j <= hi; ++j) excl.push_back(j);
+  for (int g : globals)
+    if (g < lo || g > hi) excl.push_back(g);
+  std::sort(excl.begin(), excl.end());
+  const int m = nb - static_cast<int>(excl.size());
+  const int take = std::min(n_random, m);
+  // Partial Fisher-Yates over the ascending candidate list C (implicit: C[k] =
+  // kth_free(k)), touching only the positions the shuffle swaps.
+  std::vector<std::pair<int, int>> swapped;  // position -> candidate index
+  auto get = [&](int pos) {
+    for (const auto& s : swapped)
+      if (s.first == pos) return s.second;
+    return pos;
+  };
+  auto set = [&](int pos, int val) {
+    for (auto& s : swapped)
+      if (s.first == pos) {
+        s.second = val;
+        return;
+      }
+    swapped.emplace_back(pos, val);
+  };
+  std::vector<int> rnd;
+  rnd.reserve(static_cast<size_t>(take));
+  PhiloxStream rng(seed, static_cast<uint64_t>(i), static_cast<uint64_t>(h));
+  for (int t = 0; t < take; ++t) {
+    const uint64_t u = rng.next();
+    const int j = t + static_cast<int>(u % static_cast<uint64_t>(m - t));
+    const int ct = get(t), cj = get(j);
+    set(t, cj);
+    set(j, ct);
+    rnd.push_back(kth_free(cj, excl));
+  }
+  row->insert(row->end(), excl.begin(), excl.end());
+  row->insert(row->end(), rnd.begin(), rnd.end());
+  std::sort(row->begin(), row->end());
+}
+
+}  // namespace
+
+namespace bsa {
+
+WorkspacePlan plan_workspace(const bsa_layout& lay, int B) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  WorkspacePlan p{};
+  p.tickets_off = 0;
+  p.tickets_bytes = up(std::max<size_t>(4, sizeof(int32_t) * static_cast<size_t>(B) * lay.n_split));
+  p.keybits_off = p.tickets_off + p.tickets_bytes;
+  p.keybits_bytes = up(sizeof(uint64_t) * static_cast<size_t>(B) * lay.nb);
+  p.partials_off = p.keybits_off + p.keybits_bytes;
+  p.partials_bytes =
+      up(sizeof(float) * static_cast<size_t>(kRecFloats) * static_cast<size_t>(B) * lay.n_records);
+  p.total = p.partials_off + p.partials_bytes;
+  return p;
+}
+
+}  // namespace bsa
+
+namespace {
+
+void build_tiles(bsa_layout* lay) {
+  const int nb = lay->nb, H = lay->H;
+  std::vector<uint8_t> is_global(static_cast<size_t>(nb), 0);
+  for (int g : lay->globals) is_global[static_cast<size_t>(g)] = 1;
+  // Pairs: global blocks with global blocks, the others with the others, in
+  // ascending order; an odd one out forms a single-block tile.
+  std::vector<int32_t> gl, ng;
+  for (int i = 0; i < nb; ++i) (is_global[static_cast<size_t>(i)] ? gl : ng).push_back(i);
+  lay->pair_q.clear();
+  for (const auto* lst : {&gl, &ng}) {
+    for (size_t x = 0; x < lst->size(); x += 2) {
+      lay->pair_q.push_back((*lst)[x]);
+      lay->pair_q.push_back(x + 1 < lst->size() ? (*lst)[x + 1] : -1);
+    }
+  }
+  lay->n_pairs = static_cast<int>(lay->pair_q.size() / 2);
+  const int P = lay->n_pairs;
+  lay->pair_ptr.assign(1, 0);
+  lay->pair_ent.clear();
+  for (int h = 0; h < H; ++h) {
+    for (int p = 0; p < P; ++p) {
+      const int qa = lay->pair_q[2 * p], qb = lay->pair_q[2 * p + 1];
+      const int32_t* ra = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qa];
+      const int32_t* ra_end = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qa + 1];
+      const int32_t* rb = ra_end;
+      const int32_t* rb_end = ra_end;
+      if (qb >= 0) {
+        rb = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qb];
+        rb_end = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qb + 1];
+      }
+      while (ra != ra_end || rb != rb_end) {
+        uint32_t col, bits;
+        if (rb == rb_end || (ra != ra_end && *ra < *rb)) {
+          col = static_cast<uint32_t>(*ra++);
+          bits = 1;
+        } else if (ra == ra_end || *rb < *ra) {
+          col = static_cast<uint32_t>(*rb++);
+          bits = 2;
+        } else {
+          col = static_cast<uint32_t>(*ra++);
+          ++rb;
+          bits = 3;
+        }
+        lay->pair_ent.push_back(col | (bits << bsa::kEntBitsShift));
+      }
+      lay->pair_ptr.push_back(static_cast<int32_t>(lay->pair_ent.size()));
+    }
+  }
+  // Static schedule for one batch element, head-major so that consecutive
+  // items (run concurrently by consecutive CTAs) share the head's K/V in L2.
+  lay->items.clear();
+  lay->n_split = 0;
+  lay->n_records = 0;
+  for (int h = 0; h < H; ++h) {
+    for (int p = 0; p < P; ++p) {
+      const int32_t s = lay->pair_ptr[static_cast<size_t>(h) * P + p];
+      const int32_t U = lay->pair_ptr[static_cast<size_t>(h) * P + p + 1] - s;
+      if (U <= bsa::kSplitThreshold) {
+        lay->items.push_back(bsa::WorkItem{h, p, s, U, -1, 0, 1, 0});
+        continue;
+      }
+      const int nch = (U + bsa::kSplitChunk - 1) / bsa::kSplitChunk;
+      const int slot = lay->n_split++;
+      const int base = lay->n_records;
+      lay->n_records += nch;
+      for (int c = 0; c < nch; ++c) {
+        const int cs = c * bsa::kSplitChunk;
+        lay->items.push_back(bsa::WorkItem{h, p, s + cs, std::min(bsa::kSplitChunk, U - cs),
+                                           slot, base + c, nch, base});
+      }
+    }
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_random,
+                     uint64_t seed, const int32_t* globals, bsa_layout** out) {
+  if (out == nullptr) return BSA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (block != bsa::kBlock) return BSA_ERR_UNSUPPORTED;
+  if (H < 1 || L < 1 || L % block != 0 || window < 0 || n_global < 0 || n_random < 0)
+    return BSA_ERR_INVALID_ARG;
+  const int nb = L / block;
+  if (nb > static_cast<int>(bsa::kEntColMask) || static_cast<int64_t>(H) * nb > (1 << 30))
+    return BSA_ERR_INVALID_ARG;
+  bsa_layout* lay = new (std::nothrow) bsa_layout();
+  if (lay == nullptr) return BSA_ERR_OOM;
+  try {
+    lay->H = H;
+    lay->L = L;
+    lay->block = block;
+    lay->nb = nb;
+    lay->window = window;
+    lay->n_global = n_global;
+    lay->n_random = n_random;
+    lay->seed = seed;
+    // globals
+    std::vector<int32_t> g;
+    if (globals != nullptr) {
+      for (int x = 0; x < n_global; ++x) {
+        if (globals[x] < 0 || globals[x] >= nb) {
+          delete lay;
+          return BSA_ERR_INVALID_ARG;
+        }
+        g.push_back(globals[x]);
+      }
+    } else if (n_global == 1) {
+      g.push_back(0);
+    } else if (n_global >= 2) {
+      for (int k = 0; k < n_global; ++k)
+        g.push_back(static_cast<int32_t>((static_cast<int64_t>(k) * (nb - 1)) / (n_global - 1)));
+    }
+    std::sort(g.begin(), g.end());
+    g.erase(std::unique(g.begin(), g.end()), g.end());
+    lay->globals = g;
+    std::vector<uint8_t> is_global(static_cast<size_t>(nb), 0);
+    for (int x : g) is_global[static_cast<size_t>(x)] = 1;
+    // CSR rows, head-major
+    lay->row_ptr.reserve(static_cast<size_t>(H) * nb + 1);
+    lay->row_ptr.push_back(0);
+    std::vector<int32_t> row;
+    for (int h = 0; h < H; ++h) {
+      for (int i = 0; i < nb; ++i) {
+        build_row(h, i, nb, window, g, is_global, n_random, seed, &row);
+        lay->col_idx.insert(lay->col_idx.end(), row.begin(), row.end());
+        if (lay->col_idx.size() > static_cast<size_t>(INT32_MAX)) {
+          delete lay;
+          return BSA_ERR_INVALID_ARG;
+        }
+        lay->row_ptr.push_back(static_cast<int32_t>(lay->col_idx.size()));
+      }
+    }
+    build_tiles(lay);
+    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
+      delete lay;
+      return BSA_ERR_INVALID_ARG;
+    }
+  } catch (const std::bad_alloc&) {
+    delete lay;
+    return BSA_ERR_OOM;
+  } catch (...) {
+    delete lay;
+    return BSA_ERR_INVALID_ARG;
+  }
+  *out = lay;
+  return BSA_OK;
+}
+
+int bsa_layout_csr(const bsa_layout* lay, const int32_t** row_ptr, const int32_t** col_idx,
+                   int64_t* nnz, int* nb, int* H) {
+  if (lay == nullptr) return BSA_ERR_INVALID_ARG;
+  if (row_ptr) *row_ptr = lay->row_ptr.data();
+  if (col_idx) *col_idx = lay->col_idx.data();
+  if (nnz) *nnz = static_cast<int64_t>(lay->col_idx.size());
+  if (nb) *nb = lay->nb;
+  if (H) *H = lay->H;
+  return BSA_OK;
+}
+
+int bsa_layout_globals(const bsa_layout* lay, const int32_t** globals, int* n_global) {
+  if (lay == nullptr) return BSA_ERR_INVALID_ARG;
+  if (globals) *globals = lay->globals.data();
+  if (n_global) *n_global = static_cast<int>(lay->globals.size());
+  return BSA_OK;
+}
+
+int bsa_layout_tiles(const bsa_layout* lay, const int32_t** pair_q, int* n_pairs,
+                     const int32_t** pair_ptr, const uint32_t** pair_ent, int64_t* n_ent) {
+  if (lay == nullptr) return BSA_ERR_INVALID_ARG;
+  if (pair_q) *pair_q = lay->pair_q.data();
+  if (n_pairs) *n_pairs = lay->n_pairs;
+  if (pair_ptr) *pair_ptr = lay->pair_ptr.data();
+  if (pair_ent) *pair_ent = lay->pair_ent.data();
+  if (n_ent) *n_ent = static_cast<int64_t>(lay->pair_ent.size());
+  return BSA_OK;
+}
+
+void bsa_layout_free(bsa_layout* lay) {
+  if (lay == nullptr) return;
+  bsa::free_device(lay);
+  delete lay;
+}
+
+int bsa_workspace_bytes(const bsa_layout* lay, int B, size_t* bytes) {
+  if (lay == nullptr || bytes == nullptr || B < 1) return BSA_ERR_INVALID_ARG;
+  *bytes = bsa::plan_workspace(*lay, B).total;
+  return BSA_OK;
+}
+
+const char* bsa_strerror(int status) {
+  switch (status) {
+    case BSA_OK: return "success";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported configuration (block and head dim must be 64, device must be sm_100)";
+    case BSA_ERR_CUDA: return "CUDA call failed";
+    case BSA_ERR_LAYOUT_MISMATCH: return "layout does not match H/L or is not uploaded to the current device";
+    case BSA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    case BSA_ERR_OOM: return "out of memory";
+    case BSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

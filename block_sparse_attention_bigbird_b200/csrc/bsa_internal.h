@@ -1,0 +1,79 @@
+// Internal structures shared by the host library (bsa_host.cpp) and the CUDA
+// forward (bsa_fwd_sm100.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "../../include/bsa.h"
+
+namespace bsa {
+
+// Tile geometry.  A tile is 128 query rows = two 64-row query blocks that run
+// over the sorted union of their key-block lists (tcgen05's M = 128 datapath).
+constexpr int kBlock = 64;
+constexpr int kHeadDim = 64;
+constexpr int kTileRows = 128;
+
+// A tile whose key-block union is longer than kSplitThreshold is cut into
+// chunks of kSplitChunk union entries (even, so only a tile's last chunk can
+// hold a single key block).  Each chunk writes a partial (O, m, l) record; the
+// last chunk to finish merges them.
+constexpr int kSplitThreshold = 48;
+constexpr int kSplitChunk = 32;
+
+// Partial record of one split chunk: O[128][64] fp32 (unnormalised, relative to
+// the chunk's running max), then m[128] (log2 units, scaled) and l[128].
+constexpr int kRecFloats = kTileRows * kHeadDim + 2 * kTileRows;
+
+// One unit of the static schedule (32 bytes, read with two 16-byte loads).
+struct WorkItem {
+  int32_t h;         // head
+  int32_t pair;      // tile (query-block pair) index within the head
+  int32_t start;     // first entry in pair_ent (absolute index)
+  int32_t count;     // number of union entries processed by this item (>= 1)
+  int32_t split;     // -1: whole tile; otherwise split-tile slot within a batch element
+  int32_t rec;       // partial record index within a batch element (split only)
+  int32_t nchunks;   // number of chunks of the split tile
+  int32_t rec_base;  // first record of the split tile within a batch element
+};
+static_assert(sizeof(WorkItem) == 32, "WorkItem must stay 32 bytes");
+
+constexpr uint32_t kEntColMask = 0x00FFFFFFu;
+constexpr int kEntBitsShift = 24;
+
+}  // namespace bsa
+
+struct bsa_layout {
+  int H = 0, L = 0, block = 0, nb = 0;
+  int window = 0, n_global = 0, n_random = 0;
+  uint64_t seed = 0;
+  std::vector<int32_t> globals;     // sorted, distinct
+  std::vector<int32_t> row_ptr;     // H*nb + 1
+  std::vector<int32_t> col_idx;     // nnz
+  std::vector<int32_t> pair_q;      // 2 * n_pairs
+  int n_pairs = 0;
+  std::vector<int32_t> pair_ptr;    // H*n_pairs + 1
+  std::vector<uint32_t> pair_ent;   // union entries
+  std::vector<bsa::WorkItem> items; // schedule for ONE batch element (head-major)
+  int n_split = 0;                  // split tiles per batch element
+  int n_records = 0;                // partial records per batch element
+  // device copies (bsa_layout_upload)
+  int device = -1;
+  int32_t* d_pair_q = nullptr;
+  uint32_t* d_pair_ent = nullptr;
+  bsa::WorkItem* d_items = nullptr;
+};
+
+namespace bsa {
+// Workspace carve-up for batch size B (all offsets 256-byte aligned).
+struct WorkspacePlan {
+  size_t tickets_off, tickets_bytes;
+  size_t keybits_off, keybits_bytes;
+  size_t partials_off, partials_bytes;
+  size_t total;
+};
+WorkspacePlan plan_workspace(const bsa_layout& lay, int B);
+void free_device(bsa_layout* lay);
+}  // namespace bsa

@@ -1,0 +1,181 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) BigBird block-sparse attention forward.
+ *
+ * What is computed (forward pass only), for every batch element b, head h and
+ * query token t of query block i = t / 64:
+ *
+ *     O[b,h,t,:] = softmax_{p in A(h,i)} ( q_t . k_p * scale ) . V[b,h,p,:]
+ *     lse[b,h,t] = ln sum_{p in A(h,i)} exp( q_t . k_p * scale )
+ *
+ * where A(h,i) is the union of the key tokens of the key blocks listed in
+ * row (h, i) of the layout, minus the keys the optional key-padding mask drops.
+ * This is the masked attention Softmax(Q K^T / sqrt(d_k) (.) M) V of
+ * "Adapt or Perish: 新手入门指南 – Adaptive Sparse Transformer 核心原理与实战"
+ * (section on the sparse-attention formula), with (.) M read as restricting
+ * the softmax to M -- the pages' own code fills the excluded scores with
+ * -1e9 / -1e10 ("BERT 稀疏注意力机制入门指南", PyTorch 实现; "BERT多头注意力机制深度解析",
+ * BlockSparseAttention).  A single softmax runs over the union of the three
+ * BigBird patterns ("BigBird 稀疏注意力机制解析", 核心实现): global, sliding
+ * window, random.  The mask is stored at 64x64 block granularity
+ * ("Transformer计算效率优化：SQA稀疏注意力机制详解", 3.1 and 5 问题3).
+ *
+ * Conventions for every entry point:
+ *   - Return value: BSA_OK (0) or a negative bsa_status.  No C++ exception
+ *     crosses this boundary.  Arguments are validated before anything is
+ *     launched; a failing call has no effect on the GPU.
+ *   - "device" pointers are CUDA device pointers of the current device;
+ *     "host" pointers are ordinary CPU memory.  The caller owns every buffer it
+ *     passes in; the library owns the bsa_layout object and its device copies.
+ *   - A stream argument is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  GPU work is enqueued asynchronously on it.
+ *   - Thread safety: distinct layouts may be used concurrently; one layout may
+ *     be shared by concurrent bsa_forward calls once uploaded (it is read-only
+ *     then), each call with its own workspace.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = -1,     /* null pointer, bad size or range            */
+  BSA_ERR_UNSUPPORTED = -2,     /* block != 64, d != 64, not an sm_100 device  */
+  BSA_ERR_CUDA = -3,            /* a CUDA runtime/driver call failed           */
+  BSA_ERR_LAYOUT_MISMATCH = -4, /* layout built for another H/L, or not uploaded
+                                   to the current device                       */
+  BSA_ERR_DEVICE_TIMEOUT = -5,  /* a bounded wait inside a kernel gave up      */
+  BSA_ERR_OOM = -6,             /* host or device allocation failed            */
+  BSA_ERR_WORKSPACE = -7        /* workspace missing or too small              */
+} bsa_status;
+
+/* Opaque, immutable after bsa_layout_build (bsa_layout_upload only adds
+ * device copies).  Owned by the library; release with bsa_layout_free. */
+typedef struct bsa_layout bsa_layout;
+
+/*
+ * bsa_layout_build -- host only, no GPU needed.
+ *
+ * Builds the BigBird block layout for H heads and sequence length L with
+ * nb = L / block query/key blocks ("BigBird 稀疏注意力机制解析", 核心实现 and
+ * 代码实现; window clipping from "BERT 稀疏注意力机制入门指南", PyTorch 实现):
+ *   globals  G: if `globals` is non-NULL it holds n_global block indices (any
+ *            order, duplicates allowed, each in [0, nb)); otherwise
+ *            n_global == 0 -> {}, 1 -> {0}, else floor(k (nb-1)/(n_global-1)),
+ *            k = 0..n_global-1, deduplicated (torch.linspace(...).long() of the
+ *            page, in exact integers).
+ *   row (h,i) for i in G: every block 0..nb-1.
+ *   row (h,i) otherwise: window {j : |i-j| <= window, 0 <= j < nb} union G union
+ *            R(h,i), where R(h,i) is min(n_random, m) distinct blocks drawn from
+ *            the m blocks outside window and G by a partial Fisher-Yates
+ *            shuffle (ascending candidate list; step t swaps entries t and
+ *            t + u_t mod (m - t)) driven by the raw 64-bit outputs u_0, u_1, ...
+ *            of Philox4x64-10 with key {seed, 0} and counter {0, i, h, 0},
+ *            incremented (as a 256-bit little-endian integer) before each
+ *            4-word block is produced.
+ *   Rows are sorted ascending and duplicate-free; the layout is shared by all
+ *   batch elements.  CSR rows are ordered head-major then query block.
+ *
+ * block must be 64 (else BSA_ERR_UNSUPPORTED); L > 0 and L % block == 0;
+ * H >= 1; window, n_global, n_random >= 0 (else BSA_ERR_INVALID_ARG).
+ * On success *out receives a new layout.
+ */
+int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_random,
+                     uint64_t seed, const int32_t* globals, bsa_layout** out);
+
+/*
+ * bsa_layout_csr -- host views of the CSR: row_ptr has H*nb+1 int32 entries,
+ * col_idx has nnz int32 entries (key block indices).  Any output pointer may be
+ * NULL.  The views stay valid until bsa_layout_free.
+ */
+int bsa_layout_csr(const bsa_layout* layout, const int32_t** row_ptr,
+                   const int32_t** col_idx, int64_t* nnz, int* nb, int* H);
+
+/* bsa_layout_globals -- host view of the sorted global block list. */
+int bsa_layout_globals(const bsa_layout* layout, const int32_t** globals, int* n_global);
+
+/*
+ * bsa_layout_tiles -- host views of the 128-row tile decomposition the kernel
+ * runs (two query blocks per tile over the union of their rows).
+ *   pair_q:   2*n_pairs int32, (first, second) query block; second = -1 when the
+ *             tile holds a single block.  Global blocks pair with global blocks.
+ *   pair_ptr: H*n_pairs+1 int32 offsets into pair_ent, head-major.
+ *   pair_ent: key block | (membership << 24): bit 0 = in the first block's row,
+ *             bit 1 = in the second's.
+ * Any output may be NULL.
+ */
+int bsa_layout_tiles(const bsa_layout* layout, const int32_t** pair_q, int* n_pairs,
+                     const int32_t** pair_ptr, const uint32_t** pair_ent, int64_t* n_ent);
+
+/*
+ * bsa_layout_upload -- copies the tile tables and work list to the CURRENT
+ * device (cudaMemcpyAsync on `stream`, then a stream synchronize).  Must
+ * precede bsa_forward on that device.  Calling it again re-uploads to the
+ * then-current device.  Returns BSA_ERR_OOM / BSA_ERR_CUDA on failure.
+ */
+int bsa_layout_upload(bsa_layout* layout, void* stream);
+
+/* bsa_layout_free -- releases host and device memory of the layout; NULL is a no-op. */
+void bsa_layout_free(bsa_layout* layout);
+
+/*
+ * bsa_workspace_bytes -- device scratch bytes bsa_forward needs for batch size
+ * B: split-row partial results, their arrival tickets and the per-key-block
+ * padding bits.  The workspace must be ZERO-FILLED before its first use; every
+ * call that completes without a device error leaves the ticket area zero again,
+ * so it can be reused without clearing.  After a call that ended in a device
+ * error, clear it again.
+ */
+int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
+
+/*
+ * bsa_forward -- enqueues the block-sparse attention forward on `stream`.
+ *   q, k, v   device, bf16, [B, H, L, d] contiguous, 16-byte aligned.
+ *   d         must be 64 (else BSA_ERR_UNSUPPORTED).
+ *   layout    built for this H and L and uploaded to the current device.
+ *   key_mask  device uint8 [B, L] (1 = keep, 0 = drop the key), or NULL.
+ *   scale     softmax scale applied to q.k; <= 0 selects 1/sqrt(d).
+ *   out       device, bf16, [B, H, L, d] contiguous (round-to-nearest-even).
+ *   lse       device, fp32, [B, H, L]: natural-log sum of exp of the scaled
+ *             scores over the attended keys; -inf (with O = 0) for a row whose
+ *             attended set is empty.
+ *   workspace device, at least bsa_workspace_bytes(layout, B) bytes, 256-byte
+ *             aligned, zero-filled before first use (see above).
+ * Returns after enqueueing (no synchronisation, no allocation).  A device-side
+ * timeout is reported later by bsa_sync_status.
+ */
+int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L, int d,
+                const bsa_layout* layout, const uint8_t* key_mask, float scale,
+                void* out, float* lse, void* workspace, size_t workspace_bytes,
+                void* stream);
+
+/*
+ * bsa_sync_status -- synchronises `stream`, then returns and clears the
+ * device-side status word of the current device: BSA_OK, or
+ * BSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait gave up (its outputs are
+ * then undefined).  BSA_ERR_CUDA if the synchronisation itself failed.
+ */
+int bsa_sync_status(void* stream);
+
+/* bsa_strerror -- static description of a status code. */
+const char* bsa_strerror(int status);
+
+/*
+ * bsa_debug_wait_timeout -- test hook for the bounded-wait machinery: launches
+ * one CTA that waits on a shared-memory barrier nothing ever completes, with a
+ * limit of `timeout_ns` nanoseconds (clamped to [1e3, 2e9]).  The kernel gives
+ * up, records BSA_ERR_DEVICE_TIMEOUT in the status word and returns; the
+ * context stays usable.  Read the result with bsa_sync_status.
+ */
+int bsa_debug_wait_timeout(uint64_t timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -16,3 +16,10 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_sessionstart(session):
+    # Build libbsa.so in-tree when missing or older than its sources (needs nvcc).
+    from block_sparse_attention_bigbird_b200 import build as _build
+    if _build.is_stale():
+        _build.build()
