@@ -107,7 +107,7 @@ class Layout:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
+        if h is not None and h.value and lib is not None:   # lib is None at interpreter exit
             lib.bsa_layout_free(h)
             self._h = ctypes.c_void_p(0)
 

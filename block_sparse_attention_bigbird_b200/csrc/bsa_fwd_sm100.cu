@@ -67,7 +67,8 @@ enum : int {
   kBarPFull = kBarSFull + 2,
   kBarODone = kBarPFull + 2,
   kBarMmaFinal = kBarODone + 1,
-  kNumBars = kBarMmaFinal + 1
+  kBarEpi = kBarMmaFinal + 1,  // 128 softmax threads, split-chunk epilogue
+  kNumBars = kBarEpi + 1
 };
 constexpr uint32_t kSmemMisc = kSmemBar + 8 * kNumBars;
 constexpr uint32_t kSmemUsed = kSmemMisc + 16;
@@ -313,7 +314,16 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
   const int total = p.B * p.items_per_batch;
   const float sl2 = p.scale_log2;
   uint32_t g = 0;
+  uint32_t n_epi = 0;  // uses of the epilogue barrier
   bool alive = true;
+  // Bounded 128-thread rendezvous (a plain bar.sync could not give up if another
+  // softmax warp had already aborted).
+  auto epi_sync = [&]() -> bool {
+    ptx::mbar_arrive(bar(kBarEpi));
+    const bool ok = wait_warp(bar(kBarEpi), n_epi & 1u, abort_flag, p.timeout_ns);
+    ++n_epi;
+    return ok;
+  };
   for (int t = blockIdx.x; alive && t < total; t += gridDim.x) {
     const int b = t / p.items_per_batch;
     const WorkItem w = p.items[t - b * p.items_per_batch];
@@ -466,10 +476,16 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
       rec[kTileRows * 64 + r] = m_run;
       rec[kTileRows * 64 + kTileRows + r] = l_run;
       __threadfence();
-      ptx::named_bar_sync(1, 128);
+      if (!epi_sync()) {
+        alive = false;
+        break;
+      }
       int* ticket = p.tickets + static_cast<size_t>(b) * p.n_split + w.split;
       if (r == 0) *last_flag = (atomicAdd(ticket, 1) == w.nchunks - 1) ? 1u : 0u;
-      ptx::named_bar_sync(1, 128);
+      if (!epi_sync()) {
+        alive = false;
+        break;
+      }
       if (*last_flag) {
         __threadfence();
         if (row_active) {
@@ -531,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i)
-      ptx::mbar_init(bars + 8u * i, (i == kBarPFull || i == kBarPFull + 1) ? 128u : 1u);
+      ptx::mbar_init(bars + 8u * i, (i == kBarPFull || i == kBarPFull + 1 || i == kBarEpi) ? 128u : 1u);
     misc[1] = 0;
     misc[2] = 0;
     ptx::fence_barrier_init();

@@ -1,0 +1,161 @@
+"""GPU parity: the CUDA path (through the C-ABI binding) against the fp64 oracle.
+
+Tolerances: O max-abs <= 2e-2 and lse max-abs <= 1e-3 against the unrounded
+fp64 oracle on the same bf16 inputs (O is bf16 on the GPU, so its own rounding
+alone costs up to 2^-9 relative); layouts are compared bit-exactly in the
+CPU tests.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import attention as OA
+from oracle import layout as OL
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+O_TOL = 2e-2
+LSE_TOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def bsa():
+    from block_sparse_attention_bigbird_b200 import bsa as _bsa
+    return _bsa
+
+
+def _run(bsa, w, key_mask=None, scale=None, data_seed=0, explicit_globals=None):
+    q, k, v = workloads.make_qkv(w, data_seed)
+    lay = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed,
+                               globals=explicit_globals)
+    bsa.bsa_layout_upload(lay)
+    dev = torch.device("cuda")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    kmd = key_mask.to(dev) if key_mask is not None else None
+    out, lse = bsa.bsa_forward(qd, kd, vd, lay, key_mask=kmd, scale=scale)
+    assert bsa.bsa_sync_status() == 0
+    ref_layout = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed,
+                                 explicit_globals=explicit_globals)
+    return (q, k, v), lay, ref_layout, out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _check(o_gpu, lse_gpu, o_ref, lse_ref):
+    assert np.all(np.isfinite(o_gpu))
+    err_o = np.abs(o_gpu - o_ref).max()
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isneginf(lse_gpu), ~fin)
+    err_l = np.abs(lse_gpu[fin] - lse_ref[fin]).max() if fin.any() else 0.0
+    assert err_o <= O_TOL, f"O max-abs {err_o}"
+    assert err_l <= LSE_TOL, f"lse max-abs {err_l}"
+    return err_o, err_l
+
+
+SMALL = [
+    # name, workload, key padding tail, scale
+    ("tiny_b1h2l512", workloads.get("c1"), 0, None),
+    ("odd_blocks_ragged_tail", workloads.custom(2, 3, 64 * 13, 1, 1, 2, seed=5), 0, None),
+    ("two_globals_split", workloads.custom(1, 2, 64 * 64, 1, 2, 3, seed=1), 0, None),
+    ("many_globals_split_single", workloads.custom(1, 2, 64 * 100, 2, 7, 4, seed=2), 0, None),
+    ("key_padding_partial", workloads.custom(2, 2, 64 * 20, 1, 2, 2, seed=3, key_pad_tail=100), 100, None),
+    ("dense_window", workloads.custom(1, 2, 64 * 6, 8, 0, 0), 0, None),
+    ("all_global", workloads.custom(1, 1, 64 * 70, 0, 70, 0), 0, None),
+    ("explicit_scale_sharp", workloads.custom(1, 2, 64 * 16, 1, 1, 2, k_mul=2.0), 0, 0.3),
+    ("no_random_no_global", workloads.custom(2, 2, 64 * 9, 0, 0, 0), 0, None),
+]
+
+
+@pytest.mark.parametrize("name,w,pad,scale", SMALL, ids=[s[0] for s in SMALL])
+def test_parity_small_full(bsa, name, w, pad, scale):
+    km = workloads.make_key_mask(w) if pad else None
+    (q, k, v), _, ref_lay, o, lse = _run(bsa, w, key_mask=km, scale=scale)
+    o_ref, lse_ref = OA.attention(q, k, v, ref_lay, key_mask=km, scale=scale)
+    _check(o, lse, o_ref, lse_ref)
+
+
+def test_fully_masked_rows_give_zero_and_neg_inf(bsa):
+    # window 0, no globals/random: block i attends block i only; mask block 2's keys.
+    w = workloads.custom(1, 1, 64 * 5, 0, 0, 0)
+    km = torch.ones((1, w.L), dtype=torch.uint8)
+    km[0, 128:192] = 0
+    (q, k, v), _, ref_lay, o, lse = _run(bsa, w, key_mask=km)
+    assert np.all(o[0, 0, 128:192] == 0) and np.all(np.isneginf(lse[0, 0, 128:192]))
+    o_ref, lse_ref = OA.attention(q, k, v, ref_lay, key_mask=km)
+    _check(o, lse, o_ref, lse_ref)
+
+
+def test_explicit_globals(bsa):
+    w = workloads.custom(1, 2, 64 * 30, 1, 3, 2, seed=4)
+    (q, k, v), _, ref_lay, o, lse = _run(bsa, w, explicit_globals=[29, 5, 11])
+    o_ref, lse_ref = OA.attention(q, k, v, ref_lay)
+    _check(o, lse, o_ref, lse_ref)
+
+
+def _sample_tokens(w, globals_, rng, n_random_rows=48):
+    toks = set()
+    for g in globals_[:4]:
+        toks.update([64 * g, 64 * g + 17, 64 * g + 63])
+    toks.update([0, 63, 64, w.L - 64, w.L - 1])
+    toks.update(rng.integers(0, w.L, n_random_rows).tolist())
+    return sorted(toks)
+
+
+@pytest.mark.parametrize("name", ["c2", "c3", "c4", "c5"])
+def test_parity_full_size_sampled(bsa, name):
+    """Full benchmark shapes in the launch configuration the benchmark times,
+    checked on sampled rows (all head/batch pairs' first and last rows, rows of
+    global blocks, and seeded random rows)."""
+    w = workloads.get(name)
+    km = workloads.make_key_mask(w)
+    (q, k, v), _, ref_lay, o, lse = _run(bsa, w, key_mask=km)
+    rng = np.random.default_rng(0)
+    pairs = [(b, h) for b in range(w.B) for h in range(w.H)]
+    pick = [pairs[i] for i in sorted(set([0, len(pairs) - 1] + rng.integers(0, len(pairs), 3).tolist()))]
+    worst_o = worst_l = 0.0
+    for b, h in pick:
+        toks = _sample_tokens(w, ref_lay["globals"], rng)
+        o_ref, lse_ref = OA.attention_rows(q, k, v, ref_lay, b, h, toks, key_mask=km)
+        eo, el = _check(o[b, h, toks], lse[b, h, toks], o_ref, lse_ref)
+        worst_o, worst_l = max(worst_o, eo), max(worst_l, el)
+    # every row attends unpadded global block 0, so every lse is finite
+    assert np.isfinite(lse).all()
+
+
+def test_constant_v_gives_constant_output_everywhere(bsa):
+    # A property that holds at any size: softmax rows sum to 1, so v == c gives
+    # O == c up to the bf16 rounding of P (l is summed from the unrounded fp32 p).
+    w = workloads.get("c3")
+    q, k, _ = workloads.make_qkv(w)
+    v = torch.full_like(q, 0.5)
+    lay = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(lay)
+    out, lse = bsa.bsa_forward(q.cuda(), k.cuda(), v.cuda(), lay)
+    assert bsa.bsa_sync_status() == 0
+    dev = (out.float() - 0.5).abs().max().item()
+    assert dev <= 4e-3, dev
+    assert torch.isfinite(lse).all().item()
+
+
+def test_deterministic_and_workspace_left_clean(bsa):
+    w = workloads.custom(2, 2, 64 * 64, 1, 2, 3, seed=1)
+    q, k, v = [t.cuda() for t in workloads.make_qkv(w)]
+    lay = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(lay)
+    ws = torch.zeros(bsa.bsa_workspace_bytes(lay, w.B), dtype=torch.uint8, device="cuda")
+    o1, l1 = bsa.bsa_forward(q, k, v, lay, workspace=ws)
+    o2, l2 = bsa.bsa_forward(q, k, v, lay, workspace=ws)
+    assert bsa.bsa_sync_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0   # tickets back at zero
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(bsa):
+    bsa.bsa_debug_wait_timeout(2_000_000)   # 2 ms on a barrier nothing completes
+    assert bsa.bsa_sync_status() == bsa.BSA_ERR_DEVICE_TIMEOUT
+    assert bsa.bsa_sync_status() == 0        # status word was cleared
+    x = torch.arange(10, device="cuda").sum().item()
+    assert x == 45
