@@ -1,0 +1,450 @@
+"""Benchmark: BigBird block-sparse attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {ours,reference}]
+                    [--workload NAME]
+
+Metric: effective TFLOP/s counted over the layout's non-zero 64x64 blocks
+(4 * 64 * 64 * d flop per (b, h, query block, key block); fully key-padded
+blocks excluded), and its fraction of the measured B200 dense bf16 peak.
+
+One step = one bsa_forward over one batch of the workload (inputs resident in
+HBM).  Weak scaling: under torchrun every rank runs its own batch of the same
+shape (its own data seed); there is no data-path collective, only a barrier and
+a max-over-ranks reduction of the timings.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the CPU oracle (fp64 masked-dense, as it stands) on
+the host cores, each step a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "block-sparse attn fwd TFLOP/s (non-zero blocks) and % of B200 bf16 peak"
+UNIT = "TFLOP/s"
+FLOP_PER_BLOCK = 4 * 64 * 64 * 64
+DEFAULT_WORKLOAD = "long_b4h12l16384"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except OSError:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def _source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_attention_bigbird_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_for(workload: str):
+    """DRAM bytes per launch from a committed ncu summary of the CURRENT kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except OSError:
+        return None
+    e = d.get(workload)
+    if not e or e.get("source_hash") != _source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def _dead_from(w):
+    """First key block whose 64 keys are all padded (None when nothing is padded)."""
+    if not w.key_pad_tail:
+        return None
+    return (w.L - w.key_pad_tail + 63) // 64
+
+
+def _nnz_eff(w, row_ptr, col_idx) -> int:
+    """Blocks over all (b, h, i, j), minus those whose 64 keys are all padded."""
+    per_batch = int(len(col_idx))
+    dead = _dead_from(w)
+    if dead is not None:
+        per_batch -= int(np.count_nonzero(col_idx >= dead))
+    return w.B * per_batch
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons in a background thread."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self._stop = threading.Event()
+        self._proc = None
+        sel = str(device_index)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
+        self._cmd = ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "100"]
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        try:
+            self._proc = subprocess.Popen(self._cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                          text=True)
+        except OSError:
+            return
+        for line in self._proc.stdout:
+            if self._stop.is_set():
+                break
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                self.samples.append((time.time(), float(parts[0]), float(parts[1]), parts[3:8]))
+            except ValueError:
+                continue
+
+    def start(self):
+        self._t.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except Exception:
+                self._proc.kill()
+        self._t.join(timeout=5)
+
+    def summary(self, t0: float, t1: float, t_timed0: float):
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "no nvidia-smi samples"}
+        names = ["active_mask", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for s in win:
+            for n, v in zip(names[1:], s[3][1:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(s[1] for s in win),
+                "sm_max_mhz": max(s[2] for s in win), "reasons": sorted(reasons),
+                "samples": len(win), "samples_in_timed_region": sum(1 for s in win if s[0] >= t_timed0),
+                "window": "settle run + timed region"}
+
+
+def _dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus > 1 and world == 1:
+        raise SystemExit("--gpus N > 1 needs torchrun (one process per GPU)")
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def _config(w, nnz_eff, world):
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d": w.d, "block": w.block,
+            "window": w.window, "n_global": w.n_global, "n_random": w.n_random,
+            "key_pad_tail": w.key_pad_tail, "nnz_blocks_per_rank": nnz_eff,
+            "global_batch": w.B * world, "seq_len": w.L, "parallelism": f"dp{world}",
+            "l2": "inputs larger than L2 (q,k,v %d MB + out %d MB per step vs 126 MB L2)"
+                  % (3 * w.B * w.H * w.L * w.d * 2 >> 20, w.B * w.H * w.L * w.d * 2 >> 20)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def _oracle_heads(w):
+    from oracle import layout as OL
+    return OL.build_layout(w.H, w.L, w.block, w.window, w.n_global, w.n_random, w.seed)
+
+
+def _head_view(lay, h):
+    nb = lay["nb"]
+    rp = lay["row_ptr"][h * nb:(h + 1) * nb + 1]
+    return {"H": 1, "L": lay["L"], "block": lay["block"], "nb": nb, "globals": lay["globals"],
+            "row_ptr": rp - rp[0], "col_idx": lay["col_idx"][rp[0]:rp[-1]]}
+
+
+def _oracle_cores():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"), default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def _oracle_sample(w, lay, q, k, v, km, h, n_blocks):
+    """Oracle on query blocks [0, n_blocks) of (b=0, head h); returns (seconds, flop counted)."""
+    from oracle import attention as OA
+    view = _head_view(lay, h)
+    rp, ci = view["row_ptr"], view["col_idx"]
+    nnz = int(rp[n_blocks])
+    dead = _dead_from(w)
+    if dead is not None:
+        nnz -= int(np.count_nonzero(ci[:rp[n_blocks]] >= dead))
+    sl = slice(h, h + 1)
+    kmask = None if km is None else km[0:1]
+    t0 = time.perf_counter()
+    OA.attention(q[0:1, sl], k[0:1, sl], v[0:1, sl], view, key_mask=kmask,
+                 query_blocks=range(n_blocks))
+    return time.perf_counter() - t0, nnz * FLOP_PER_BLOCK
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    lay = _oracle_heads(w)
+    q, k, v = workloads.make_qkv(w, 0)
+    km = workloads.make_key_mask(w)
+    nb = w.nb
+    n_blocks = max(1, min(nb, int(os.environ.get("BSA_REF_BLOCKS", "8"))))
+    for s in range(args.warmup):
+        _oracle_sample(w, lay, q, k, v, km, s % w.H, n_blocks)
+    tot_t = tot_f = 0.0
+    for s in range(args.steps):
+        dt, fl = _oracle_sample(w, lay, q, k, v, km, s % w.H, n_blocks)
+        tot_t += dt
+        tot_f += fl
+    val = tot_f / tot_t / 1e12
+    cores = _oracle_cores()
+    sample = (f"per step: query blocks 0..{n_blocks - 1} of batch 0, head step%H "
+              f"({n_blocks * 64} of {w.L} query rows), fp64 masked-dense")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(w, None, world),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, w, world, rank, local):
+    from block_sparse_attention_bigbird_b200 import bsa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    q, k, v = workloads.make_qkv(w, data_seed=rank)
+    km = workloads.make_key_mask(w)
+    lay = bsa.bsa_layout_build(w.H, w.L, w.block, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(lay)
+    row_ptr, col_idx = bsa.bsa_layout_csr(lay)
+    nnz_eff = _nnz_eff(w, row_ptr, col_idx)
+    flop_step = nnz_eff * FLOP_PER_BLOCK
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    kmd = km.to(dev) if km is not None else None
+    out = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    ws = torch.zeros(bsa.bsa_workspace_bytes(lay, w.B), dtype=torch.uint8, device=dev)
+    launches_per_step = 1 + (1 if km is not None else 0)
+
+    def step():
+        bsa.bsa_forward(qd, kd, vd, lay, key_mask=kmd, out=out, lse=lse, workspace=ws, stream=stream)
+
+    sampler = ClockSampler(local).start() if rank == 0 else None
+    for _ in range(max(3, args.warmup)):
+        step()
+    _barrier(world)
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error during warm-up")
+    # settle run so clock samples reflect the loaded GPU (untimed)
+    t_settle = time.time()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    per = max(e0.elapsed_time(e1), 1e-3)
+    for _ in range(int(min(4000, 1500.0 / per))):
+        step()
+    # ---- timed region: exactly K steps
+    _barrier(world)
+    t_timed0 = time.time()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    end.record(stream)
+    _barrier(world)
+    t_timed1 = time.time()
+    status = bsa.bsa_sync_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} in the timed region")
+    total_ms = _max_over_ranks(start.elapsed_time(end), world)
+    kernel_ms = _max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, world)
+    clocks = sampler.summary(t_settle, t_timed1, t_timed0) if sampler else None
+    if sampler:
+        sampler.stop()
+
+    # ---- end to end through the public API: pinned host buffers, copies inside the region
+    e2e_steps = max(1, min(args.steps, 20))
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    kmh = km.pin_memory() if km is not None else None
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = 3 * qh.numel() * qh.element_size() + (kmh.numel() if kmh is not None else 0)
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        if kmh is not None:
+            kmd.copy_(kmh, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    _barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    _barrier(world)
+    e2e_ms = _max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error in the end-to-end run")
+
+    ms_per_step = total_ms / args.steps
+    value = world * flop_step / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = _peaks()
+    achieved = flop_step / (kernel_ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = _traffic_for(w.name)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = _cpu_baseline(w)
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded randn, see workloads.py)",
+        "config": _config(w, nnz_eff, world),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "bsa_fwd_kernel", "peak_source": f"{peak_src} bf16 burst",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
+        "e2e": {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _cpu_baseline(w):
+    lay = _oracle_heads(w)
+    q, k, v = workloads.make_qkv(w, 0)
+    km = workloads.make_key_mask(w)
+    budget = float(os.environ.get("BSA_CPU_BUDGET_S", "12"))
+    tot_t = tot_f = 0.0
+    n_blocks = min(w.nb, 16)
+    h = 0
+    while tot_t < budget and h < w.H:
+        dt, fl = _oracle_sample(w, lay, q, k, v, km, h, n_blocks)
+        tot_t += dt
+        tot_f += fl
+        h += 1
+    return {"value": tot_f / tot_t / 1e12, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"query blocks 0..{n_blocks - 1} of batch 0 for heads 0..{h - 1} "
+                      f"({h * n_blocks * 64} query rows, {tot_t:.1f} s of fp64 masked-dense)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = workloads.get(args.workload)
+    if args.impl == "reference":
+        # rank 0 alone times the CPU oracle; the other ranks exit without work
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, w, world, rank)
+        return
+    world, rank, local = _dist_setup(args)
+    try:
+        run_ours(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -64,8 +64,12 @@ def masked_softmax_av(s: np.ndarray, allowed: np.ndarray, v: np.ndarray):
     return o, lse
 
 
-def attention(q, k, v, layout: dict, key_mask=None, scale=None):
-    """O [B,H,L,d] and lse [B,H,L] in fp64 for the block layout (masked-dense)."""
+def attention(q, k, v, layout: dict, key_mask=None, scale=None, query_blocks=None):
+    """O [B,H,L,d] and lse [B,H,L] in fp64 for the block layout (masked-dense).
+
+    ``query_blocks`` optionally restricts the computation to those query blocks
+    (the other rows of the result stay zero); the arithmetic is unchanged.
+    """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
     B, H, L, d = q.shape
     if scale is None:
@@ -78,7 +82,7 @@ def attention(q, k, v, layout: dict, key_mask=None, scale=None):
     for b in range(B):
         for h in range(H):
             kt = k[b, h].T
-            for i in range(nb):
+            for i in (range(nb) if query_blocks is None else query_blocks):
                 allowed = token_mask_row(layout, h, i, L)
                 if km is not None:
                     allowed = allowed & km[b]
