@@ -8,17 +8,26 @@
 // per-tile list of 64-key blocks ("SQA 稀疏注意力机制详解" 3.1: block-sparse mask,
 // attention only on non-zero blocks).
 //
-// Kernel design (one persistent CTA per SM, 192 threads):
-//   warp 4      TMA producer: Q tile (2 x 64 rows), then K and V blocks of the tile's
-//               key-block union into a kStages-deep shared-memory ring.
-//   warp 5      tcgen05 issuer: S = Q K^T (M=128, N=64|128, K=64) into one of two TMEM
-//               S buffers, then O += P V (A = P read from TMEM, M=128, N=64).
-//   warps 0-3   softmax + epilogue: thread r owns tile row r = TMEM lane r.  Reads S,
-//               applies the tile's membership bits and key padding, keeps the running
-//               max / sum in fp32, writes P (bf16) over S in TMEM, rescales O when the
-//               max grows by more than kRescaleLog2, and finally normalises O.
+// Kernel design (one persistent CTA per SM, 352 threads):
+//   warp 8      TMA producer: Q tile (2 x 64 rows), then K and V of two key blocks per
+//               chunk of the tile's key-block union into a K ring (released when the
+//               chunk's S is done) and a deeper V ring (released after its PV).
+//   warp 9      tcgen05 S issuer: S = Q K^T (M=128, N=64|128, K=64) into one of three
+//               TMEM S buffers.
+//   warp 10     tcgen05 PV issuer: per key block O_x += P_x V_x (A = P from TMEM, M=128,
+//               N=64, K=64) into that block's own accumulator.  Two issuing threads
+//               keep the tensor pipe fed: each tcgen05 instruction, barrier wait and
+//               commit blocks its thread, and d = 64 makes every MMA short.
+//   warps 0-7   softmax + epilogue, two warpgroups.  Warpgroup x (warps 4x..4x+3)
+//               handles key block x of every chunk: thread (warp w, lane l) owns tile
+//               row r = 32 (w % 4) + l = TMEM lane r.  Each warpgroup keeps its own
+//               running max m_x and sum l_x (fp32) and its own O_x accumulator, writes
+//               P_x (bf16) over its half of S, and rescales O_x when m_x grows by more
+//               than kRescaleLog2.  The epilogue merges (m_A, l_A, O_A) and
+//               (m_B, l_B, O_B); each warpgroup finishes 32 of the 64 output columns.
 // A tile is two query blocks of the same (b, h) over the sorted union of their rows;
-// entries carry per-block membership bits so each half sees exactly its own row.
+// entries carry per-block membership bits so each half of the tile sees exactly its
+// own row, and a warp whose half does not attend a block skips its exponentials.
 // Long unions (global rows) are cut into chunks processed by different CTAs; each
 // chunk stores a partial (O, m, l) and the last one to arrive merges them.
 // Every wait is bounded (globaltimer); on expiry the CTA records
@@ -37,14 +46,19 @@
 
 namespace bsa {
 
-constexpr int kThreads = 192;
-constexpr int kStages = 4;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;  // S issuer; also allocates and frees TMEM
+constexpr int kPvWarp = 10;
+constexpr int kThreads = 352;
+constexpr int kKStages = 3;  // == kSBufs: K stage g % 3 is free once S(g) is done
+constexpr int kVStages = 5;  // V stage g % 5 is free once PV(g) is done
 constexpr uint32_t kBlkBytes = 64 * 128;         // one 64 x 64 bf16 block
 constexpr uint32_t kQBytes = 2 * kBlkBytes;      // 128-row Q tile
 constexpr uint32_t kStageBytes = 2 * kBlkBytes;  // two key blocks
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemS = 0;      // S buffers at columns [0,128) and [128,256)
-constexpr uint32_t kTmemO = 256;    // O accumulator at [256, 320)
+constexpr uint32_t kSBufs = 3;    // S buffers of 128 columns at [0,128), [128,256), [256,384)
+constexpr uint32_t kTmemS = 0;
+constexpr uint32_t kTmemO = 384;  // O_A [384,448), O_B [448,512)
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
@@ -54,24 +68,26 @@ constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 // shared memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + 2 * kQBytes;
-constexpr uint32_t kSmemV = kSmemK + kStages * kStageBytes;
-constexpr uint32_t kSmemBar = kSmemV + kStages * kStageBytes;
+constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
+constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
 enum : int {
   kBarQFull = 0,
   kBarQEmpty = 2,
-  kBarKFull = 4,
-  kBarKEmpty = kBarKFull + kStages,
-  kBarVFull = kBarKEmpty + kStages,
-  kBarVEmpty = kBarVFull + kStages,
-  kBarSFull = kBarVEmpty + kStages,
-  kBarPFull = kBarSFull + 2,
-  kBarODone = kBarPFull + 2,
-  kBarMmaFinal = kBarODone + 1,
-  kBarEpi = kBarMmaFinal + 1,  // 128 softmax threads, split-chunk epilogue
+  kBarKFull = 4,                          // [K stage] K of the stage landed (TMA)
+  kBarVFull = kBarKFull + kKStages,       // [V stage] V of the stage landed (TMA)
+  kBarVFree = kBarVFull + kVStages,       // [V stage] MMA commit after the chunk's PV: the V
+                                          // stage is reusable and both O_x hold that chunk
+  kBarSFull = kBarVFree + kVStages,       // [S buffer] MMA commit after S: S readable, and
+                                          // the K stage of the same index reusable
+  kBarPFull = kBarSFull + kSBufs,         // [S buffer] both warpgroups' P written, 256 arrivals
+  kBarOFree = kBarPFull + kSBufs,         // 256 arrivals once the epilogue has read O
+  kBarMmaFinal = kBarOFree + 1,           // [2 issuers]
+  kBarEpi = kBarMmaFinal + 2,        // 256 softmax threads, epilogue rendezvous
   kNumBars = kBarEpi + 1
 };
 constexpr uint32_t kSmemMisc = kSmemBar + 8 * kNumBars;
-constexpr uint32_t kSmemUsed = kSmemMisc + 16;
+constexpr uint32_t kSmemXch = (kSmemMisc + 16 + 15) & ~15u;  // [2 tile parity][2 wg][2 (m,l)][128] fp32
+constexpr uint32_t kSmemUsed = kSmemXch + 2 * 2 * 2 * kTileRows * 4;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 
@@ -129,71 +145,69 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ------------------------------------------------------------ roles
+// Single-thread wait (the TMA and MMA roles run on one elected lane).
+__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t timeout_ns) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, abort_flag, timeout_ns, true);
+}
+
+// TMA producer, one thread: Q tile, then for each chunk c its K into K stage c % 3
+// (once S(c - 3) is done) and its V into V stage c % 5 (once PV(c - 5) is done).
 __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sQ, uint32_t sK,
-                                              uint32_t sV, uint32_t bars, int lane,
-                                              volatile int* abort_flag) {
+                                              uint32_t sV, uint32_t bars, volatile int* abort_flag) {
+  static_assert(kKStages == static_cast<int>(kSBufs), "K stages are released by the S-full commits");
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   const uint64_t pol_q = ptx::policy_evict_first();
   const uint64_t pol_kv = ptx::policy_evict_last();
   const int total = p.B * p.items_per_batch;
-  uint32_t nq = 0, nq_issued = 0, nk = 0, nv = 0;  // tiles visited; loads issued per ring
+  uint32_t nq = 0, nk = 0, nv = 0;  // Q tiles, K chunks, V chunks issued
   bool alive = true;
-  for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nq) {
+  for (int t = blockIdx.x; alive && t < total; t += gridDim.x) {
     const int b = t / p.items_per_batch;
     const WorkItem w = p.items[t - b * p.items_per_batch];
     const int row0 = (b * p.H + w.h) * p.L;
     const int qa = p.pair_q[2 * w.pair], qb = p.pair_q[2 * w.pair + 1];
     const uint32_t qs = nq & 1u;
-    if (!wait_warp(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+    if (!wait_one(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
       alive = false;
       break;
     }
-    if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(bar(kBarQFull + qs), kQBytes);
-      ptx::tma_load_2d(sQ + qs * kQBytes, &p.tm_q, bar(kBarQFull + qs), 0, row0 + qa * 64, pol_q);
-      ptx::tma_load_2d(sQ + qs * kQBytes + kBlkBytes, &p.tm_q, bar(kBarQFull + qs), 0,
-                       row0 + (qb >= 0 ? qb : qa) * 64, pol_q);
-    }
-    __syncwarp();
-    ++nq_issued;
-    const int nch = (w.count + 1) >> 1;
-    for (int n = 0; n < nch; ++n) {
-      const int e = w.start + 2 * n;
-      const int j0 = static_cast<int>(p.pair_ent[e] & kEntColMask);
-      const bool two = 2 * n + 1 < w.count;
-      const int j1 = two ? static_cast<int>(p.pair_ent[e + 1] & kEntColMask) : 0;
+    ptx::mbar_arrive_expect_tx(bar(kBarQFull + qs), kQBytes);
+    ptx::tma_load_2d(sQ + qs * kQBytes, &p.tm_q, bar(kBarQFull + qs), 0, row0 + qa * 64, pol_q);
+    ptx::tma_load_2d(sQ + qs * kQBytes + kBlkBytes, &p.tm_q, bar(kBarQFull + qs), 0,
+                     row0 + (qb >= 0 ? qb : qa) * 64, pol_q);
+    ++nq;
+    const uint32_t* ent = p.pair_ent + w.start;
+    for (int e = 0; e < w.count; e += 2) {
+      const int j0 = static_cast<int>(ent[e] & kEntColMask);
+      const bool two = e + 1 < w.count;
+      const int j1 = two ? static_cast<int>(ent[e + 1] & kEntColMask) : 0;
       const uint32_t bytes = two ? 2 * kBlkBytes : kBlkBytes;
-      const uint32_t st = nk % kStages;
-      if (!wait_warp(bar(kBarKEmpty + st), ((nk / kStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+      const uint32_t ks = nk % kKStages;
+      if (!wait_one(bar(kBarSFull + ks), ((nk / kKStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
-      if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(bar(kBarKFull + st), bytes);
-        ptx::tma_load_2d(sK + st * kStageBytes, &p.tm_k, bar(kBarKFull + st), 0, row0 + j0 * 64, pol_kv);
-        if (two)
-          ptx::tma_load_2d(sK + st * kStageBytes + kBlkBytes, &p.tm_k, bar(kBarKFull + st), 0,
-                           row0 + j1 * 64, pol_kv);
-      }
-      __syncwarp();
+      const uint32_t dk = sK + ks * kStageBytes;
+      ptx::mbar_arrive_expect_tx(bar(kBarKFull + ks), bytes);
+      ptx::tma_load_2d(dk, &p.tm_k, bar(kBarKFull + ks), 0, row0 + j0 * 64, pol_kv);
+      if (two) ptx::tma_load_2d(dk + kBlkBytes, &p.tm_k, bar(kBarKFull + ks), 0, row0 + j1 * 64, pol_kv);
       ++nk;
-      if (!wait_warp(bar(kBarVEmpty + st), ((nv / kStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+      const uint32_t vs = nv % kVStages;
+      if (!wait_one(bar(kBarVFree + vs), ((nv / kVStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
-      if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(bar(kBarVFull + st), bytes);
-        ptx::tma_load_2d(sV + st * kStageBytes, &p.tm_v, bar(kBarVFull + st), 0, row0 + j0 * 64, pol_kv);
-        if (two)
-          ptx::tma_load_2d(sV + st * kStageBytes + kBlkBytes, &p.tm_v, bar(kBarVFull + st), 0,
-                           row0 + j1 * 64, pol_kv);
-      }
-      __syncwarp();
+      const uint32_t dv = sV + vs * kStageBytes;
+      ptx::mbar_arrive_expect_tx(bar(kBarVFull + vs), bytes);
+      ptx::tma_load_2d(dv, &p.tm_v, bar(kBarVFull + vs), 0, row0 + j0 * 64, pol_kv);
+      if (two) ptx::tma_load_2d(dv + kBlkBytes, &p.tm_v, bar(kBarVFull + vs), 0, row0 + j1 * 64, pol_kv);
       ++nv;
     }
   }
   if (!alive) {
-    // Aborted: let every copy this warp issued land before the CTA exits.  The
+    // Aborted: let every copy this thread issued land before the CTA exits.  The
     // last issue into ring slot s had index s + R * floor((n - 1 - s) / R).
     auto drain = [&](int first_bar, uint32_t n, uint32_t ring) {
       for (uint32_t s = 0; s < ring; ++s) {
@@ -203,176 +217,342 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sQ, u
         }
       }
     };
-    drain(kBarQFull, nq_issued, 2u);
-    drain(kBarKFull, nk, static_cast<uint32_t>(kStages));
-    drain(kBarVFull, nv, static_cast<uint32_t>(kStages));
+    drain(kBarQFull, nq, 2u);
+    drain(kBarKFull, nk, static_cast<uint32_t>(kKStages));
+    drain(kBarVFull, nv, static_cast<uint32_t>(kVStages));
   }
 }
 
-__device__ __forceinline__ void mma_role(const FwdParams& p, uint32_t sQ, uint32_t sK, uint32_t sV,
-                                         uint32_t bars, uint32_t tmem, int lane,
-                                         volatile int* abort_flag) {
+// tcgen05 S issuer, one thread.  S(g) = Q K_g^T into S buffer g % 3 once K(g) has
+// landed and PV(g - 3), the previous reader of that buffer, is done.  Its commit
+// also releases K stage g % 3 to the producer.
+__device__ __forceinline__ void s_issuer(const FwdParams& p, uint32_t sQ, uint32_t sK, uint32_t bars,
+                                         uint32_t tmem, volatile int* abort_flag) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   constexpr uint32_t kIdescS128 = ptx::idesc_bf16_f32(128, 128, false);
   constexpr uint32_t kIdescS64 = ptx::idesc_bf16_f32(128, 64, false);
-  constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 64, true);
+  // descriptor start-address fields count 16-byte units
+  const uint64_t dq0 = ptx::smem_desc_sw128(sQ, 16);
+  const uint64_t dk0 = ptx::smem_desc_sw128(sK, 16);
   const int total = p.B * p.items_per_batch;
-  uint32_t g = 0;   // global chunk counter (== K/V ring position)
-  uint32_t nq = 0;  // tiles started
+  uint32_t g = 0, nq = 0;
   bool alive = true;
-  bool have_prev = false;
-  uint32_t prev_g = 0, prev_two = 0, prev_first = 0;
-
-  auto issue_pv = [&](uint32_t pg, uint32_t two, uint32_t first) -> bool {
-    const uint32_t sb = pg & 1u;
-    if (!wait_warp(bar(kBarPFull + sb), (pg >> 1) & 1u, abort_flag, p.timeout_ns)) return false;
-    const uint32_t st = pg % kStages;
-    if (!wait_warp(bar(kBarVFull + st), (pg / kStages) & 1u, abort_flag, p.timeout_ns)) return false;
-    ptx::tc_fence_after();
-    if (lane == 0) {
-      const uint32_t vbase = sV + st * kStageBytes;
-      const int ksteps = two ? 8 : 4;  // 16 keys per MMA
-      for (int k = 0; k < ksteps; ++k) {
-        const uint64_t bdesc = ptx::smem_desc_sw128(vbase + static_cast<uint32_t>(k) * 2048u, 0);
-        ptx::mma_ts(tmem + kTmemO, tmem + kTmemS + sb * 128u + static_cast<uint32_t>(k) * 8u, bdesc,
-                    kIdescPV, (k > 0 || !first) ? 1u : 0u);
-      }
-      ptx::mma_commit(bar(kBarODone));
-      ptx::mma_commit(bar(kBarVEmpty + st));
-    }
-    __syncwarp();
-    return true;
-  };
-
   for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nq) {
     const int b = t / p.items_per_batch;
     const WorkItem w = p.items[t - b * p.items_per_batch];
     const uint32_t qs = nq & 1u;
-    if (!wait_warp(bar(kBarQFull + qs), (nq >> 1) & 1u, abort_flag, p.timeout_ns)) {
-      alive = false;
-      break;
-    }
+    if (!wait_one(bar(kBarQFull + qs), (nq >> 1) & 1u, abort_flag, p.timeout_ns)) break;
+    const uint64_t dq = dq0 + qs * (kQBytes >> 4);
     const int nch = (w.count + 1) >> 1;
     for (int n = 0; n < nch; ++n, ++g) {
-      const uint32_t st = g % kStages;
-      if (!wait_warp(bar(kBarKFull + st), (g / kStages) & 1u, abort_flag, p.timeout_ns)) {
+      const uint32_t ks = g % kKStages;
+      if (!wait_one(bar(kBarKFull + ks), (g / kKStages) & 1u, abort_flag, p.timeout_ns)) {
+        alive = false;
+        break;
+      }
+      if (g >= kSBufs) {
+        const uint32_t gp = g - kSBufs;
+        if (!wait_one(bar(kBarVFree + gp % kVStages), (gp / kVStages) & 1u, abort_flag, p.timeout_ns)) {
+          alive = false;
+          break;
+        }
+      }
+      ptx::tc_fence_after();
+      const bool two = 2 * n + 1 < w.count;
+      const uint64_t dk = dk0 + ks * (kStageBytes >> 4);
+      const uint32_t d = tmem + kTmemS + (g % kSBufs) * 128u;
+      const uint32_t id = two ? kIdescS128 : kIdescS64;
+      ptx::mma_ss(d, dq, dk, id, 0u);  // head dim 64 = 4 x 16: +32 bytes per step
+      ptx::mma_ss(d, dq + 2, dk + 2, id, 1u);
+      ptx::mma_ss(d, dq + 4, dk + 4, id, 1u);
+      ptx::mma_ss(d, dq + 6, dk + 6, id, 1u);
+      ptx::mma_commit(bar(kBarSFull + g % kSBufs));
+      if (n == nch - 1) ptx::mma_commit(bar(kBarQEmpty + qs));
+    }
+  }
+  // Every MMA this thread issued must finish before TMEM is released.
+  ptx::mma_commit(bar(kBarMmaFinal));
+  wait_force(bar(kBarMmaFinal), 0, abort_flag, p.timeout_ns);
+}
+
+// tcgen05 PV issuer, one thread.  Chunk g: once V(g) has landed and both warpgroups
+// have written P(g), O_x (+)= P_x V_x for the chunk's key blocks, then one commit
+// that frees V stage g % 5, tells the S issuer S buffer g % 3 is free, and tells the
+// softmax warps that O holds chunk g.  A tile's first PV waits until the previous
+// tile's epilogue has read O.
+__device__ __forceinline__ void pv_issuer(const FwdParams& p, uint32_t sV, uint32_t bars, uint32_t tmem,
+                                          volatile int* abort_flag) {
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 64, true);
+  const uint64_t dv0 = ptx::smem_desc_sw128(sV, 0);
+  const int total = p.B * p.items_per_batch;
+  uint32_t g = 0, nq = 0;
+  bool alive = true;
+  for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nq) {
+    const int b = t / p.items_per_batch;
+    const WorkItem w = p.items[t - b * p.items_per_batch];
+    const int nch = (w.count + 1) >> 1;
+    for (int n = 0; n < nch; ++n, ++g) {
+      if (n == 0 && !wait_one(bar(kBarOFree), (nq & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+        alive = false;
+        break;
+      }
+      const uint32_t vs = g % kVStages, sb = g % kSBufs;
+      if (!wait_one(bar(kBarVFull + vs), (g / kVStages) & 1u, abort_flag, p.timeout_ns) ||
+          !wait_one(bar(kBarPFull + sb), (g / kSBufs) & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
       ptx::tc_fence_after();
       const bool two = 2 * n + 1 < w.count;
-      if (lane == 0) {
-        const uint32_t qbase = sQ + qs * kQBytes;
-        const uint32_t kbase = sK + st * kStageBytes;
-        for (int k = 0; k < 4; ++k) {  // head dim 64 = 4 x 16, +32 bytes per step
-          const uint64_t adesc = ptx::smem_desc_sw128(qbase + static_cast<uint32_t>(k) * 32u, 16);
-          const uint64_t bdesc = ptx::smem_desc_sw128(kbase + static_cast<uint32_t>(k) * 32u, 16);
-          ptx::mma_ss(tmem + kTmemS + (g & 1u) * 128u, adesc, bdesc, two ? kIdescS128 : kIdescS64,
-                      k > 0 ? 1u : 0u);
-        }
-        ptx::mma_commit(bar(kBarSFull + (g & 1u)));
-        ptx::mma_commit(bar(kBarKEmpty + st));
-        if (n == nch - 1) ptx::mma_commit(bar(kBarQEmpty + qs));
+      const uint32_t acc0 = n == 0 ? 0u : 1u;
+      const uint64_t dv = dv0 + vs * (kStageBytes >> 4);
+      for (uint32_t x = 0; x < (two ? 2u : 1u); ++x) {
+        const uint32_t d = tmem + kTmemO + x * 64u;
+        const uint32_t a = tmem + kTmemS + sb * 128u + x * 64u;
+        const uint64_t bx = dv + x * (kBlkBytes >> 4);
+        ptx::mma_ts(d, a, bx, kIdescPV, acc0);  // 16 keys per MMA
+        ptx::mma_ts(d, a + 8u, bx + (2048u >> 4), kIdescPV, 1u);
+        ptx::mma_ts(d, a + 16u, bx + (4096u >> 4), kIdescPV, 1u);
+        ptx::mma_ts(d, a + 24u, bx + (6144u >> 4), kIdescPV, 1u);
       }
-      __syncwarp();
-      if (have_prev && !issue_pv(prev_g, prev_two, prev_first)) {
-        alive = false;
-        break;
-      }
-      have_prev = true;
-      prev_g = g;
-      prev_two = two ? 1u : 0u;
-      prev_first = n == 0 ? 1u : 0u;
+      ptx::mma_commit(bar(kBarVFree + vs));
     }
   }
-  if (alive && have_prev) issue_pv(prev_g, prev_two, prev_first);
-  // Every MMA this thread issued must finish before TMEM is released.
-  if (lane == 0) ptx::mma_commit(bar(kBarMmaFinal));
-  __syncwarp();
-  wait_force(bar(kBarMmaFinal), 0, abort_flag, p.timeout_ns);
+  ptx::mma_commit(bar(kBarMmaFinal + 1));
+  wait_force(bar(kBarMmaFinal + 1), 0, abort_flag, p.timeout_ns);
 }
 
-__device__ __forceinline__ void mask_block(float (&s)[128], int off, unsigned long long mk) {
+__device__ __forceinline__ void mask_cols(float (&s)[64], unsigned long long mk) {
   if (mk == ~0ull) return;
-  if (mk == 0ull) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) s[off + c] = -INFINITY;
-    return;
-  }
 #pragma unroll
   for (int c = 0; c < 64; ++c)
-    if (!((mk >> c) & 1ull)) s[off + c] = -INFINITY;
+    if (!((mk >> c) & 1ull)) s[c] = -INFINITY;
 }
 
-__device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, uint32_t tmem,
-                                             int warp, volatile int* abort_flag,
-                                             volatile uint32_t* last_flag) {
+// What the epilogue of a finished tile needs; it runs one chunk later (after the
+// first chunk of the next tile) so the wait for the tile's last PV is hidden.  The
+// epilogue's 256-thread rendezvous is an mbarrier with a bounded wait (a plain
+// bar.sync could not give up if another softmax warp had already aborted).
+struct TileDone {
+  int t;            // work item index (its fields are reloaded by the epilogue)
+  uint32_t g_last;  // global index of the tile's last chunk
+  uint32_t nt;      // tile count of this CTA when the tile started
+  float m, l;       // this warpgroup's running max (log2 units) and sum for the row
+};
+
+// Epilogue of a finished tile: merge (m_A, l_A, O_A) with (m_B, l_B, O_B), store O
+// and lse (or the split chunk's partial record, merging when last).  Kept out of
+// line: it runs once per tile and would otherwise crowd the chunk loop's registers.
+__device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& td, uint32_t bars,
+                                           uint32_t obase, int warp, int lane, volatile int* abort_flag,
+                                           volatile uint32_t* last_flag, float* xch, uint32_t* n_epi) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  const int r = threadIdx.x;  // tile row == TMEM lane
+  const int wg = warp >> 2;
+  const int r = (warp & 3) * 32 + lane;
   const int half = r >> 6;
-  const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+  auto epi_sync = [&]() -> bool {
+    ptx::mbar_arrive(bar(kBarEpi));
+    const bool ok = wait_warp(bar(kBarEpi), *n_epi & 1u, abort_flag, p.timeout_ns);
+    ++*n_epi;
+    return ok;
+  };
+  {
+    const int tb = td.t / p.items_per_batch;
+    const WorkItem tw = p.items[td.t - tb * p.items_per_batch];
+    const int tqa = p.pair_q[2 * tw.pair], tqb = p.pair_q[2 * tw.pair + 1];
+    const int tbh = tb * p.H + tw.h;
+    // PV of the tile's last chunk.  Unambiguous phase: S(g_last) was seen, and it
+    // was issued after PV(g_last - 3) was done; PV(g_last + kVStages) needs P this
+    // warpgroup has not produced.
+    if (!wait_warp(bar(kBarVFree + static_cast<int>(td.g_last % kVStages)), (td.g_last / kVStages) & 1u,
+                   abort_flag, p.timeout_ns))
+      return false;
+    // (m, l) exchange, double-buffered by tile parity: a warpgroup that runs ahead
+    // into the next tile cannot overwrite values the other has not read yet.
+    float* xt = xch + (td.nt & 1u) * (2 * 2 * kTileRows);
+    xt[(wg * 2 + 0) * kTileRows + r] = td.m;
+    xt[(wg * 2 + 1) * kTileRows + r] = td.l;
+    if (!epi_sync()) return false;
+    ptx::tc_fence_after();
+    const float m_o = xt[((1 - wg) * 2 + 0) * kTileRows + r];
+    const float l_o = xt[((1 - wg) * 2 + 1) * kTileRows + r];
+    const float mA = wg == 0 ? td.m : m_o, lA = wg == 0 ? td.l : l_o;
+    const float mB = wg == 0 ? m_o : td.m, lB = wg == 0 ? l_o : td.l;
+    const float m = fmaxf(mA, mB);
+    const bool useA = lA > 0.f, useB = lB > 0.f;  // an unused O_x may hold stale values
+    const float fA = useA ? ptx::ex2_approx(mA - m) : 0.f;
+    const float fB = useB ? ptx::ex2_approx(mB - m) : 0.f;
+    const float l = lA * fA + lB * fB;
+    // this warpgroup finishes output columns [32 wg, 32 wg + 32)
+    uint32_t oa[32], ob[32];
+    ptx::tmem_ld32(obase + static_cast<uint32_t>(wg) * 32u, oa);
+    ptx::tmem_ld32(obase + 64u + static_cast<uint32_t>(wg) * 32u, ob);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence(oa);
+    ptx::reg_fence(ob);
+    ptx::tc_fence_before();
+    ptx::mbar_arrive(bar(kBarOFree));  // O may now be overwritten by the next tile
+    float o[32];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+      const float a = useA ? __uint_as_float(oa[c]) * fA : 0.f;
+      const float bb = useB ? __uint_as_float(ob[c]) * fB : 0.f;
+      o[c] = a + bb;
+    }
+    const bool row_active = half == 0 || tqb >= 0;
+    const int qblk = half ? tqb : tqa;
+    const size_t row = static_cast<size_t>(tbh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
+    if (tw.split < 0) {
+      if (row_active) {
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64 + wg * 32);
+#pragma unroll
+        for (int v8 = 0; v8 < 4; ++v8) {
+          uint4 u;
+          u.x = pack_bf16x2(o[v8 * 8 + 0] * inv, o[v8 * 8 + 1] * inv);
+          u.y = pack_bf16x2(o[v8 * 8 + 2] * inv, o[v8 * 8 + 3] * inv);
+          u.z = pack_bf16x2(o[v8 * 8 + 4] * inv, o[v8 * 8 + 5] * inv);
+          u.w = pack_bf16x2(o[v8 * 8 + 6] * inv, o[v8 * 8 + 7] * inv);
+          dst[v8] = u;
+        }
+        if (wg == 0) p.lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+      }
+      return true;
+    }
+    // ---- split chunk: store the partial record, then the last arriver merges
+    float* rec = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec) * kRecFloats;
+    float4* orow = reinterpret_cast<float4*>(rec + r * 64 + wg * 32);
+#pragma unroll
+    for (int v4 = 0; v4 < 8; ++v4)
+      orow[v4] = make_float4(o[v4 * 4 + 0], o[v4 * 4 + 1], o[v4 * 4 + 2], o[v4 * 4 + 3]);
+    if (wg == 0) {
+      rec[kTileRows * 64 + r] = l > 0.f ? m : -INFINITY;
+      rec[kTileRows * 64 + kTileRows + r] = l;
+    }
+    __threadfence();
+    if (!epi_sync()) return false;
+    int* ticket = p.tickets + static_cast<size_t>(tb) * p.n_split + tw.split;
+    if (warp == 0 && lane == 0) *last_flag = (atomicAdd(ticket, 1) == tw.nchunks - 1) ? 1u : 0u;
+    if (!epi_sync()) return false;
+    if (!*last_flag) return true;
+    __threadfence();
+    if (row_active) {
+      const float* base = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec_base) * kRecFloats;
+      float ms = -INFINITY;
+      for (int c = 0; c < tw.nchunks; ++c)
+        ms = fmaxf(ms, __ldcg(base + static_cast<size_t>(c) * kRecFloats + kTileRows * 64 + r));
+      float acc[32];
+#pragma unroll
+      for (int x = 0; x < 32; ++x) acc[x] = 0.f;
+      float lsum = 0.f;
+      if (ms != -INFINITY) {
+        for (int c = 0; c < tw.nchunks; ++c) {
+          const float* rc = base + static_cast<size_t>(c) * kRecFloats;
+          const float mc = __ldcg(rc + kTileRows * 64 + r);
+          const float lc = __ldcg(rc + kTileRows * 64 + kTileRows + r);
+          if (mc == -INFINITY) continue;
+          const float f = ptx::ex2_approx(mc - ms);
+          lsum += lc * f;
+          const float4* oc = reinterpret_cast<const float4*>(rc + r * 64 + wg * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4) {
+            const float4 x = __ldcg(oc + v4);
+            acc[v4 * 4 + 0] += f * x.x;
+            acc[v4 * 4 + 1] += f * x.y;
+            acc[v4 * 4 + 2] += f * x.z;
+            acc[v4 * 4 + 3] += f * x.w;
+          }
+        }
+      }
+      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64 + wg * 32);
+#pragma unroll
+      for (int v8 = 0; v8 < 4; ++v8) {
+        uint4 u;
+        u.x = pack_bf16x2(acc[v8 * 8 + 0] * inv, acc[v8 * 8 + 1] * inv);
+        u.y = pack_bf16x2(acc[v8 * 8 + 2] * inv, acc[v8 * 8 + 3] * inv);
+        u.z = pack_bf16x2(acc[v8 * 8 + 4] * inv, acc[v8 * 8 + 5] * inv);
+        u.w = pack_bf16x2(acc[v8 * 8 + 6] * inv, acc[v8 * 8 + 7] * inv);
+        dst[v8] = u;
+      }
+      if (wg == 0) p.lse[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
+    }
+    if (warp == 0 && lane == 0) *ticket = 0;  // leave the workspace clean for the next call
+    return true;
+  }
+}
+
+
+__device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, uint32_t tmem,
+                                             int warp, int lane, volatile int* abort_flag,
+                                             volatile uint32_t* last_flag, float* xch) {
+  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  const int wg = warp >> 2;              // key block of each chunk handled here
+  const int r = (warp & 3) * 32 + lane;  // tile row == TMEM lane
+  const int half = r >> 6;
+  const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const uint32_t obase = tmem + lane_addr + kTmemO;
   const int total = p.B * p.items_per_batch;
   const float sl2 = p.scale_log2;
   uint32_t g = 0;
   uint32_t n_epi = 0;  // uses of the epilogue barrier
+  uint32_t nt = 0;     // tiles started
   bool alive = true;
-  // Bounded 128-thread rendezvous (a plain bar.sync could not give up if another
-  // softmax warp had already aborted).
-  auto epi_sync = [&]() -> bool {
-    ptx::mbar_arrive(bar(kBarEpi));
-    const bool ok = wait_warp(bar(kBarEpi), n_epi & 1u, abort_flag, p.timeout_ns);
-    ++n_epi;
-    return ok;
-  };
-  for (int t = blockIdx.x; alive && t < total; t += gridDim.x) {
+
+  TileDone pend{};
+  bool have_pend = false;
+  for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nt) {
     const int b = t / p.items_per_batch;
     const WorkItem w = p.items[t - b * p.items_per_batch];
-    const int bh = b * p.H + w.h;
     const int qa = p.pair_q[2 * w.pair], qb = p.pair_q[2 * w.pair + 1];
-    const bool row_active = half == 0 || qb >= 0;
+    // The tile's union entries (at most 64) and their key-padding bits, one or two
+    // per lane; each chunk picks its entry with a shuffle.
+    const uint32_t ent_lo = lane < w.count ? p.pair_ent[w.start + lane] : 0u;
+    const uint32_t ent_hi = lane + 32 < w.count ? p.pair_ent[w.start + 32 + lane] : 0u;
+    unsigned long long kb_lo = ~0ull, kb_hi = ~0ull;
+    if (p.keybits != nullptr) {
+      const size_t kb0 = static_cast<size_t>(b) * p.nb;
+      if (lane < w.count) kb_lo = p.keybits[kb0 + (ent_lo & kEntColMask)];
+      if (lane + 32 < w.count) kb_hi = p.keybits[kb0 + (ent_hi & kEntColMask)];
+    }
     float m_run = -INFINITY, l_run = 0.f;
     const int nch = (w.count + 1) >> 1;
     for (int n = 0; n < nch; ++n, ++g) {
-      const int e = w.start + 2 * n;
-      const uint32_t e0 = p.pair_ent[e];
-      const bool two = 2 * n + 1 < w.count;
-      const uint32_t e1 = two ? p.pair_ent[e + 1] : 0u;
-      unsigned long long mk0 = ((e0 >> (kEntBitsShift + half)) & 1u) ? ~0ull : 0ull;
-      unsigned long long mk1 = ((e1 >> (kEntBitsShift + half)) & 1u) ? ~0ull : 0ull;
-      if (p.keybits != nullptr) {
-        mk0 &= p.keybits[static_cast<size_t>(b) * p.nb + (e0 & kEntColMask)];
-        if (two) mk1 &= p.keybits[static_cast<size_t>(b) * p.nb + (e1 & kEntColMask)];
-      }
-      const uint32_t sb = g & 1u;
-      if (!wait_warp(bar(kBarSFull + sb), (g >> 1) & 1u, abort_flag, p.timeout_ns)) {
+      const int idx = 2 * n + wg;  // warp-uniform
+      const bool has = idx < w.count;
+      const uint32_t e = __shfl_sync(0xffffffffu, idx < 32 ? ent_lo : ent_hi, idx & 31);
+      const unsigned long long kb = __shfl_sync(0xffffffffu, idx < 32 ? kb_lo : kb_hi, idx & 31);
+      // warp-uniform: a warp's 32 rows lie in one half of the tile
+      const unsigned long long mk = (has && ((e >> (kEntBitsShift + half)) & 1u)) ? kb : 0ull;
+      const uint32_t sb = g % kSBufs;
+      if (!wait_warp(bar(kBarSFull + static_cast<int>(sb)), (g / kSBufs) & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
       ptx::tc_fence_after();
-      uint32_t raw[4][32];
-      const uint32_t sbase = tmem + lane_addr + kTmemS + sb * 128u;
-      ptx::tmem_ld32(sbase + 0, raw[0]);
-      ptx::tmem_ld32(sbase + 32, raw[1]);
-      ptx::tmem_ld32(sbase + 64, raw[2]);
-      ptx::tmem_ld32(sbase + 96, raw[3]);
-      ptx::tmem_wait_ld();
-      ptx::reg_fence(raw[0]);
-      ptx::reg_fence(raw[1]);
-      ptx::reg_fence(raw[2]);
-      ptx::reg_fence(raw[3]);
-      float s[128];
+      const uint32_t sbase = tmem + lane_addr + kTmemS + sb * 128u + static_cast<uint32_t>(wg) * 64u;
+      float s[64];
+      float mxs = -INFINITY;
+      if (mk != 0ull) {
+        uint32_t raw[2][32];
+        ptx::tmem_ld32(sbase + 0, raw[0]);
+        ptx::tmem_ld32(sbase + 32, raw[1]);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence(raw[0]);
+        ptx::reg_fence(raw[1]);
 #pragma unroll
-      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
-      mask_block(s, 0, mk0);
-      mask_block(s, 64, mk1);
-      float mx8[8];
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
+        mask_cols(s, mk);
+        float mx8[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx8[c] = s[c];
+        for (int c = 0; c < 8; ++c) mx8[c] = s[c];
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float mxs = mx * sl2;  // scale > 0: -inf stays -inf
+        for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        mxs = mx * sl2;  // scale > 0: -inf stays -inf
+      }
       float m_new = m_run;
       bool rescale = false;
       if (n == 0) {
@@ -382,158 +562,71 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
         m_new = fmaxf(m_run, mxs);
       }
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      uint32_t pk[2][32];
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[32];
+      float psum = 0.f;
+      if (mk != 0ull) {
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = ptx::ex2_approx(fmaf(s[2 * c], sl2, -m_use));
-        const float p1 = ptx::ex2_approx(fmaf(s[2 * c + 1], sl2, -m_use));
-        sum4[c & 3] += p0 + p1;
-        pk[c >> 5][c & 31] = pack_bf16x2(p0, p1);
-      }
-      const float psum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      // PV of the previous chunk must be done before O is touched (and this keeps
-      // the O-done phase tracking exact: one wait per completed PV).
-      if (g > 0) {
-        if (!wait_warp(bar(kBarODone), (g - 1u) & 1u, abort_flag, p.timeout_ns)) {
-          alive = false;
-          break;
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ptx::ex2_approx(fmaf(s[2 * c], sl2, -m_use));
+          const float p1 = ptx::ex2_approx(fmaf(s[2 * c + 1], sl2, -m_use));
+          sum4[c & 3] += p0 + p1;
+          pk[c] = pack_bf16x2(p0, p1);
         }
-        ptx::tc_fence_after();
+        psum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
+      // P_x over S_x: the buffer's previous reader, PV of chunk g - 3, completed
+      // before S(g) was issued.
+      if (has) ptx::tmem_st32(sbase, pk);
       if (n == 0) {
         l_run = psum;
       } else {
         const float alpha = (m_new == m_run) ? 1.f : ptx::ex2_approx(m_run - m_new);
         l_run = l_run * alpha + psum;
         if (rescale) {  // warp-uniform
-          uint32_t o[2][32];
-          const uint32_t obase = tmem + lane_addr + kTmemO;
-          ptx::tmem_ld32(obase + 0, o[0]);
-          ptx::tmem_ld32(obase + 32, o[1]);
-          ptx::tmem_wait_ld();
-          ptx::reg_fence(o[0]);
-          ptx::reg_fence(o[1]);
+          // O_x must hold PV of chunk g - 1 before it is rescaled: wait for its
+          // V-free phase.  Unambiguous: S(g) was issued after PV(g - 3) was done, and
+          // PV(g - 1 + kVStages) needs this warpgroup's P first.
+          const uint32_t gp = g - 1u;
+          if (!wait_warp(bar(kBarVFree + static_cast<int>(gp % kVStages)), (gp / kVStages) & 1u,
+                         abort_flag, p.timeout_ns)) {
+            alive = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t ox = obase + static_cast<uint32_t>(wg) * 64u;
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            o[c >> 5][c & 31] = __float_as_uint(__uint_as_float(o[c >> 5][c & 31]) * alpha);
-          ptx::tmem_st32(obase + 0, o[0]);
-          ptx::tmem_st32(obase + 32, o[1]);
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            uint32_t o[32];
+            ptx::tmem_ld32(ox + 32u * hlf, o);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            ptx::tmem_st32(ox + 32u * hlf, o);
+          }
         }
       }
       m_run = m_new;
-      ptx::tmem_st32(sbase + 0, pk[0]);
-      ptx::tmem_st32(sbase + 32, pk[1]);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(kBarPFull + sb));
-    }
-    if (!alive || nch == 0) break;
-    // ---- epilogue: wait for the tile's last PV, then read O
-    if (!wait_warp(bar(kBarODone), (g - 1u) & 1u, abort_flag, p.timeout_ns)) {
-      alive = false;
-      break;
-    }
-    ptx::tc_fence_after();
-    uint32_t o[2][32];
-    const uint32_t obase = tmem + lane_addr + kTmemO;
-    ptx::tmem_ld32(obase + 0, o[0]);
-    ptx::tmem_ld32(obase + 32, o[1]);
-    ptx::tmem_wait_ld();
-    ptx::reg_fence(o[0]);
-    ptx::reg_fence(o[1]);
-    const int qblk = half ? qb : qa;
-    if (w.split < 0) {
-      if (row_active) {
-        const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64);
-#pragma unroll
-        for (int v8 = 0; v8 < 8; ++v8) {
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 0]) * inv,
-                            __uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 1]) * inv);
-          u.y = pack_bf16x2(__uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 2]) * inv,
-                            __uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 3]) * inv);
-          u.z = pack_bf16x2(__uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 4]) * inv,
-                            __uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 5]) * inv);
-          u.w = pack_bf16x2(__uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 6]) * inv,
-                            __uint_as_float(o[v8 >> 2][(v8 & 3) * 8 + 7]) * inv);
-          dst[v8] = u;
+      ptx::mbar_arrive(bar(kBarPFull + static_cast<int>(sb)));
+      if (n == 0 && have_pend) {  // the previous tile's epilogue, one chunk late
+        have_pend = false;
+        if (!tile_epilogue(p, pend, bars, obase, warp, lane, abort_flag, last_flag, xch, &n_epi)) {
+          alive = false;
+          break;
         }
-        p.lse[row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-      }
-    } else {
-      // ---- split chunk: store the partial record, then the last arriver merges
-      float* rec = p.partials + (static_cast<size_t>(b) * p.n_records + w.rec) * kRecFloats;
-      float4* orow = reinterpret_cast<float4*>(rec + r * 64);
-#pragma unroll
-      for (int v4 = 0; v4 < 16; ++v4)
-        orow[v4] = make_float4(__uint_as_float(o[v4 >> 3][(v4 & 7) * 4 + 0]),
-                               __uint_as_float(o[v4 >> 3][(v4 & 7) * 4 + 1]),
-                               __uint_as_float(o[v4 >> 3][(v4 & 7) * 4 + 2]),
-                               __uint_as_float(o[v4 >> 3][(v4 & 7) * 4 + 3]));
-      rec[kTileRows * 64 + r] = m_run;
-      rec[kTileRows * 64 + kTileRows + r] = l_run;
-      __threadfence();
-      if (!epi_sync()) {
-        alive = false;
-        break;
-      }
-      int* ticket = p.tickets + static_cast<size_t>(b) * p.n_split + w.split;
-      if (r == 0) *last_flag = (atomicAdd(ticket, 1) == w.nchunks - 1) ? 1u : 0u;
-      if (!epi_sync()) {
-        alive = false;
-        break;
-      }
-      if (*last_flag) {
-        __threadfence();
-        if (row_active) {
-          const float* base = p.partials + (static_cast<size_t>(b) * p.n_records + w.rec_base) * kRecFloats;
-          float ms = -INFINITY;
-          for (int c = 0; c < w.nchunks; ++c)
-            ms = fmaxf(ms, __ldcg(base + static_cast<size_t>(c) * kRecFloats + kTileRows * 64 + r));
-          const size_t row = static_cast<size_t>(bh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
-          float acc[64];
-#pragma unroll
-          for (int x = 0; x < 64; ++x) acc[x] = 0.f;
-          float lsum = 0.f;
-          if (ms != -INFINITY) {
-            for (int c = 0; c < w.nchunks; ++c) {
-              const float* rc = base + static_cast<size_t>(c) * kRecFloats;
-              const float mc = __ldcg(rc + kTileRows * 64 + r);
-              const float lc = __ldcg(rc + kTileRows * 64 + kTileRows + r);
-              if (mc == -INFINITY) continue;
-              const float f = ptx::ex2_approx(mc - ms);
-              lsum += lc * f;
-              const float4* oc = reinterpret_cast<const float4*>(rc + r * 64);
-#pragma unroll
-              for (int v4 = 0; v4 < 16; ++v4) {
-                const float4 x = __ldcg(oc + v4);
-                acc[v4 * 4 + 0] += f * x.x;
-                acc[v4 * 4 + 1] += f * x.y;
-                acc[v4 * 4 + 2] += f * x.z;
-                acc[v4 * 4 + 3] += f * x.w;
-              }
-            }
-          }
-          const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-          uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64);
-#pragma unroll
-          for (int v8 = 0; v8 < 8; ++v8) {
-            uint4 u;
-            u.x = pack_bf16x2(acc[v8 * 8 + 0] * inv, acc[v8 * 8 + 1] * inv);
-            u.y = pack_bf16x2(acc[v8 * 8 + 2] * inv, acc[v8 * 8 + 3] * inv);
-            u.z = pack_bf16x2(acc[v8 * 8 + 4] * inv, acc[v8 * 8 + 5] * inv);
-            u.w = pack_bf16x2(acc[v8 * 8 + 6] * inv, acc[v8 * 8 + 7] * inv);
-            dst[v8] = u;
-          }
-          p.lse[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
-        }
-        if (r == 0) *ticket = 0;  // leave the workspace clean for the next call
       }
     }
+    if (!alive) break;
+    pend = TileDone{t, g - 1u, nt, m_run, l_run};
+    have_pend = true;
   }
+  if (alive && have_pend) tile_epilogue(p, pend, bars, obase, warp, lane, abort_flag, last_flag, xch, &n_epi);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -543,21 +636,26 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t sQ = base + kSmemQ, sK = base + kSmemK, sV = base + kSmemV, bars = base + kSmemBar;
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kSmemMisc);
+  float* xch = reinterpret_cast<float*>(smem + kSmemXch);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i)
-      ptx::mbar_init(bars + 8u * i, (i == kBarPFull || i == kBarPFull + 1 || i == kBarEpi) ? 128u : 1u);
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t count = 1;
+      if ((i >= kBarPFull && i < kBarPFull + static_cast<int>(kSBufs)) || i == kBarOFree || i == kBarEpi)
+        count = 256;
+      ptx::mbar_init(bars + 8u * i, count);
+    }
     misc[1] = 0;
     misc[2] = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     ptx::prefetch_tensormap(&p.tm_q);
     ptx::prefetch_tensormap(&p.tm_k);
     ptx::prefetch_tensormap(&p.tm_v);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     ptx::tmem_alloc(ptx::smem_addr(const_cast<uint32_t*>(&misc[0])), kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -567,18 +665,23 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   const uint32_t tmem = misc[0];
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
-  if (warp == 4) {
-    producer_role(p, sQ, sK, sV, bars, lane, abort_flag);
-  } else if (warp == 5) {
-    mma_role(p, sQ, sK, sV, bars, tmem, lane, abort_flag);
+  if (warp == kProducerWarp) {
+    if (lane == 0) producer_role(p, sQ, sK, sV, bars, abort_flag);
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) s_issuer(p, sQ, sK, bars, tmem, abort_flag);
+    __syncwarp();
+  } else if (warp == kPvWarp) {
+    if (lane == 0) pv_issuer(p, sV, bars, tmem, abort_flag);
+    __syncwarp();
   } else {
-    softmax_role(p, bars, tmem, warp, abort_flag, &misc[2]);
+    softmax_role(p, bars, tmem, warp, lane, abort_flag, &misc[2], xch);
   }
 
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 5) ptx::tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
 // Per (b, key block): bit c set when key 64*j + c is kept by the padding mask.
