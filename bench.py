@@ -35,6 +35,7 @@ import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 import workloads  # noqa: E402
+from block_sparse_attention_bigbird_b200 import sharding  # noqa: E402
 
 METRIC = "block-sparse attn fwd TFLOP/s (non-zero blocks) and % of B200 bf16 peak"
 UNIT = "TFLOP/s"
@@ -176,15 +177,6 @@ def _dist_setup(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     return world, rank, local
-
-
-def _max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
 
 
 def _barrier(world: int):
@@ -332,8 +324,8 @@ def run_ours(args, w, world, rank, local):
     status = bsa.bsa_sync_status(stream)
     if status != 0:
         raise RuntimeError(f"device status {status} in the timed region")
-    total_ms = _max_over_ranks(start.elapsed_time(end), world)
-    kernel_ms = _max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, world)
+    total_ms = sharding.max_over_ranks(start.elapsed_time(end), world)
+    kernel_ms = sharding.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / args.steps, world)
     clocks = sampler.summary(t_settle, t_timed1, t_timed0) if sampler else None
     if sampler:
         sampler.stop()
@@ -365,7 +357,7 @@ def run_ours(args, w, world, rank, local):
         e2e_step()
     b.record(stream)
     _barrier(world)
-    e2e_ms = _max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
+    e2e_ms = sharding.max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
     if bsa.bsa_sync_status(stream) != 0:
         raise RuntimeError("device status error in the end-to-end run")
 

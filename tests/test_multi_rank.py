@@ -1,0 +1,78 @@
+"""Multi-rank host logic on CPU with two gloo ranks (no GPU).
+
+A forward split by batch element across ranks, each rank computing its shard
+(here with the fp64 oracle, since no GPU is present), must reproduce the
+single-process result once gathered; the timing reduction must return the
+maximum over ranks.
+"""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import workloads
+from block_sparse_attention_bigbird_b200 import sharding
+from oracle import attention as OA
+from oracle import layout as OL
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, queue):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = workloads.custom(3, 2, 64 * 6, 1, 1, 2, seed=3)
+        q, k, v = workloads.make_qkv(w)
+        lay = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+        b0, b1 = sharding.batch_shard(w.B, rank, world)
+        o, lse = OA.attention(q[b0:b1], k[b0:b1], v[b0:b1], lay)
+        shards = [None] * world
+        dist.all_gather_object(shards, (b0, b1, o, lse))
+        slowest = sharding.max_over_ranks(0.5 + rank, world)
+        if rank == 0:
+            queue.put((shards, slowest))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_batch_shard_covers_exactly():
+    for B in range(0, 9):
+        for world in range(1, 5):
+            spans = [sharding.batch_shard(B, r, world) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == B
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            sizes = [b - a for a, b in spans]
+            assert max(sizes) - min(sizes) <= 1
+
+
+def test_two_gloo_ranks_reproduce_single_process():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, queue)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    shards, slowest = queue.get(timeout=120)
+    for pr in procs:
+        pr.join(timeout=120)
+        assert pr.exitcode == 0
+    assert slowest == 1.5
+    w = workloads.custom(3, 2, 64 * 6, 1, 1, 2, seed=3)
+    q, k, v = workloads.make_qkv(w)
+    lay = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    o_ref, lse_ref = OA.attention(q, k, v, lay)
+    o = np.concatenate([s[2] for s in sorted(shards, key=lambda x: x[0])])
+    lse = np.concatenate([s[3] for s in sorted(shards, key=lambda x: x[0])])
+    assert np.array_equal(o, o_ref) and np.array_equal(lse, lse_ref)
