@@ -64,6 +64,7 @@ constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr uint32_t kMaxSpin = 1u << 24;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+constexpr uint32_t kWaitSleepNs = 20000;  // upper bound on one sleep inside a barrier wait
 
 // shared memory map (offsets from a 1024-aligned base)
 constexpr uint32_t kSmemQ = 0;
@@ -113,7 +114,9 @@ __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile i
                                        uint64_t timeout_ns, bool honor_abort) {
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    // sleeping in the barrier instead of spinning leaves issue slots to the
+    // warps that share this SM sub-partition
+    if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if ((it & 15u) == 0) {
       if (honor_abort && *abort_flag) return false;
       if (ptx::globaltimer_ns() - t0 > timeout_ns || it > kMaxSpin) {
@@ -505,7 +508,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
   for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nt) {
     const int b = t / p.items_per_batch;
     const WorkItem w = p.items[t - b * p.items_per_batch];
-    const int qa = p.pair_q[2 * w.pair], qb = p.pair_q[2 * w.pair + 1];
     // The tile's union entries (at most 64) and their key-padding bits, one or two
     // per lane; each chunk picks its entry with a shuffle.
     const uint32_t ent_lo = lane < w.count ? p.pair_ent[w.start + lane] : 0u;
@@ -532,7 +534,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
       }
       ptx::tc_fence_after();
       const uint32_t sbase = tmem + lane_addr + kTmemS + sb * 128u + static_cast<uint32_t>(wg) * 64u;
-      float s[64];
+      // Pass 1: the row maximum of this warpgroup's 64 scores.
       float mxs = -INFINITY;
       if (mk != 0ull) {
         uint32_t raw[2][32];
@@ -541,16 +543,14 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
         ptx::tmem_wait_ld();
         ptx::reg_fence(raw[0]);
         ptx::reg_fence(raw[1]);
+        float s[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
         mask_cols(s, mk);
-        float mx8[8];
+        float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mx8[c] = s[c];
-#pragma unroll
-        for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 4; c < 64; c += 2) mx4[(c >> 1) & 3] = ptx::fmax3(mx4[(c >> 1) & 3], s[c], s[c + 1]);
+        const float mx = fmaxf(ptx::fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
         mxs = mx * sl2;  // scale > 0: -inf stays -inf
       }
       float m_new = m_run;
@@ -562,25 +562,53 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
         m_new = fmaxf(m_run, mxs);
       }
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      uint32_t pk[32];
+      // Pass 2: p = 2^(s * scale * log2 e - m) 32 columns at a time, reloaded from TMEM
+      // to keep few registers live; P_x (bf16, two keys per column) goes over S
+      // columns already read.  The buffer's previous reader, PV of chunk g - 3,
+      // completed before S(g) was issued.
       float psum = 0.f;
       if (mk != 0ull) {
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_use, -m_use);
+        uint64_t acc0 = 0ull, acc1 = 0ull;  // packed partial row sums
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = ptx::ex2_approx(fmaf(s[2 * c], sl2, -m_use));
-          const float p1 = ptx::ex2_approx(fmaf(s[2 * c + 1], sl2, -m_use));
-          sum4[c & 3] += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+        for (int hb = 0; hb < 2; ++hb) {
+          uint32_t raw[32];
+          ptx::tmem_ld32(sbase + 32u * hb, raw);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(raw);
+          float s[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(raw[c]);
+          const uint32_t mh = static_cast<uint32_t>(mk >> (32 * hb));
+          if (mh != 0xffffffffu) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (!((mh >> c) & 1u)) s[c] = -INFINITY;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            float x0, x1;
+            ptx::unpack2(ptx::ffma2(ptx::pack2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
+            const float p0 = ptx::ex2_approx(x0), p1 = ptx::ex2_approx(x1);
+            if (c & 1)
+              acc1 = ptx::fadd2(acc1, ptx::pack2(p0, p1));
+            else
+              acc0 = ptx::fadd2(acc0, ptx::pack2(p0, p1));
+            pk[c] = pack_bf16x2(p0, p1);
+          }
+          ptx::tmem_st16(sbase + 16u * hb, pk);
         }
-        psum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      } else {
+        float a0, a1;
+        ptx::unpack2(ptx::fadd2(acc0, acc1), a0, a1);
+        psum = a0 + a1;
+      } else if (has) {
+        // this half of the tile does not attend the block: its P rows are zero
+        uint32_t zero[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        for (int c = 0; c < 32; ++c) zero[c] = 0u;
+        ptx::tmem_st32(sbase, zero);
       }
-      // P_x over S_x: the buffer's previous reader, PV of chunk g - 3, completed
-      // before S(g) was issued.
-      if (has) ptx::tmem_st32(sbase, pk);
       if (n == 0) {
         l_run = psum;
       } else {
