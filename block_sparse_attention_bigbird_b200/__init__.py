@@ -12,7 +12,7 @@ import importlib
 
 __all__ = ["bsa_layout_build", "bsa_layout_csr", "bsa_layout_globals", "bsa_layout_tiles",
            "bsa_layout_upload", "bsa_workspace_bytes", "bsa_forward", "bsa_sync_status",
-           "bsa_strerror", "bsa_debug_wait_timeout", "Layout", "BsaError"]
+           "bsa_strerror", "bsa_debug_wait_timeout", "bsa_forward_static_ws", "Layout", "BsaError"]
 
 
 def __getattr__(name):

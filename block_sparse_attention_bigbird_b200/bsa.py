@@ -23,6 +23,8 @@ BSA_ERR_LAYOUT_MISMATCH = -4
 BSA_ERR_DEVICE_TIMEOUT = -5
 BSA_ERR_OOM = -6
 BSA_ERR_WORKSPACE = -7
+BSA_ERR_STATIC_WORKSPACE = -8
+STATIC_WORKSPACE_BYTES = 32 * 1024 * 1024  # BSA_STATIC_WORKSPACE_BYTES in include/bsa.h
 
 # name -> (restype, argtypes); mirrors include/bsa.h
 _SIGNATURES = {
@@ -46,6 +48,10 @@ _SIGNATURES = {
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "bsa_forward_static_ws": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                             ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                             ctypes.c_void_p]),
     "bsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p]),
@@ -214,6 +220,30 @@ def bsa_forward(q, k, v, layout: Layout, key_mask=None, scale: Optional[float] =
                            lse.data_ptr(), workspace.data_ptr(), workspace.numel(),
                            ctypes.c_void_p(_stream_ptr(stream)))
     _check(code, "bsa_forward")
+    return out, lse
+
+
+def bsa_forward_static_ws(q, k, v, layout: Layout, key_mask=None, scale: Optional[float] = None,
+                          out=None, lse=None, stream=None):
+    """bsa_forward for callers that cannot allocate device memory.
+
+    The library's built-in scratch buffer (STATIC_WORKSPACE_BYTES per device)
+    replaces the workspace; nothing is allocated by the call itself (``out`` and
+    ``lse`` must then be given by such a caller).  Calls on one device share that
+    buffer: serialise them.  Raises BsaError(BSA_ERR_STATIC_WORKSPACE) when the
+    problem needs more scratch than the buffer holds.
+    """
+    import torch
+    B, H, L, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    code = lib.bsa_forward_static_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L, d, layout.handle,
+                                     key_mask.data_ptr() if key_mask is not None else None,
+                                     ctypes.c_float(scale if scale is not None else 0.0), out.data_ptr(),
+                                     lse.data_ptr(), ctypes.c_void_p(_stream_ptr(stream)))
+    _check(code, "bsa_forward_static_ws")
     return out, lse
 
 

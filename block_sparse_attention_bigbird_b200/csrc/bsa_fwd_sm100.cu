@@ -938,3 +938,53 @@ int bsa_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ allocation-free entry
+// Scratch of bsa_forward_static_ws: a file-scope device array, so that callers who
+// cannot allocate device memory can still run the forward.  In host code its name
+// is only a stand-in; the device address is looked up per device below.
+static __device__ __align__(256) unsigned char g_bsa_static_ws[BSA_STATIC_WORKSPACE_BYTES];
+
+namespace {
+void* g_static_ws_addr[kMaxDevices];
+cudaError_t g_static_ws_err[kMaxDevices];
+std::once_flag g_static_ws_once[kMaxDevices];
+}  // namespace
+
+extern "C" int bsa_forward_static_ws(const void* q, const void* k, const void* v, int B, int H, int L,
+                                     int d, const bsa_layout* lay, const uint8_t* key_mask, float scale,
+                                     void* out, float* lse, void* stream) {
+  // The checks bsa_forward makes before touching the GPU, repeated so that a bad
+  // call enqueues nothing (not even the ticket clear below).
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr ||
+      lay == nullptr || B < 1 || H < 1 || L < 1)
+    return BSA_ERR_INVALID_ARG;
+  if (d != kHeadDim) return BSA_ERR_UNSUPPORTED;
+  if (H != lay->H || L != lay->L) return BSA_ERR_LAYOUT_MISMATCH;
+  if (static_cast<int64_t>(B) * H * L > INT32_MAX - 64) return BSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return BSA_ERR_INVALID_ARG;
+  if (!(scale == scale) || std::isinf(scale)) return BSA_ERR_INVALID_ARG;
+  const WorkspacePlan plan = plan_workspace(*lay, B);
+  if (plan.total > BSA_STATIC_WORKSPACE_BYTES) return BSA_ERR_STATIC_WORKSPACE;
+  if (lay->device < 0) return BSA_ERR_LAYOUT_MISMATCH;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+  if (dev != lay->device) return BSA_ERR_LAYOUT_MISMATCH;
+  if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
+  DeviceInfo info;
+  const int st = device_setup(dev, &info);
+  if (st != BSA_OK) return st;
+  // once per device, with that device current: the array's address on it
+  std::call_once(g_static_ws_once[dev], [dev] {
+    g_static_ws_err[dev] = cudaGetSymbolAddress(&g_static_ws_addr[dev], g_bsa_static_ws);
+  });
+  if (g_static_ws_err[dev] != cudaSuccess || g_static_ws_addr[dev] == nullptr) return BSA_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(g_static_ws_addr[dev]);
+  // the arrival tickets must start at zero; the other regions are written before read
+  if (cudaMemsetAsync(ws + plan.tickets_off, 0, plan.tickets_bytes, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return BSA_ERR_CUDA;
+  return bsa_forward(q, k, v, B, H, L, d, lay, key_mask, scale, out, lse, ws, BSA_STATIC_WORKSPACE_BYTES,
+                     stream);
+}

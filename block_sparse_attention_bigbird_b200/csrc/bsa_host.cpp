@@ -371,6 +371,7 @@ const char* bsa_strerror(int status) {
     case BSA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
     case BSA_ERR_OOM: return "out of memory";
     case BSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case BSA_ERR_STATIC_WORKSPACE: return "problem needs more scratch than the built-in static workspace holds";
     default: return "unknown status";
   }
 }

@@ -51,7 +51,9 @@ typedef enum {
                                    to the current device                       */
   BSA_ERR_DEVICE_TIMEOUT = -5,  /* a bounded wait inside a kernel gave up      */
   BSA_ERR_OOM = -6,             /* host or device allocation failed            */
-  BSA_ERR_WORKSPACE = -7        /* workspace missing or too small              */
+  BSA_ERR_WORKSPACE = -7,       /* workspace missing or too small              */
+  BSA_ERR_STATIC_WORKSPACE = -8 /* problem needs more scratch than the library's
+                                   built-in buffer (bsa_forward_static_ws)     */
 } bsa_status;
 
 /* Opaque, immutable after bsa_layout_build (bsa_layout_upload only adds
@@ -153,6 +155,33 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
                 const bsa_layout* layout, const uint8_t* key_mask, float scale,
                 void* out, float* lse, void* workspace, size_t workspace_bytes,
                 void* stream);
+
+/*
+ * bsa_forward_static_ws -- bsa_forward for callers that cannot allocate device
+ * memory: code running where cudaMalloc is unavailable or forbidden, e.g. inside
+ * a host runtime that owns every allocation, a plugin with no allocator hook, or
+ * a path where an allocation would synchronise the device.  It allocates
+ * nothing: the scratch (split-row partials, their arrival tickets, key-padding
+ * bits) lives in one buffer of BSA_STATIC_WORKSPACE_BYTES (32 MiB) compiled into
+ * the library, which every GPU that loads the library holds until process exit.
+ * The pages define no such entry point; it has no counterpart there.
+ *
+ * Arguments and results are those of bsa_forward, minus the workspace.
+ *   - Returns BSA_ERR_STATIC_WORKSPACE, before anything is enqueued, when
+ *     bsa_workspace_bytes(layout, B) exceeds BSA_STATIC_WORKSPACE_BYTES.
+ *   - The first call on a device looks up the buffer's device address for that
+ *     device (cudaGetSymbolAddress, no allocation); make that first call before
+ *     any stream capture.
+ *   - Every call clears the buffer's ticket area with cudaMemsetAsync on
+ *     `stream`, then enqueues the forward.  All calls on a device share the one
+ *     buffer, which keeps the last call's contents: calls whose execution
+ *     overlaps on the GPU (different streams, no ordering between them) race on
+ *     it and give undefined results.  Serialise them.
+ */
+#define BSA_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
+int bsa_forward_static_ws(const void* q, const void* k, const void* v, int B, int H, int L, int d,
+                          const bsa_layout* layout, const uint8_t* key_mask, float scale,
+                          void* out, float* lse, void* stream);
 
 /*
  * bsa_sync_status -- synchronises `stream`, then returns and clears the
