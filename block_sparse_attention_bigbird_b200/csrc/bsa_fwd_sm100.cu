@@ -8,23 +8,25 @@
 // per-tile list of 64-key blocks ("SQA 稀疏注意力机制详解" 3.1: block-sparse mask,
 // attention only on non-zero blocks).
 //
-// Kernel design (one persistent CTA per SM, 352 threads):
-//   warp 8      TMA producer: Q tile (2 x 64 rows), then K and V of two key blocks per
+// Kernel design: one persistent CTA per SM (448 threads) running two independent
+// pipelines ("slots") side by side, each with its own work items, shared-memory
+// rings, barriers and 256 TMEM columns.  The ex2 unit (16 results per clock per
+// SM) bounds this d = 64 forward; with two slots one softmax warpgroup runs its
+// exponentials while the other is between chunks, so their phases interleave
+// instead of running in lockstep.  Slot s (0 or 1) has:
+//   warps 4s..4s+3  softmax + epilogue: thread (warp w, lane l) owns tile row
+//               r = 32 (w % 4) + l = TMEM lane r, keeps the running max m and sum l
+//               (fp32), writes P (bf16) over the S columns it has read, and raises
+//               m (rescaling l and O) only when a chunk's p would outgrow 2^12.
+//   warp 8+s    TMA producer: Q tile (2 x 64 rows), then K and V of one key block per
 //               chunk of the tile's key-block union into a K ring (released when the
 //               chunk's S is done) and a deeper V ring (released after its PV).
-//   warp 9      tcgen05 S issuer: S = Q K^T (M=128, N=64|128, K=64) into one of three
-//               TMEM S buffers.
-//   warp 10     tcgen05 PV issuer: per key block O_x += P_x V_x (A = P from TMEM, M=128,
-//               N=64, K=64) into that block's own accumulator.  Two issuing threads
-//               keep the tensor pipe fed: each tcgen05 instruction, barrier wait and
-//               commit blocks its thread, and d = 64 makes every MMA short.
-//   warps 0-7   softmax + epilogue, two warpgroups.  Warpgroup x (warps 4x..4x+3)
-//               handles key block x of every chunk: thread (warp w, lane l) owns tile
-//               row r = 32 (w % 4) + l = TMEM lane r.  Each warpgroup keeps its own
-//               running max m_x and sum l_x (fp32) and its own O_x accumulator, writes
-//               P_x (bf16) over its half of S, and rescales O_x when m_x grows by more
-//               than kRescaleLog2.  The epilogue merges (m_A, l_A, O_A) and
-//               (m_B, l_B, O_B); each warpgroup finishes 32 of the 64 output columns.
+//   warp 10+2s  tcgen05 S issuer: S = Q K^T (M=128, N=64, K=64) into one of three
+//               TMEM S buffers (warp 10 also allocates and frees TMEM).
+//   warp 11+2s  tcgen05 PV issuer: O += P V (A = P from TMEM, M=128, N=64, K=64).
+//               Two issuing threads per slot keep the tensor pipe fed: each tcgen05
+//               instruction, barrier wait and commit blocks its thread, and d = 64
+//               makes every MMA short.
 // A tile is two query blocks of the same (b, h) over the sorted union of their rows;
 // entries carry per-block membership bits so each half of the tile sees exactly its
 // own row, and a warp whose half does not attend a block skips its exponentials.
@@ -46,51 +48,86 @@
 
 namespace bsa {
 
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;  // S issuer; also allocates and frees TMEM
-constexpr int kPvWarp = 10;
-constexpr int kThreads = 352;
+constexpr int kSlots = 2;
+constexpr int kProducerWarp = 8;  // + slot
+constexpr int kMmaWarp = 10;      // + 2 slot: S issuer; warp 10 allocates and frees TMEM
+constexpr int kPvWarp = 11;       // + 2 slot
+constexpr int kThreads = 448;
+constexpr int kSoftmaxThreads = 128;  // per slot
+constexpr int kItemRing = 4;  // work-item indices a slot's producer may publish ahead
 constexpr int kKStages = 3;  // == kSBufs: K stage g % 3 is free once S(g) is done
 constexpr int kVStages = 5;  // V stage g % 5 is free once PV(g) is done
-constexpr uint32_t kBlkBytes = 64 * 128;         // one 64 x 64 bf16 block
-constexpr uint32_t kQBytes = 2 * kBlkBytes;      // 128-row Q tile
-constexpr uint32_t kStageBytes = 2 * kBlkBytes;  // two key blocks
+constexpr uint32_t kBlkBytes = 64 * 128;     // one 64 x 64 bf16 block
+constexpr uint32_t kQBytes = 2 * kBlkBytes;  // 128-row Q tile
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSBufs = 3;    // S buffers of 128 columns at [0,128), [128,256), [256,384)
+constexpr uint32_t kSlotCols = 256;          // slot s owns columns [256 s, 256 s + 256)
+constexpr uint32_t kSBufs = 3;               // S buffers of 64 columns at +0, +64, +128
 constexpr uint32_t kTmemS = 0;
-constexpr uint32_t kTmemO = 384;  // O_A [384,448), O_B [448,512)
-constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kTmemO = 192;             // O at +192
+constexpr float kLazyBound = 4096.0f;  // 2^kLazyLog2, kLazyLog2 = 12: bound on a chunk's sum of p
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 constexpr uint32_t kMaxSpin = 1u << 24;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 constexpr uint32_t kWaitSleepNs = 20000;  // upper bound on one sleep inside a barrier wait
 
-// shared memory map (offsets from a 1024-aligned base)
+// shared memory map of one slot (offsets from its 1024-aligned base)
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + 2 * kQBytes;
-constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
-constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
+constexpr uint32_t kSmemV = kSmemK + kKStages * kBlkBytes;
+constexpr uint32_t kSmemBar = kSmemV + kVStages * kBlkBytes;
 enum : int {
   kBarQFull = 0,
   kBarQEmpty = 2,
   kBarKFull = 4,                          // [K stage] K of the stage landed (TMA)
   kBarVFull = kBarKFull + kKStages,       // [V stage] V of the stage landed (TMA)
   kBarVFree = kBarVFull + kVStages,       // [V stage] MMA commit after the chunk's PV: the V
-                                          // stage is reusable and both O_x hold that chunk
+                                          // stage is reusable and O holds that chunk
   kBarSFull = kBarVFree + kVStages,       // [S buffer] MMA commit after S: S readable, and
                                           // the K stage of the same index reusable
-  kBarPFull = kBarSFull + kSBufs,         // [S buffer] both warpgroups' P written, 256 arrivals
-  kBarOFree = kBarPFull + kSBufs,         // 256 arrivals once the epilogue has read O
+  kBarPFull = kBarSFull + kSBufs,         // [S buffer] P written, 128 arrivals
+  kBarOFree = kBarPFull + kSBufs,         // 128 arrivals once the epilogue has read O
   kBarMmaFinal = kBarOFree + 1,           // [2 issuers]
-  kBarEpi = kBarMmaFinal + 2,        // 256 softmax threads, epilogue rendezvous
-  kNumBars = kBarEpi + 1
+  kBarEpi = kBarMmaFinal + 2,             // 128 softmax threads, split-record rendezvous
+  kBarItemFull = kBarEpi + 1,             // [item ring] the producer published a work item
+  kBarItemEmpty = kBarItemFull + kItemRing,  // [item ring] 6 arrivals: both issuers and the
+                                             // four softmax warps have read it
+  kNumBars = kBarItemEmpty + kItemRing
 };
-constexpr uint32_t kSmemMisc = kSmemBar + 8 * kNumBars;
-constexpr uint32_t kSmemXch = (kSmemMisc + 16 + 15) & ~15u;  // [2 tile parity][2 wg][2 (m,l)][128] fp32
-constexpr uint32_t kSmemUsed = kSmemXch + 2 * 2 * 2 * kTileRows * 4;
+constexpr uint32_t kItemReaders = 6;
+
+// One published work item in shared memory: its index, its fields, its query-block
+// pair and, per union entry, the entry and the key-padding bits of its key block.
+constexpr int kMaxItemEntries = 64;
+static_assert(kSplitThreshold <= kMaxItemEntries && kSplitChunk <= kMaxItemEntries,
+              "an item's entries must fit its stage");
+struct ItemStage {
+  int t;  // work item index, or kItemNone
+  int qa, qb;
+  int b;
+  int pad[4];
+  WorkItem w;
+  uint32_t ent[kMaxItemEntries];
+  unsigned long long kb[kMaxItemEntries];  // all ones without a key mask
+};
+static_assert(sizeof(ItemStage) % 16 == 0, "stage alignment");
+constexpr uint32_t kSmemItems = (kSmemBar + 8 * kNumBars + 15) & ~15u;  // ItemStage[kItemRing]
+constexpr uint32_t kSmemLast = kSmemItems + sizeof(ItemStage) * kItemRing;  // u32: last arriver flag
+constexpr uint32_t kSlotBytes = (kSmemLast + 4 + 1023) & ~1023u;
+constexpr uint32_t kSmemMisc = kSlots * kSlotBytes;          // u32 TMEM base, int abort flag
+constexpr uint32_t kSmemUsed = kSmemMisc + 16;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+
+// Where one slot's roles find their resources.  Work items are handed out
+// dynamically: the slot's producer takes the next index from a global counter and
+// publishes it to the slot's other roles through a small ring in shared memory.
+struct Slot {
+  uint32_t sQ, sK, sV, bars;
+  ItemStage* items;  // the item ring
+  volatile uint32_t* last_flag;
+  uint32_t tmem;  // TMEM address of the slot's column 0
+};
 
 struct FwdParams {
   CUtensorMap tm_q, tm_k, tm_v;
@@ -101,6 +138,7 @@ struct FwdParams {
   const uint32_t* pair_ent;
   const unsigned long long* keybits;  // [B, nb] or null
   float* partials;
+  int* sched;    // [0] next work item, [1] slots finished; zero between calls
   int* tickets;
   int B, H, L, nb, items_per_batch, n_split, n_records;
   float scale_log2;
@@ -155,61 +193,140 @@ __device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile
   return wait_slow(bar, parity, abort_flag, timeout_ns, true);
 }
 
-// TMA producer, one thread: Q tile, then for each chunk c its K into K stage c % 3
-// (once S(c - 3) is done) and its V into V stage c % 5 (once PV(c - 5) is done).
-__device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sQ, uint32_t sK,
-                                              uint32_t sV, uint32_t bars, volatile int* abort_flag) {
+constexpr int kItemNone = -1;   // no work left
+constexpr int kItemAbort = -2;  // a wait gave up
+
+// The slot's k-th work item for an issuer (one thread): its index and entry count.
+// The stage is released at once.
+__device__ __forceinline__ int take_item_one(const Slot& sl, uint32_t k, int* count, volatile int* abort_flag,
+                                             uint64_t timeout_ns) {
+  const uint32_t i = k % kItemRing;
+  if (!wait_one(sl.bars + 8u * (kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
+    return kItemAbort;
+  const ItemStage& st = sl.items[i];
+  const int t = st.t;
+  *count = st.w.count;
+  ptx::mbar_arrive(sl.bars + 8u * (kBarItemEmpty + i));
+  return t;
+}
+
+// The slot's k-th work item for a softmax warp, which keeps reading its stage until
+// the item's epilogue and then releases it (release_item_warp).
+__device__ __forceinline__ int take_item_warp(const Slot& sl, uint32_t k, volatile int* abort_flag,
+                                              uint64_t timeout_ns) {
+  const uint32_t i = k % kItemRing;
+  if (!wait_warp(sl.bars + 8u * (kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
+    return kItemAbort;
+  return sl.items[i].t;
+}
+
+__device__ __forceinline__ void release_item_warp(const Slot& sl, uint32_t k, int lane) {
+  __syncwarp();
+  if (lane == 0) ptx::mbar_arrive(sl.bars + 8u * (kBarItemEmpty + k % kItemRing));
+}
+
+// TMA producer, one warp.  Per work item the warp stages the item, its union
+// entries and their key-padding bits in the slot's item ring; then lane 0 issues
+// the loads: the Q tile, and for each chunk g (one key block) its K into K stage
+// g % 3 (once S(g - 3) is done) and its V into V stage g % 5 (once PV(g - 5) is
+// done).
+__device__ __forceinline__ void producer_role(const FwdParams& p, const Slot& sl, int lane,
+                                              volatile int* abort_flag) {
+  const uint32_t sQ = sl.sQ, sK = sl.sK, sV = sl.sV, bars = sl.bars;
   static_assert(kKStages == static_cast<int>(kSBufs), "K stages are released by the S-full commits");
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   const uint64_t pol_q = ptx::policy_evict_first();
   const uint64_t pol_kv = ptx::policy_evict_last();
   const int total = p.B * p.items_per_batch;
-  uint32_t nq = 0, nk = 0, nv = 0;  // Q tiles, K chunks, V chunks issued
+  uint32_t nq = 0, nk = 0, nv = 0;  // Q tiles, K blocks, V blocks issued (lane 0)
   bool alive = true;
-  for (int t = blockIdx.x; alive && t < total; t += gridDim.x) {
-    const int b = t / p.items_per_batch;
-    const WorkItem w = p.items[t - b * p.items_per_batch];
-    const int row0 = (b * p.H + w.h) * p.L;
-    const int qa = p.pair_q[2 * w.pair], qb = p.pair_q[2 * w.pair + 1];
-    const uint32_t qs = nq & 1u;
-    if (!wait_one(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+  int t_next = lane == 0 ? atomicAdd(p.sched, 1) : 0;
+  for (uint32_t k = 0;; ++k) {
+    t_next = __shfl_sync(0xffffffffu, t_next, 0);
+    const int t = t_next < total ? t_next : kItemNone;
+    const uint32_t ii = k % kItemRing;
+    bool ok = true;
+    if (lane == 0)
+      ok = wait_one(bar(kBarItemEmpty + static_cast<int>(ii)), ((k / kItemRing) & 1u) ^ 1u, abort_flag,
+                    p.timeout_ns);
+    if (!__shfl_sync(0xffffffffu, ok, 0)) {
       alive = false;
       break;
     }
-    ptx::mbar_arrive_expect_tx(bar(kBarQFull + qs), kQBytes);
-    ptx::tma_load_2d(sQ + qs * kQBytes, &p.tm_q, bar(kBarQFull + qs), 0, row0 + qa * 64, pol_q);
-    ptx::tma_load_2d(sQ + qs * kQBytes + kBlkBytes, &p.tm_q, bar(kBarQFull + qs), 0,
-                     row0 + (qb >= 0 ? qb : qa) * 64, pol_q);
-    ++nq;
-    const uint32_t* ent = p.pair_ent + w.start;
-    for (int e = 0; e < w.count; e += 2) {
-      const int j0 = static_cast<int>(ent[e] & kEntColMask);
-      const bool two = e + 1 < w.count;
-      const int j1 = two ? static_cast<int>(ent[e + 1] & kEntColMask) : 0;
-      const uint32_t bytes = two ? 2 * kBlkBytes : kBlkBytes;
-      const uint32_t ks = nk % kKStages;
-      if (!wait_one(bar(kBarSFull + ks), ((nk / kKStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
-        alive = false;
-        break;
+    // stage the item for the slot's other roles
+    ItemStage& st = sl.items[ii];
+    if (t >= 0) {
+      // t enumerates (item, batch element) item-major: the items' order holds for
+      // the whole batch
+      const int i = t / p.B, b = t - i * p.B;
+      const WorkItem w = p.items[i];
+      for (int e = lane; e < w.count; e += 32) {
+        const uint32_t en = p.pair_ent[w.start + e];
+        st.ent[e] = en;
+        st.kb[e] = p.keybits != nullptr ? p.keybits[static_cast<size_t>(b) * p.nb + (en & kEntColMask)] : ~0ull;
       }
-      const uint32_t dk = sK + ks * kStageBytes;
-      ptx::mbar_arrive_expect_tx(bar(kBarKFull + ks), bytes);
-      ptx::tma_load_2d(dk, &p.tm_k, bar(kBarKFull + ks), 0, row0 + j0 * 64, pol_kv);
-      if (two) ptx::tma_load_2d(dk + kBlkBytes, &p.tm_k, bar(kBarKFull + ks), 0, row0 + j1 * 64, pol_kv);
-      ++nk;
-      const uint32_t vs = nv % kVStages;
-      if (!wait_one(bar(kBarVFree + vs), ((nv / kVStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
-        alive = false;
-        break;
+      if (lane == 0) {
+        st.w = w;
+        st.b = b;
+        st.qa = p.pair_q[2 * w.pair];
+        st.qb = p.pair_q[2 * w.pair + 1];
       }
-      const uint32_t dv = sV + vs * kStageBytes;
-      ptx::mbar_arrive_expect_tx(bar(kBarVFull + vs), bytes);
-      ptx::tma_load_2d(dv, &p.tm_v, bar(kBarVFull + vs), 0, row0 + j0 * 64, pol_kv);
-      if (two) ptx::tma_load_2d(dv + kBlkBytes, &p.tm_v, bar(kBarVFull + vs), 0, row0 + j1 * 64, pol_kv);
-      ++nv;
+    }
+    if (lane == 0) st.t = t;
+    __threadfence_block();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar(kBarItemFull + static_cast<int>(ii)));
+    if (t < 0) break;
+    if (lane == 0) {
+      t_next = atomicAdd(p.sched, 1);  // the next item's index arrives while this tile loads
+      const WorkItem& w = st.w;
+      const int row0 = (st.b * p.H + w.h) * p.L;
+      const int qa = st.qa, qb = st.qb;
+      const uint32_t qs = nq & 1u;
+      if (!wait_one(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+        alive = false;
+      } else {
+        ptx::mbar_arrive_expect_tx(bar(kBarQFull + qs), kQBytes);
+        ptx::tma_load_2d(sQ + qs * kQBytes, &p.tm_q, bar(kBarQFull + qs), 0, row0 + qa * 64, pol_q);
+        ptx::tma_load_2d(sQ + qs * kQBytes + kBlkBytes, &p.tm_q, bar(kBarQFull + qs), 0,
+                         row0 + (qb >= 0 ? qb : qa) * 64, pol_q);
+        ++nq;
+        for (int e = 0; e < w.count; ++e) {
+          const int j = static_cast<int>(st.ent[e] & kEntColMask);
+          const uint32_t ks = nk % kKStages;
+          if (!wait_one(bar(kBarSFull + ks), ((nk / kKStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+            alive = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(bar(kBarKFull + ks), kBlkBytes);
+          ptx::tma_load_2d(sK + ks * kBlkBytes, &p.tm_k, bar(kBarKFull + ks), 0, row0 + j * 64, pol_kv);
+          ++nk;
+          const uint32_t vs = nv % kVStages;
+          if (!wait_one(bar(kBarVFree + vs), ((nv / kVStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+            alive = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(bar(kBarVFull + vs), kBlkBytes);
+          ptx::tma_load_2d(sV + vs * kBlkBytes, &p.tm_v, bar(kBarVFull + vs), 0, row0 + j * 64, pol_kv);
+          ++nv;
+        }
+      }
+    }
+    if (!__shfl_sync(0xffffffffu, alive, 0)) {
+      alive = false;
+      break;
     }
   }
-  if (!alive) {
+  if (lane != 0) return;
+  if (alive) {
+    // Every slot's producer counts itself out once it has drawn its last index; the
+    // last one resets both counters for the next call.
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1) == kSlots * static_cast<int>(gridDim.x) - 1) {
+      p.sched[0] = 0;
+      p.sched[1] = 0;
+    }
+  } else {
     // Aborted: let every copy this thread issued land before the CTA exits.  The
     // last issue into ring slot s had index s + R * floor((n - 1 - s) / R).
     auto drain = [&](int first_bar, uint32_t n, uint32_t ring) {
@@ -229,25 +346,22 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, uint32_t sQ, u
 // tcgen05 S issuer, one thread.  S(g) = Q K_g^T into S buffer g % 3 once K(g) has
 // landed and PV(g - 3), the previous reader of that buffer, is done.  Its commit
 // also releases K stage g % 3 to the producer.
-__device__ __forceinline__ void s_issuer(const FwdParams& p, uint32_t sQ, uint32_t sK, uint32_t bars,
-                                         uint32_t tmem, volatile int* abort_flag) {
+__device__ __forceinline__ void s_issuer(const FwdParams& p, const Slot& sl, volatile int* abort_flag) {
+  const uint32_t sQ = sl.sQ, sK = sl.sK, bars = sl.bars, tmem = sl.tmem;
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  constexpr uint32_t kIdescS128 = ptx::idesc_bf16_f32(128, 128, false);
-  constexpr uint32_t kIdescS64 = ptx::idesc_bf16_f32(128, 64, false);
+  constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, false);
   // descriptor start-address fields count 16-byte units
   const uint64_t dq0 = ptx::smem_desc_sw128(sQ, 16);
   const uint64_t dk0 = ptx::smem_desc_sw128(sK, 16);
-  const int total = p.B * p.items_per_batch;
-  uint32_t g = 0, nq = 0;
+  uint32_t g = 0;
   bool alive = true;
-  for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nq) {
-    const int b = t / p.items_per_batch;
-    const WorkItem w = p.items[t - b * p.items_per_batch];
+  for (uint32_t nq = 0; alive; ++nq) {
+    int count = 0;
+    if (take_item_one(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
     const uint32_t qs = nq & 1u;
     if (!wait_one(bar(kBarQFull + qs), (nq >> 1) & 1u, abort_flag, p.timeout_ns)) break;
     const uint64_t dq = dq0 + qs * (kQBytes >> 4);
-    const int nch = (w.count + 1) >> 1;
-    for (int n = 0; n < nch; ++n, ++g) {
+    for (int n = 0; n < count; ++n, ++g) {
       const uint32_t ks = g % kKStages;
       if (!wait_one(bar(kBarKFull + ks), (g / kKStages) & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
@@ -261,16 +375,14 @@ __device__ __forceinline__ void s_issuer(const FwdParams& p, uint32_t sQ, uint32
         }
       }
       ptx::tc_fence_after();
-      const bool two = 2 * n + 1 < w.count;
-      const uint64_t dk = dk0 + ks * (kStageBytes >> 4);
-      const uint32_t d = tmem + kTmemS + (g % kSBufs) * 128u;
-      const uint32_t id = two ? kIdescS128 : kIdescS64;
-      ptx::mma_ss(d, dq, dk, id, 0u);  // head dim 64 = 4 x 16: +32 bytes per step
-      ptx::mma_ss(d, dq + 2, dk + 2, id, 1u);
-      ptx::mma_ss(d, dq + 4, dk + 4, id, 1u);
-      ptx::mma_ss(d, dq + 6, dk + 6, id, 1u);
+      const uint64_t dk = dk0 + ks * (kBlkBytes >> 4);
+      const uint32_t d = tmem + kTmemS + (g % kSBufs) * 64u;
+      ptx::mma_ss(d, dq, dk, kIdescS, 0u);  // head dim 64 = 4 x 16: +32 bytes per step
+      ptx::mma_ss(d, dq + 2, dk + 2, kIdescS, 1u);
+      ptx::mma_ss(d, dq + 4, dk + 4, kIdescS, 1u);
+      ptx::mma_ss(d, dq + 6, dk + 6, kIdescS, 1u);
       ptx::mma_commit(bar(kBarSFull + g % kSBufs));
-      if (n == nch - 1) ptx::mma_commit(bar(kBarQEmpty + qs));
+      if (n == count - 1) ptx::mma_commit(bar(kBarQEmpty + qs));
     }
   }
   // Every MMA this thread issued must finish before TMEM is released.
@@ -278,24 +390,21 @@ __device__ __forceinline__ void s_issuer(const FwdParams& p, uint32_t sQ, uint32
   wait_force(bar(kBarMmaFinal), 0, abort_flag, p.timeout_ns);
 }
 
-// tcgen05 PV issuer, one thread.  Chunk g: once V(g) has landed and both warpgroups
-// have written P(g), O_x (+)= P_x V_x for the chunk's key blocks, then one commit
-// that frees V stage g % 5, tells the S issuer S buffer g % 3 is free, and tells the
-// softmax warps that O holds chunk g.  A tile's first PV waits until the previous
-// tile's epilogue has read O.
-__device__ __forceinline__ void pv_issuer(const FwdParams& p, uint32_t sV, uint32_t bars, uint32_t tmem,
-                                          volatile int* abort_flag) {
+// tcgen05 PV issuer, one thread.  Chunk g: once V(g) has landed and the softmax has
+// written P(g), O (+)= P V, then one commit that frees V stage g % 5, tells the S
+// issuer S buffer g % 3 is free, and tells the softmax warps that O holds chunk g.
+// A tile's first PV waits until the previous tile's epilogue has read O.
+__device__ __forceinline__ void pv_issuer(const FwdParams& p, const Slot& sl, volatile int* abort_flag) {
+  const uint32_t sV = sl.sV, bars = sl.bars, tmem = sl.tmem;
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 64, true);
   const uint64_t dv0 = ptx::smem_desc_sw128(sV, 0);
-  const int total = p.B * p.items_per_batch;
-  uint32_t g = 0, nq = 0;
+  uint32_t g = 0;
   bool alive = true;
-  for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nq) {
-    const int b = t / p.items_per_batch;
-    const WorkItem w = p.items[t - b * p.items_per_batch];
-    const int nch = (w.count + 1) >> 1;
-    for (int n = 0; n < nch; ++n, ++g) {
+  for (uint32_t nq = 0; alive; ++nq) {
+    int count = 0;
+    if (take_item_one(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
+    for (int n = 0; n < count; ++n, ++g) {
       if (n == 0 && !wait_one(bar(kBarOFree), (nq & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
@@ -307,18 +416,14 @@ __device__ __forceinline__ void pv_issuer(const FwdParams& p, uint32_t sV, uint3
         break;
       }
       ptx::tc_fence_after();
-      const bool two = 2 * n + 1 < w.count;
       const uint32_t acc0 = n == 0 ? 0u : 1u;
-      const uint64_t dv = dv0 + vs * (kStageBytes >> 4);
-      for (uint32_t x = 0; x < (two ? 2u : 1u); ++x) {
-        const uint32_t d = tmem + kTmemO + x * 64u;
-        const uint32_t a = tmem + kTmemS + sb * 128u + x * 64u;
-        const uint64_t bx = dv + x * (kBlkBytes >> 4);
-        ptx::mma_ts(d, a, bx, kIdescPV, acc0);  // 16 keys per MMA
-        ptx::mma_ts(d, a + 8u, bx + (2048u >> 4), kIdescPV, 1u);
-        ptx::mma_ts(d, a + 16u, bx + (4096u >> 4), kIdescPV, 1u);
-        ptx::mma_ts(d, a + 24u, bx + (6144u >> 4), kIdescPV, 1u);
-      }
+      const uint64_t dv = dv0 + vs * (kBlkBytes >> 4);
+      const uint32_t d = tmem + kTmemO;
+      const uint32_t a = tmem + kTmemS + sb * 64u;
+      ptx::mma_ts(d, a, dv, kIdescPV, acc0);  // 16 keys per MMA
+      ptx::mma_ts(d, a + 8u, dv + (2048u >> 4), kIdescPV, 1u);
+      ptx::mma_ts(d, a + 16u, dv + (4096u >> 4), kIdescPV, 1u);
+      ptx::mma_ts(d, a + 24u, dv + (6144u >> 4), kIdescPV, 1u);
       ptx::mma_commit(bar(kBarVFree + vs));
     }
   }
@@ -334,24 +439,89 @@ __device__ __forceinline__ void mask_cols(float (&s)[64], unsigned long long mk)
 }
 
 // What the epilogue of a finished tile needs; it runs one chunk later (after the
-// first chunk of the next tile) so the wait for the tile's last PV is hidden.  The
-// epilogue's 256-thread rendezvous is an mbarrier with a bounded wait (a plain
-// bar.sync could not give up if another softmax warp had already aborted).
+// first chunk of the next tile) so the wait for the tile's last PV is hidden.
 struct TileDone {
-  int t;            // work item index (its fields are reloaded by the epilogue)
+  uint32_t k;       // the item's position in the slot's item sequence (its stage: k % ring)
   uint32_t g_last;  // global index of the tile's last chunk
-  uint32_t nt;      // tile count of this CTA when the tile started
-  float m, l;       // this warpgroup's running max (log2 units) and sum for the row
+  float m, l;       // the row's running max (log2 units) and sum
 };
 
-// Epilogue of a finished tile: merge (m_A, l_A, O_A) with (m_B, l_B, O_B), store O
-// and lse (or the split chunk's partial record, merging when last).  Kept out of
-// line: it runs once per tile and would otherwise crowd the chunk loop's registers.
-__device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& td, uint32_t bars,
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst_row, const float* o, float inv) {
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+  for (int v8 = 0; v8 < 8; ++v8) {
+    uint4 u;
+    u.x = pack_bf16x2(o[v8 * 8 + 0] * inv, o[v8 * 8 + 1] * inv);
+    u.y = pack_bf16x2(o[v8 * 8 + 2] * inv, o[v8 * 8 + 3] * inv);
+    u.z = pack_bf16x2(o[v8 * 8 + 4] * inv, o[v8 * 8 + 5] * inv);
+    u.w = pack_bf16x2(o[v8 * 8 + 6] * inv, o[v8 * 8 + 7] * inv);
+    dst[v8] = u;
+  }
+}
+
+// The last-arriving chunk of a split tile merges the tile's partial records into
+// row `row` of O and lse.  Out of line: it runs once per split tile.
+__device__ __noinline__ void merge_split_row(const FwdParams& p, const WorkItem& tw, int tb, int r, size_t row) {
+  // The max over the records, then the sums of l and O with record c weighted by
+  // 2^(m_c - max); a record whose row attended nothing has m = -inf, O = 0 and
+  // weight 0.  The record loop is unrolled so that loads of several records are
+  // in flight together.
+  const float* base = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec_base) * kRecFloats;
+  const int nc = tw.nchunks;
+  constexpr int kM = kTileRows * 64, kL = kTileRows * 64 + kTileRows;
+  float ms = -INFINITY;
+#pragma unroll 8
+  for (int c = 0; c < nc; ++c) ms = fmaxf(ms, __ldcg(base + static_cast<size_t>(c) * kRecFloats + kM + r));
+  float lsum = 0.f;
+#pragma unroll 8
+  for (int c = 0; c < nc; ++c) {
+    const float* rc = base + static_cast<size_t>(c) * kRecFloats;
+    const float mc = __ldcg(rc + kM + r);
+    lsum += mc == -INFINITY ? 0.f : __ldcg(rc + kL + r) * ptx::ex2_approx(mc - ms);
+  }
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll 1
+  for (int hh = 0; hh < 2; ++hh) {  // output columns [32 hh, 32 hh + 32)
+    float acc[32];
+#pragma unroll
+    for (int x = 0; x < 32; ++x) acc[x] = 0.f;
+#pragma unroll 2
+    for (int c = 0; c < nc; ++c) {
+      const float* rc = base + static_cast<size_t>(c) * kRecFloats;
+      float4 x[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) x[v] = __ldcg(reinterpret_cast<const float4*>(rc + r * 64 + 32 * hh) + v);
+      const float mc = __ldcg(rc + kM + r);
+      const float f = mc == -INFINITY ? 0.f : ptx::ex2_approx(mc - ms);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        acc[4 * v + 0] += f * x[v].x;
+        acc[4 * v + 1] += f * x[v].y;
+        acc[4 * v + 2] += f * x[v].z;
+        acc[4 * v + 3] += f * x[v].w;
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64 + 32 * hh);
+#pragma unroll
+    for (int v8 = 0; v8 < 4; ++v8) {
+      uint4 u;
+      u.x = pack_bf16x2(acc[v8 * 8 + 0] * inv, acc[v8 * 8 + 1] * inv);
+      u.y = pack_bf16x2(acc[v8 * 8 + 2] * inv, acc[v8 * 8 + 3] * inv);
+      u.z = pack_bf16x2(acc[v8 * 8 + 4] * inv, acc[v8 * 8 + 5] * inv);
+      u.w = pack_bf16x2(acc[v8 * 8 + 6] * inv, acc[v8 * 8 + 7] * inv);
+      dst[v8] = u;
+    }
+  }
+  p.lse[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
+}
+
+// Epilogue of a finished tile: normalise O and store it with lse (or the split
+// chunk's partial record, merging when last).  Kept out of line: it runs once per
+// tile and would otherwise crowd the chunk loop's registers.
+__device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& td, const ItemStage& st, uint32_t bars,
                                            uint32_t obase, int warp, int lane, volatile int* abort_flag,
-                                           volatile uint32_t* last_flag, float* xch, uint32_t* n_epi) {
+                                           volatile uint32_t* last_flag, uint32_t* n_epi) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  const int wg = warp >> 2;
   const int r = (warp & 3) * 32 + lane;
   const int half = r >> 6;
   auto epi_sync = [&]() -> bool {
@@ -360,234 +530,133 @@ __device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& t
     ++*n_epi;
     return ok;
   };
+  const int tb = st.b;
+  const WorkItem& tw = st.w;
+  const int tqa = st.qa, tqb = st.qb;
+  const int tbh = tb * p.H + tw.h;
+  // PV of the tile's last chunk.  Unambiguous phase: S(g_last) was seen, and it was
+  // issued after PV(g_last - 3) was done; PV(g_last + kVStages) needs P this warp
+  // has not produced.
+  if (!wait_warp(bar(kBarVFree + static_cast<int>(td.g_last % kVStages)), (td.g_last / kVStages) & 1u,
+                 abort_flag, p.timeout_ns))
+    return false;
+  ptx::tc_fence_after();
+  float o[64];
   {
-    const int tb = td.t / p.items_per_batch;
-    const WorkItem tw = p.items[td.t - tb * p.items_per_batch];
-    const int tqa = p.pair_q[2 * tw.pair], tqb = p.pair_q[2 * tw.pair + 1];
-    const int tbh = tb * p.H + tw.h;
-    // PV of the tile's last chunk.  Unambiguous phase: S(g_last) was seen, and it
-    // was issued after PV(g_last - 3) was done; PV(g_last + kVStages) needs P this
-    // warpgroup has not produced.
-    if (!wait_warp(bar(kBarVFree + static_cast<int>(td.g_last % kVStages)), (td.g_last / kVStages) & 1u,
-                   abort_flag, p.timeout_ns))
-      return false;
-    // (m, l) exchange, double-buffered by tile parity: a warpgroup that runs ahead
-    // into the next tile cannot overwrite values the other has not read yet.
-    float* xt = xch + (td.nt & 1u) * (2 * 2 * kTileRows);
-    xt[(wg * 2 + 0) * kTileRows + r] = td.m;
-    xt[(wg * 2 + 1) * kTileRows + r] = td.l;
-    if (!epi_sync()) return false;
-    ptx::tc_fence_after();
-    const float m_o = xt[((1 - wg) * 2 + 0) * kTileRows + r];
-    const float l_o = xt[((1 - wg) * 2 + 1) * kTileRows + r];
-    const float mA = wg == 0 ? td.m : m_o, lA = wg == 0 ? td.l : l_o;
-    const float mB = wg == 0 ? m_o : td.m, lB = wg == 0 ? l_o : td.l;
-    const float m = fmaxf(mA, mB);
-    const bool useA = lA > 0.f, useB = lB > 0.f;  // an unused O_x may hold stale values
-    const float fA = useA ? ptx::ex2_approx(mA - m) : 0.f;
-    const float fB = useB ? ptx::ex2_approx(mB - m) : 0.f;
-    const float l = lA * fA + lB * fB;
-    // this warpgroup finishes output columns [32 wg, 32 wg + 32)
-    uint32_t oa[32], ob[32];
-    ptx::tmem_ld32(obase + static_cast<uint32_t>(wg) * 32u, oa);
-    ptx::tmem_ld32(obase + 64u + static_cast<uint32_t>(wg) * 32u, ob);
+    uint32_t raw[2][32];
+    ptx::tmem_ld32(obase, raw[0]);
+    ptx::tmem_ld32(obase + 32u, raw[1]);
     ptx::tmem_wait_ld();
-    ptx::reg_fence(oa);
-    ptx::reg_fence(ob);
-    ptx::tc_fence_before();
-    ptx::mbar_arrive(bar(kBarOFree));  // O may now be overwritten by the next tile
-    float o[32];
+    ptx::reg_fence(raw[0]);
+    ptx::reg_fence(raw[1]);
 #pragma unroll
-    for (int c = 0; c < 32; ++c) {
-      const float a = useA ? __uint_as_float(oa[c]) * fA : 0.f;
-      const float bb = useB ? __uint_as_float(ob[c]) * fB : 0.f;
-      o[c] = a + bb;
-    }
-    const bool row_active = half == 0 || tqb >= 0;
-    const int qblk = half ? tqb : tqa;
-    const size_t row = static_cast<size_t>(tbh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
-    if (tw.split < 0) {
-      if (row_active) {
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64 + wg * 32);
-#pragma unroll
-        for (int v8 = 0; v8 < 4; ++v8) {
-          uint4 u;
-          u.x = pack_bf16x2(o[v8 * 8 + 0] * inv, o[v8 * 8 + 1] * inv);
-          u.y = pack_bf16x2(o[v8 * 8 + 2] * inv, o[v8 * 8 + 3] * inv);
-          u.z = pack_bf16x2(o[v8 * 8 + 4] * inv, o[v8 * 8 + 5] * inv);
-          u.w = pack_bf16x2(o[v8 * 8 + 6] * inv, o[v8 * 8 + 7] * inv);
-          dst[v8] = u;
-        }
-        if (wg == 0) p.lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
-      }
-      return true;
-    }
-    // ---- split chunk: store the partial record, then the last arriver merges
-    float* rec = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec) * kRecFloats;
-    float4* orow = reinterpret_cast<float4*>(rec + r * 64 + wg * 32);
-#pragma unroll
-    for (int v4 = 0; v4 < 8; ++v4)
-      orow[v4] = make_float4(o[v4 * 4 + 0], o[v4 * 4 + 1], o[v4 * 4 + 2], o[v4 * 4 + 3]);
-    if (wg == 0) {
-      rec[kTileRows * 64 + r] = l > 0.f ? m : -INFINITY;
-      rec[kTileRows * 64 + kTileRows + r] = l;
-    }
-    __threadfence();
-    if (!epi_sync()) return false;
-    int* ticket = p.tickets + static_cast<size_t>(tb) * p.n_split + tw.split;
-    if (warp == 0 && lane == 0) *last_flag = (atomicAdd(ticket, 1) == tw.nchunks - 1) ? 1u : 0u;
-    if (!epi_sync()) return false;
-    if (!*last_flag) return true;
-    __threadfence();
+    for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(raw[c >> 5][c & 31]);
+  }
+  ptx::tc_fence_before();
+  ptx::mbar_arrive(bar(kBarOFree));  // O may now be overwritten by the next tile
+  const float m = td.m, l = td.l;
+  const bool row_active = half == 0 || tqb >= 0;
+  const int qblk = half ? tqb : tqa;
+  const size_t row = static_cast<size_t>(tbh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
+  if (tw.split < 0) {
     if (row_active) {
-      const float* base = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec_base) * kRecFloats;
-      float ms = -INFINITY;
-      for (int c = 0; c < tw.nchunks; ++c)
-        ms = fmaxf(ms, __ldcg(base + static_cast<size_t>(c) * kRecFloats + kTileRows * 64 + r));
-      float acc[32];
-#pragma unroll
-      for (int x = 0; x < 32; ++x) acc[x] = 0.f;
-      float lsum = 0.f;
-      if (ms != -INFINITY) {
-        for (int c = 0; c < tw.nchunks; ++c) {
-          const float* rc = base + static_cast<size_t>(c) * kRecFloats;
-          const float mc = __ldcg(rc + kTileRows * 64 + r);
-          const float lc = __ldcg(rc + kTileRows * 64 + kTileRows + r);
-          if (mc == -INFINITY) continue;
-          const float f = ptx::ex2_approx(mc - ms);
-          lsum += lc * f;
-          const float4* oc = reinterpret_cast<const float4*>(rc + r * 64 + wg * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4) {
-            const float4 x = __ldcg(oc + v4);
-            acc[v4 * 4 + 0] += f * x.x;
-            acc[v4 * 4 + 1] += f * x.y;
-            acc[v4 * 4 + 2] += f * x.z;
-            acc[v4 * 4 + 3] += f * x.w;
-          }
-        }
-      }
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64 + wg * 32);
-#pragma unroll
-      for (int v8 = 0; v8 < 4; ++v8) {
-        uint4 u;
-        u.x = pack_bf16x2(acc[v8 * 8 + 0] * inv, acc[v8 * 8 + 1] * inv);
-        u.y = pack_bf16x2(acc[v8 * 8 + 2] * inv, acc[v8 * 8 + 3] * inv);
-        u.z = pack_bf16x2(acc[v8 * 8 + 4] * inv, acc[v8 * 8 + 5] * inv);
-        u.w = pack_bf16x2(acc[v8 * 8 + 6] * inv, acc[v8 * 8 + 7] * inv);
-        dst[v8] = u;
-      }
-      if (wg == 0) p.lse[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
+      store_row_bf16(p.out + row * 64, o, l > 0.f ? 1.f / l : 0.f);
+      p.lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
-    if (warp == 0 && lane == 0) *ticket = 0;  // leave the workspace clean for the next call
     return true;
   }
+  // ---- split chunk: store the partial record, then the last arriver merges
+  float* rec = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec) * kRecFloats;
+  float4* orow = reinterpret_cast<float4*>(rec + r * 64);
+#pragma unroll
+  for (int v4 = 0; v4 < 16; ++v4)
+    orow[v4] = make_float4(o[v4 * 4 + 0], o[v4 * 4 + 1], o[v4 * 4 + 2], o[v4 * 4 + 3]);
+  rec[kTileRows * 64 + r] = l > 0.f ? m : -INFINITY;
+  rec[kTileRows * 64 + kTileRows + r] = l;
+  __threadfence();
+  if (!epi_sync()) return false;
+  int* ticket = p.tickets + static_cast<size_t>(tb) * p.n_split + tw.split;
+  if (r == 0) *last_flag = (atomicAdd(ticket, 1) == tw.nchunks - 1) ? 1u : 0u;
+  if (!epi_sync()) return false;
+  if (!*last_flag) return true;
+  __threadfence();
+  if (row_active) merge_split_row(p, tw, tb, r, row);
+  if (r == 0) *ticket = 0;  // leave the workspace clean for the next call
+  return true;
 }
 
-
-__device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, uint32_t tmem,
-                                             int warp, int lane, volatile int* abort_flag,
-                                             volatile uint32_t* last_flag, float* xch) {
+__device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl, int warp, int lane,
+                                             volatile int* abort_flag) {
+  const uint32_t bars = sl.bars, tmem = sl.tmem;
+  volatile uint32_t* last_flag = sl.last_flag;
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  const int wg = warp >> 2;              // key block of each chunk handled here
-  const int r = (warp & 3) * 32 + lane;  // tile row == TMEM lane
-  const int half = r >> 6;
+  const int r = (warp & 3) * 32 + lane;  // tile row == TMEM lane (warp w reaches lanes 32 (w % 4)..)
+  const int half = r >> 6;               // warp-uniform: a warp's 32 rows lie in one half
   const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const uint32_t obase = tmem + lane_addr + kTmemO;
-  const int total = p.B * p.items_per_batch;
   const float sl2 = p.scale_log2;
   uint32_t g = 0;
   uint32_t n_epi = 0;  // uses of the epilogue barrier
-  uint32_t nt = 0;     // tiles started
   bool alive = true;
 
   TileDone pend{};
   bool have_pend = false;
-  for (int t = blockIdx.x; alive && t < total; t += gridDim.x, ++nt) {
-    const int b = t / p.items_per_batch;
-    const WorkItem w = p.items[t - b * p.items_per_batch];
-    // The tile's union entries (at most 64) and their key-padding bits, one or two
-    // per lane; each chunk picks its entry with a shuffle.
-    const uint32_t ent_lo = lane < w.count ? p.pair_ent[w.start + lane] : 0u;
-    const uint32_t ent_hi = lane + 32 < w.count ? p.pair_ent[w.start + 32 + lane] : 0u;
-    unsigned long long kb_lo = ~0ull, kb_hi = ~0ull;
-    if (p.keybits != nullptr) {
-      const size_t kb0 = static_cast<size_t>(b) * p.nb;
-      if (lane < w.count) kb_lo = p.keybits[kb0 + (ent_lo & kEntColMask)];
-      if (lane + 32 < w.count) kb_hi = p.keybits[kb0 + (ent_hi & kEntColMask)];
+  for (uint32_t k = 0; alive; ++k) {
+    const int t = take_item_warp(sl, k, abort_flag, p.timeout_ns);
+    if (t < 0) {
+      if (t == kItemAbort) alive = false;
+      break;
     }
+    // the tile's union entries and their key-padding bits, staged by the producer
+    const ItemStage& st = sl.items[k % kItemRing];
+    const int count = st.w.count;
     float m_run = -INFINITY, l_run = 0.f;
-    const int nch = (w.count + 1) >> 1;
-    for (int n = 0; n < nch; ++n, ++g) {
-      const int idx = 2 * n + wg;  // warp-uniform
-      const bool has = idx < w.count;
-      const uint32_t e = __shfl_sync(0xffffffffu, idx < 32 ? ent_lo : ent_hi, idx & 31);
-      const unsigned long long kb = __shfl_sync(0xffffffffu, idx < 32 ? kb_lo : kb_hi, idx & 31);
-      // warp-uniform: a warp's 32 rows lie in one half of the tile
-      const unsigned long long mk = (has && ((e >> (kEntBitsShift + half)) & 1u)) ? kb : 0ull;
+    for (int n = 0; n < count; ++n, ++g) {
+      const uint32_t e = st.ent[n];
+      const unsigned long long kb = st.kb[n];
+      const unsigned long long mk = ((e >> (kEntBitsShift + half)) & 1u) ? kb : 0ull;
       const uint32_t sb = g % kSBufs;
       if (!wait_warp(bar(kBarSFull + static_cast<int>(sb)), (g / kSBufs) & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
       ptx::tc_fence_after();
-      const uint32_t sbase = tmem + lane_addr + kTmemS + sb * 128u + static_cast<uint32_t>(wg) * 64u;
-      // Pass 1: the row maximum of this warpgroup's 64 scores.
-      float mxs = -INFINITY;
-      if (mk != 0ull) {
-        uint32_t raw[2][32];
-        ptx::tmem_ld32(sbase + 0, raw[0]);
-        ptx::tmem_ld32(sbase + 32, raw[1]);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence(raw[0]);
-        ptx::reg_fence(raw[1]);
-        float s[64];
-#pragma unroll
-        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
-        mask_cols(s, mk);
-        float mx4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-        for (int c = 4; c < 64; c += 2) mx4[(c >> 1) & 3] = ptx::fmax3(mx4[(c >> 1) & 3], s[c], s[c + 1]);
-        const float mx = fmaxf(ptx::fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
-        mxs = mx * sl2;  // scale > 0: -inf stays -inf
-      }
-      float m_new = m_run;
-      bool rescale = false;
-      if (n == 0) {
-        m_new = mxs;
-      } else if (__any_sync(0xffffffffu, mxs > m_run + kRescaleLog2)) {
-        rescale = true;
-        m_new = fmaxf(m_run, mxs);
-      }
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      // Pass 2: p = 2^(s * scale * log2 e - m) 32 columns at a time, reloaded from TMEM
-      // to keep few registers live; P_x (bf16, two keys per column) goes over S
-      // columns already read.  The buffer's previous reader, PV of chunk g - 3,
-      // completed before S(g) was issued.
+      const uint32_t sbase = tmem + lane_addr + kTmemS + sb * 64u;
+      // p = 2^(s * scale * log2 e - m) with the row's running max m as it stands (a
+      // lazy max): m is raised only on the row's first attended chunk, or when the
+      // chunk's sum of p would exceed 2^kLazyLog2 -- then the chunk is redone with
+      // its own max folded into m, and l and O are rescaled.  So every p stays below
+      // 2^kLazyLog2, which bf16 P and fp32 O and l hold without loss of relative
+      // precision, and the common chunk reads S once and takes no max.
       float psum = 0.f;
+      float m_new = m_run;
+      uint32_t pk[32];
       if (mk != 0ull) {
-        const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_use, -m_use);
-        uint64_t acc0 = 0ull, acc1 = 0ull;  // packed partial row sums
-#pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          uint32_t raw[32];
-          ptx::tmem_ld32(sbase + 32u * hb, raw);
+        bool need_max = __any_sync(0xffffffffu, m_run == -INFINITY);
+        const uint64_t sc2 = ptx::pack2(sl2, sl2);
+        for (;;) {
+          uint32_t raw[2][32];
+          ptx::tmem_ld32(sbase + 0, raw[0]);
+          ptx::tmem_ld32(sbase + 32, raw[1]);
           ptx::tmem_wait_ld();
-          ptx::reg_fence(raw);
-          float s[32];
+          ptx::reg_fence(raw[0]);
+          ptx::reg_fence(raw[1]);
+          float s[64];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) s[c] = __uint_as_float(raw[c]);
-          const uint32_t mh = static_cast<uint32_t>(mk >> (32 * hb));
-          if (mh != 0xffffffffu) {
+          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
+          mask_cols(s, mk);
+          if (need_max) {  // warp-uniform
+            float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (!((mh >> c) & 1u)) s[c] = -INFINITY;
+            for (int c = 4; c < 64; c += 2) mx4[(c >> 1) & 3] = ptx::fmax3(mx4[(c >> 1) & 3], s[c], s[c + 1]);
+            const float mx = fmaxf(ptx::fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
+            // mk != 0 keeps at least one key, so mx is finite (scale > 0)
+            m_new = fmaxf(m_run, mx * sl2);
           }
-          uint32_t pk[16];
+          const uint64_t nm2 = ptx::pack2(-m_new, -m_new);
+          uint64_t acc0 = 0ull, acc1 = 0ull;  // packed partial row sums
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < 32; ++c) {
             float x0, x1;
             ptx::unpack2(ptx::ffma2(ptx::pack2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
             const float p0 = ptx::ex2_approx(x0), p1 = ptx::ex2_approx(x1);
@@ -597,45 +666,47 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
               acc0 = ptx::fadd2(acc0, ptx::pack2(p0, p1));
             pk[c] = pack_bf16x2(p0, p1);
           }
-          ptx::tmem_st16(sbase + 16u * hb, pk);
+          float a0, a1;
+          ptx::unpack2(ptx::fadd2(acc0, acc1), a0, a1);
+          psum = a0 + a1;
+          // !(<=) also catches an infinite or NaN sum
+          if (need_max || !__any_sync(0xffffffffu, !(psum <= kLazyBound))) break;
+          need_max = true;
         }
-        float a0, a1;
-        ptx::unpack2(ptx::fadd2(acc0, acc1), a0, a1);
-        psum = a0 + a1;
-      } else if (has) {
-        // this half of the tile does not attend the block: its P rows are zero
-        uint32_t zero[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) zero[c] = 0u;
-        ptx::tmem_st32(sbase, zero);
-      }
-      if (n == 0) {
-        l_run = psum;
+        // P (bf16, two keys per column) over S columns already read.  The buffer's
+        // previous reader, PV of chunk g - 3, completed before S(g) was issued.
+        ptx::tmem_st32(sbase, pk);
       } else {
-        const float alpha = (m_new == m_run) ? 1.f : ptx::ex2_approx(m_run - m_new);
-        l_run = l_run * alpha + psum;
-        if (rescale) {  // warp-uniform
-          // O_x must hold PV of chunk g - 1 before it is rescaled: wait for its
-          // V-free phase.  Unambiguous: S(g) was issued after PV(g - 3) was done, and
-          // PV(g - 1 + kVStages) needs this warpgroup's P first.
-          const uint32_t gp = g - 1u;
-          if (!wait_warp(bar(kBarVFree + static_cast<int>(gp % kVStages)), (gp / kVStages) & 1u,
-                         abort_flag, p.timeout_ns)) {
-            alive = false;
-            break;
-          }
-          ptx::tc_fence_after();
-          const uint32_t ox = obase + static_cast<uint32_t>(wg) * 64u;
+        // this half of the tile does not attend the block (or all of its keys are
+        // padding): its P rows are zero
 #pragma unroll
-          for (int hlf = 0; hlf < 2; ++hlf) {
-            uint32_t o[32];
-            ptx::tmem_ld32(ox + 32u * hlf, o);
-            ptx::tmem_wait_ld();
-            ptx::reg_fence(o);
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        ptx::tmem_st32(sbase, pk);
+      }
+      const bool grew = m_new != m_run;
+      const float alpha = grew ? ptx::ex2_approx(m_run - m_new) : 1.f;  // 2^-inf = 0
+      const bool had_mass = l_run > 0.f;
+      l_run = l_run * alpha + psum;
+      if (n > 0 && __any_sync(0xffffffffu, grew && had_mass)) {
+        // O must hold PV of chunk g - 1 before it is rescaled: wait for its V-free
+        // phase.  Unambiguous: S(g) was issued after PV(g - 3) was done, and
+        // PV(g - 1 + kVStages) needs this warp's P first.
+        const uint32_t gp = g - 1u;
+        if (!wait_warp(bar(kBarVFree + static_cast<int>(gp % kVStages)), (gp / kVStages) & 1u, abort_flag,
+                       p.timeout_ns)) {
+          alive = false;
+          break;
+        }
+        ptx::tc_fence_after();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            ptx::tmem_st32(ox + 32u * hlf, o);
-          }
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          uint32_t o[32];
+          ptx::tmem_ld32(obase + 32u * hlf, o);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(o);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          ptx::tmem_st32(obase + 32u * hlf, o);
         }
       }
       m_run = m_new;
@@ -644,17 +715,21 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, uint32_t bars, 
       ptx::mbar_arrive(bar(kBarPFull + static_cast<int>(sb)));
       if (n == 0 && have_pend) {  // the previous tile's epilogue, one chunk late
         have_pend = false;
-        if (!tile_epilogue(p, pend, bars, obase, warp, lane, abort_flag, last_flag, xch, &n_epi)) {
+        if (!tile_epilogue(p, pend, sl.items[pend.k % kItemRing], bars, obase, warp, lane, abort_flag,
+                           last_flag, &n_epi)) {
           alive = false;
           break;
         }
+        release_item_warp(sl, pend.k, lane);
       }
     }
     if (!alive) break;
-    pend = TileDone{t, g - 1u, nt, m_run, l_run};
+    pend = TileDone{k, g - 1u, m_run, l_run};
     have_pend = true;
   }
-  if (alive && have_pend) tile_epilogue(p, pend, bars, obase, warp, lane, abort_flag, last_flag, xch, &n_epi);
+  if (alive && have_pend &&
+      tile_epilogue(p, pend, sl.items[pend.k % kItemRing], bars, obase, warp, lane, abort_flag, last_flag, &n_epi))
+    release_item_warp(sl, pend.k, lane);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -662,20 +737,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  const uint32_t sQ = base + kSmemQ, sK = base + kSmemK, sV = base + kSmemV, bars = base + kSmemBar;
   volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kSmemMisc);
-  float* xch = reinterpret_cast<float*>(smem + kSmemXch);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i) {
-      uint32_t count = 1;
-      if ((i >= kBarPFull && i < kBarPFull + static_cast<int>(kSBufs)) || i == kBarOFree || i == kBarEpi)
-        count = 256;
-      ptx::mbar_init(bars + 8u * i, count);
+    for (int s = 0; s < kSlots; ++s) {
+      const uint32_t bars = base + s * kSlotBytes + kSmemBar;
+      for (int i = 0; i < kNumBars; ++i) {
+        uint32_t count = 1;
+        if ((i >= kBarPFull && i < kBarPFull + static_cast<int>(kSBufs)) || i == kBarOFree || i == kBarEpi)
+          count = kSoftmaxThreads;
+        if (i >= kBarItemEmpty && i < kBarItemEmpty + kItemRing) count = kItemReaders;
+        ptx::mbar_init(bars + 8u * i, count);
+      }
+      *reinterpret_cast<volatile uint32_t*>(smem + s * kSlotBytes + kSmemLast) = 0;
     }
     misc[1] = 0;
-    misc[2] = 0;
     ptx::fence_barrier_init();
   }
   if (warp == kProducerWarp && lane == 0) {
@@ -690,26 +767,35 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  const uint32_t tmem = misc[0];
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
-  if (warp == kProducerWarp) {
-    if (lane == 0) producer_role(p, sQ, sK, sV, bars, abort_flag);
+  const int slot = warp < 8 ? (warp >> 2) : warp < kMmaWarp ? warp - kProducerWarp : (warp - kMmaWarp) >> 1;
+  Slot sl;
+  sl.sQ = base + slot * kSlotBytes + kSmemQ;
+  sl.sK = base + slot * kSlotBytes + kSmemK;
+  sl.sV = base + slot * kSlotBytes + kSmemV;
+  sl.bars = base + slot * kSlotBytes + kSmemBar;
+  sl.items = reinterpret_cast<ItemStage*>(smem + slot * kSlotBytes + kSmemItems);
+  sl.last_flag = reinterpret_cast<volatile uint32_t*>(smem + slot * kSlotBytes + kSmemLast);
+  sl.tmem = misc[0] + static_cast<uint32_t>(slot) * kSlotCols;
+
+  if (warp < 8) {
+    softmax_role(p, sl, warp, lane, abort_flag);
+  } else if (warp < kMmaWarp) {
+    producer_role(p, sl, lane, abort_flag);
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) s_issuer(p, sQ, sK, bars, tmem, abort_flag);
+  } else if (warp == kMmaWarp + 2 * slot) {
+    if (lane == 0) s_issuer(p, sl, abort_flag);
     __syncwarp();
-  } else if (warp == kPvWarp) {
-    if (lane == 0) pv_issuer(p, sV, bars, tmem, abort_flag);
+  } else if (warp == kPvWarp + 2 * slot) {
+    if (lane == 0) pv_issuer(p, sl, abort_flag);
     __syncwarp();
-  } else {
-    softmax_role(p, bars, tmem, warp, lane, abort_flag, &misc[2], xch);
   }
 
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == kMmaWarp) ptx::tmem_dealloc(tmem, kTmemCols);
+  if (warp == kMmaWarp) ptx::tmem_dealloc(misc[0], kTmemCols);
 }
 
 // Per (b, key block): bit c set when key 64*j + c is kept by the padding mask.
@@ -887,7 +973,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
   prm.pair_ent = lay->d_pair_ent;
   prm.keybits = key_mask ? reinterpret_cast<const unsigned long long*>(ws + plan.keybits_off) : nullptr;
   prm.partials = reinterpret_cast<float*>(ws + plan.partials_off);
-  prm.tickets = reinterpret_cast<int*>(ws + plan.tickets_off);
+  prm.sched = reinterpret_cast<int*>(ws + plan.tickets_off);
+  prm.tickets = reinterpret_cast<int*>(ws + plan.tickets_off + kSchedBytes);
   prm.B = B;
   prm.H = H;
   prm.L = L;
@@ -907,7 +994,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   const int64_t total = static_cast<int64_t>(B) * prm.items_per_batch;
-  const int grid = static_cast<int>(std::min<int64_t>(total, info.sms));
+  // two slots per CTA; items are drawn dynamically
+  const int grid = static_cast<int>(std::min<int64_t>((total + kSlots - 1) / kSlots, info.sms));
   if (grid < 1) return BSA_OK;
   bsa_fwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;

@@ -155,7 +155,7 @@ WorkspacePlan plan_workspace(const bsa_layout& lay, int B) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   WorkspacePlan p{};
   p.tickets_off = 0;
-  p.tickets_bytes = up(std::max<size_t>(4, sizeof(int32_t) * static_cast<size_t>(B) * lay.n_split));
+  p.tickets_bytes = up(kSchedBytes + sizeof(int32_t) * static_cast<size_t>(B) * lay.n_split);
   p.keybits_off = p.tickets_off + p.tickets_bytes;
   p.keybits_bytes = up(sizeof(uint64_t) * static_cast<size_t>(B) * lay.nb);
   p.partials_off = p.keybits_off + p.keybits_bytes;
@@ -188,6 +188,7 @@ void build_tiles(bsa_layout* lay) {
   const int P = lay->n_pairs;
   lay->pair_ptr.assign(1, 0);
   lay->pair_ent.clear();
+  std::vector<uint32_t> both, only_a, only_b;
   for (int h = 0; h < H; ++h) {
     for (int p = 0; p < P; ++p) {
       const int qa = lay->pair_q[2 * p], qb = lay->pair_q[2 * p + 1];
@@ -199,45 +200,60 @@ void build_tiles(bsa_layout* lay) {
         rb = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qb];
         rb_end = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qb + 1];
       }
+      // Union entries: the blocks both query blocks attend, then the blocks only one
+      // of them attends, alternating first/second; each group ascending.  The order
+      // is free (one softmax over the union), and this one keeps the two halves of
+      // the tile -- whose warps skip the exponentials of a block their half does not
+      // attend -- doing equal work chunk by chunk.
+      both.clear();
+      only_a.clear();
+      only_b.clear();
       while (ra != ra_end || rb != rb_end) {
-        uint32_t col, bits;
         if (rb == rb_end || (ra != ra_end && *ra < *rb)) {
-          col = static_cast<uint32_t>(*ra++);
-          bits = 1;
+          only_a.push_back(static_cast<uint32_t>(*ra++) | (1u << bsa::kEntBitsShift));
         } else if (ra == ra_end || *rb < *ra) {
-          col = static_cast<uint32_t>(*rb++);
-          bits = 2;
+          only_b.push_back(static_cast<uint32_t>(*rb++) | (2u << bsa::kEntBitsShift));
         } else {
-          col = static_cast<uint32_t>(*ra++);
+          both.push_back(static_cast<uint32_t>(*ra++) | (3u << bsa::kEntBitsShift));
           ++rb;
-          bits = 3;
         }
-        lay->pair_ent.push_back(col | (bits << bsa::kEntBitsShift));
+      }
+      lay->pair_ent.insert(lay->pair_ent.end(), both.begin(), both.end());
+      for (size_t x = 0; x < std::max(only_a.size(), only_b.size()); ++x) {
+        if (x < only_a.size()) lay->pair_ent.push_back(only_a[x]);
+        if (x < only_b.size()) lay->pair_ent.push_back(only_b[x]);
       }
       lay->pair_ptr.push_back(static_cast<int32_t>(lay->pair_ent.size()));
     }
   }
-  // Static schedule for one batch element, head-major so that consecutive
-  // items (run concurrently by consecutive CTAs) share the head's K/V in L2.
+  // Work items of one batch element, in the order they are handed out (the
+  // forward draws item i for every batch element before item i + 1): first the
+  // chunks of split tiles -- the longest items, and the ones whose last chunk
+  // merges the others -- then the other tiles, head-major so that items running
+  // at the same time share the head's K/V in L2.
   lay->items.clear();
   lay->n_split = 0;
   lay->n_records = 0;
-  for (int h = 0; h < H; ++h) {
-    for (int p = 0; p < P; ++p) {
-      const int32_t s = lay->pair_ptr[static_cast<size_t>(h) * P + p];
-      const int32_t U = lay->pair_ptr[static_cast<size_t>(h) * P + p + 1] - s;
-      if (U <= bsa::kSplitThreshold) {
-        lay->items.push_back(bsa::WorkItem{h, p, s, U, -1, 0, 1, 0});
-        continue;
-      }
-      const int nch = (U + bsa::kSplitChunk - 1) / bsa::kSplitChunk;
-      const int slot = lay->n_split++;
-      const int base = lay->n_records;
-      lay->n_records += nch;
-      for (int c = 0; c < nch; ++c) {
-        const int cs = c * bsa::kSplitChunk;
-        lay->items.push_back(bsa::WorkItem{h, p, s + cs, std::min(bsa::kSplitChunk, U - cs),
-                                           slot, base + c, nch, base});
+  for (const bool split_pass : {true, false}) {
+    for (int h = 0; h < H; ++h) {
+      for (int p = 0; p < P; ++p) {
+        const int32_t s = lay->pair_ptr[static_cast<size_t>(h) * P + p];
+        const int32_t U = lay->pair_ptr[static_cast<size_t>(h) * P + p + 1] - s;
+        const bool split = U > bsa::kSplitThreshold;
+        if (split != split_pass) continue;
+        if (!split) {
+          lay->items.push_back(bsa::WorkItem{h, p, s, U, -1, 0, 1, 0});
+          continue;
+        }
+        const int nch = (U + bsa::kSplitChunk - 1) / bsa::kSplitChunk;
+        const int slot = lay->n_split++;
+        const int base = lay->n_records;
+        lay->n_records += nch;
+        for (int c = 0; c < nch; ++c) {
+          const int cs = c * bsa::kSplitChunk;
+          lay->items.push_back(bsa::WorkItem{h, p, s + cs, std::min(bsa::kSplitChunk, U - cs),
+                                             slot, base + c, nch, base});
+        }
       }
     }
   }

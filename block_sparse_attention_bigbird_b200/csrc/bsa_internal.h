@@ -69,11 +69,15 @@ struct bsa_layout {
 namespace bsa {
 // Workspace carve-up for batch size B (all offsets 256-byte aligned).
 struct WorkspacePlan {
+  // [tickets_off, +tickets_bytes): the area that must be zero before a call and is
+  // zero again after one: the work-item counter and finished-slot counter of the
+  // dynamic schedule (kSchedBytes), then one arrival ticket per split tile.
   size_t tickets_off, tickets_bytes;
   size_t keybits_off, keybits_bytes;
   size_t partials_off, partials_bytes;
   size_t total;
 };
+constexpr size_t kSchedBytes = 16;
 WorkspacePlan plan_workspace(const bsa_layout& lay, int B);
 void free_device(bsa_layout* lay);
 }  // namespace bsa

@@ -108,7 +108,9 @@ int bsa_layout_globals(const bsa_layout* layout, const int32_t** globals, int* n
  *             tile holds a single block.  Global blocks pair with global blocks.
  *   pair_ptr: H*n_pairs+1 int32 offsets into pair_ent, head-major.
  *   pair_ent: key block | (membership << 24): bit 0 = in the first block's row,
- *             bit 1 = in the second's.
+ *             bit 1 = in the second's.  Per tile: the blocks in both rows, then
+ *             the blocks in one row only, alternating first/second; each group
+ *             ascending.
  * Any output may be NULL.
  */
 int bsa_layout_tiles(const bsa_layout* layout, const int32_t** pair_q, int* n_pairs,

@@ -60,6 +60,12 @@ def test_tile_decomposition():
                 bits = ent >> 24
                 ra = set(OL.row(ref, h, a).tolist())
                 rb = set(OL.row(ref, h, b).tolist()) if b >= 0 else set()
-                assert list(cols) == sorted(ra | rb)
+                assert sorted(cols) == sorted(ra | rb) and len(set(cols)) == len(cols)
                 for c, bt in zip(cols, bits):
                     assert bool(bt & 1) == (c in ra) and bool(bt & 2) == (c in rb)
+                # order: blocks of both rows, then one-row blocks alternating a/b
+                both = sorted(ra & rb)
+                oa, ob = sorted(ra - rb), sorted(rb - ra)
+                alt = [x for i in range(max(len(oa), len(ob)))
+                       for x in (oa[i:i + 1] + ob[i:i + 1])]
+                assert list(cols) == both + alt
