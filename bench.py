@@ -84,6 +84,13 @@ def _dead_from(w):
     return (w.L - w.key_pad_tail + 63) // 64
 
 
+def _has_split_rows(lay) -> bool:
+    """Whether bsa_forward launches its split-row merge for this layout."""
+    from block_sparse_attention_bigbird_b200 import bsa
+    _, pair_ptr, _ = bsa.bsa_layout_tiles(lay)
+    return bool(np.any(np.diff(pair_ptr) > bsa.SPLIT_THRESHOLD))
+
+
 def _nnz_eff(w, row_ptr, col_idx) -> int:
     """Blocks over all (b, h, i, j), minus those whose 64 keys are all padded."""
     per_batch = int(len(col_idx))
@@ -284,7 +291,8 @@ def run_ours(args, w, world, rank, local):
     out = torch.empty_like(qd)
     lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
     ws = torch.zeros(bsa.bsa_workspace_bytes(lay, w.B), dtype=torch.uint8, device=dev)
-    launches_per_step = 1 + (1 if km is not None else 0)
+    # forward, plus the key-bit kernel with a key mask and the merge with split rows
+    launches_per_step = 1 + (1 if km is not None else 0) + (1 if _has_split_rows(lay) else 0)
 
     def step():
         bsa.bsa_forward(qd, kd, vd, lay, key_mask=kmd, out=out, lse=lse, workspace=ws, stream=stream)

@@ -25,6 +25,7 @@ BSA_ERR_OOM = -6
 BSA_ERR_WORKSPACE = -7
 BSA_ERR_STATIC_WORKSPACE = -8
 STATIC_WORKSPACE_BYTES = 32 * 1024 * 1024  # BSA_STATIC_WORKSPACE_BYTES in include/bsa.h
+SPLIT_THRESHOLD = 48  # BSA_SPLIT_THRESHOLD in include/bsa.h: longer tile unions are split
 
 # name -> (restype, argtypes); mirrors include/bsa.h
 _SIGNATURES = {

@@ -30,8 +30,9 @@
 // A tile is two query blocks of the same (b, h) over the sorted union of their rows;
 // entries carry per-block membership bits so each half of the tile sees exactly its
 // own row, and a warp whose half does not attend a block skips its exponentials.
-// Long unions (global rows) are cut into chunks processed by different CTAs; each
-// chunk stores a partial (O, m, l) and the last one to arrive merges them.
+// Long unions (global rows) are cut into chunks run as separate work items; each
+// stores a partial (O, m, l) record, and bsa_merge_kernel, launched after the
+// forward, merges a split tile's records into its output rows.
 // Every wait is bounded (globaltimer); on expiry the CTA records
 // BSA_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -56,7 +57,7 @@ constexpr int kThreads = 448;
 constexpr int kSoftmaxThreads = 128;  // per slot
 constexpr int kItemRing = 4;  // work-item indices a slot's producer may publish ahead
 constexpr int kKStages = 3;  // == kSBufs: K stage g % 3 is free once S(g) is done
-constexpr int kVStages = 5;  // V stage g % 5 is free once PV(g) is done
+constexpr int kVStages = 4;  // V stage g % 4 is free once PV(g) is done
 constexpr uint32_t kBlkBytes = 64 * 128;     // one 64 x 64 bf16 block
 constexpr uint32_t kQBytes = 2 * kBlkBytes;  // 128-row Q tile
 constexpr uint32_t kTmemCols = 512;
@@ -75,7 +76,9 @@ constexpr uint32_t kWaitSleepNs = 20000;  // upper bound on one sleep inside a b
 constexpr uint32_t kSmemQ = 0;
 constexpr uint32_t kSmemK = kSmemQ + 2 * kQBytes;
 constexpr uint32_t kSmemV = kSmemK + kKStages * kBlkBytes;
-constexpr uint32_t kSmemBar = kSmemV + kVStages * kBlkBytes;
+constexpr uint32_t kSmemOStage = kSmemV + kVStages * kBlkBytes;  // 4 x (32 rows x 128 B) O staging
+constexpr uint32_t kOStageBytes = 32 * 128;
+constexpr uint32_t kSmemBar = kSmemOStage + 4 * kOStageBytes;
 enum : int {
   kBarQFull = 0,
   kBarQEmpty = 2,
@@ -88,8 +91,7 @@ enum : int {
   kBarPFull = kBarSFull + kSBufs,         // [S buffer] P written, 128 arrivals
   kBarOFree = kBarPFull + kSBufs,         // 128 arrivals once the epilogue has read O
   kBarMmaFinal = kBarOFree + 1,           // [2 issuers]
-  kBarEpi = kBarMmaFinal + 2,             // 128 softmax threads, split-record rendezvous
-  kBarItemFull = kBarEpi + 1,             // [item ring] the producer published a work item
+  kBarItemFull = kBarMmaFinal + 2,             // [item ring] the producer published a work item
   kBarItemEmpty = kBarItemFull + kItemRing,  // [item ring] 6 arrivals: both issuers and the
                                              // four softmax warps have read it
   kNumBars = kBarItemEmpty + kItemRing
@@ -112,8 +114,7 @@ struct ItemStage {
 };
 static_assert(sizeof(ItemStage) % 16 == 0, "stage alignment");
 constexpr uint32_t kSmemItems = (kSmemBar + 8 * kNumBars + 15) & ~15u;  // ItemStage[kItemRing]
-constexpr uint32_t kSmemLast = kSmemItems + sizeof(ItemStage) * kItemRing;  // u32: last arriver flag
-constexpr uint32_t kSlotBytes = (kSmemLast + 4 + 1023) & ~1023u;
+constexpr uint32_t kSlotBytes = (kSmemItems + sizeof(ItemStage) * kItemRing + 1023) & ~1023u;
 constexpr uint32_t kSmemMisc = kSlots * kSlotBytes;          // u32 TMEM base, int abort flag
 constexpr uint32_t kSmemUsed = kSmemMisc + 16;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // slack for 1024-byte alignment
@@ -124,13 +125,15 @@ static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 // publishes it to the slot's other roles through a small ring in shared memory.
 struct Slot {
   uint32_t sQ, sK, sV, bars;
+  uint8_t* ostage;   // O staging of softmax warp w at ostage + (w % 4) * kOStageBytes
+  uint32_t sO;       // its shared-memory address
   ItemStage* items;  // the item ring
-  volatile uint32_t* last_flag;
   uint32_t tmem;  // TMEM address of the slot's column 0
 };
 
 struct FwdParams {
   CUtensorMap tm_q, tm_k, tm_v;
+  CUtensorMap tm_o;  // O as [B*H*L, 64] bf16, 32-row boxes (epilogue stores)
   __nv_bfloat16* out;
   float* lse;
   const WorkItem* items;
@@ -139,8 +142,8 @@ struct FwdParams {
   const unsigned long long* keybits;  // [B, nb] or null
   float* partials;
   int* sched;    // [0] next work item, [1] slots finished; zero between calls
-  int* tickets;
   int B, H, L, nb, items_per_batch, n_split, n_records;
+  int split_items;  // the first split_items items of a batch element are split-tile chunks
   float scale_log2;
   unsigned long long timeout_ns;
 };
@@ -256,9 +259,19 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const Slot& sl
     // stage the item for the slot's other roles
     ItemStage& st = sl.items[ii];
     if (t >= 0) {
-      // t enumerates (item, batch element) item-major: the items' order holds for
-      // the whole batch
-      const int i = t / p.B, b = t - i * p.B;
+      // t enumerates (batch element, item): first the split-tile chunks of every
+      // batch element (the longest items, kept away from the end of the run), then
+      // the other tiles batch element by batch element (its K/V stay in L2)
+      const int ns = p.split_items;
+      int b, i;
+      if (t < p.B * ns) {
+        i = t / p.B;
+        b = t - i * p.B;
+      } else {
+        const int nn = p.items_per_batch - ns, u = t - p.B * ns;
+        b = u / nn;
+        i = ns + (u - b * nn);
+      }
       const WorkItem w = p.items[i];
       for (int e = lane; e < w.count; e += 32) {
         const uint32_t en = p.pair_ent[w.start + e];
@@ -446,90 +459,15 @@ struct TileDone {
   float m, l;       // the row's running max (log2 units) and sum
 };
 
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst_row, const float* o, float inv) {
-  uint4* dst = reinterpret_cast<uint4*>(dst_row);
-#pragma unroll
-  for (int v8 = 0; v8 < 8; ++v8) {
-    uint4 u;
-    u.x = pack_bf16x2(o[v8 * 8 + 0] * inv, o[v8 * 8 + 1] * inv);
-    u.y = pack_bf16x2(o[v8 * 8 + 2] * inv, o[v8 * 8 + 3] * inv);
-    u.z = pack_bf16x2(o[v8 * 8 + 4] * inv, o[v8 * 8 + 5] * inv);
-    u.w = pack_bf16x2(o[v8 * 8 + 6] * inv, o[v8 * 8 + 7] * inv);
-    dst[v8] = u;
-  }
-}
-
-// The last-arriving chunk of a split tile merges the tile's partial records into
-// row `row` of O and lse.  Out of line: it runs once per split tile.
-__device__ __noinline__ void merge_split_row(const FwdParams& p, const WorkItem& tw, int tb, int r, size_t row) {
-  // The max over the records, then the sums of l and O with record c weighted by
-  // 2^(m_c - max); a record whose row attended nothing has m = -inf, O = 0 and
-  // weight 0.  The record loop is unrolled so that loads of several records are
-  // in flight together.
-  const float* base = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec_base) * kRecFloats;
-  const int nc = tw.nchunks;
-  constexpr int kM = kTileRows * 64, kL = kTileRows * 64 + kTileRows;
-  float ms = -INFINITY;
-#pragma unroll 8
-  for (int c = 0; c < nc; ++c) ms = fmaxf(ms, __ldcg(base + static_cast<size_t>(c) * kRecFloats + kM + r));
-  float lsum = 0.f;
-#pragma unroll 8
-  for (int c = 0; c < nc; ++c) {
-    const float* rc = base + static_cast<size_t>(c) * kRecFloats;
-    const float mc = __ldcg(rc + kM + r);
-    lsum += mc == -INFINITY ? 0.f : __ldcg(rc + kL + r) * ptx::ex2_approx(mc - ms);
-  }
-  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-#pragma unroll 1
-  for (int hh = 0; hh < 2; ++hh) {  // output columns [32 hh, 32 hh + 32)
-    float acc[32];
-#pragma unroll
-    for (int x = 0; x < 32; ++x) acc[x] = 0.f;
-#pragma unroll 2
-    for (int c = 0; c < nc; ++c) {
-      const float* rc = base + static_cast<size_t>(c) * kRecFloats;
-      float4 x[8];
-#pragma unroll
-      for (int v = 0; v < 8; ++v) x[v] = __ldcg(reinterpret_cast<const float4*>(rc + r * 64 + 32 * hh) + v);
-      const float mc = __ldcg(rc + kM + r);
-      const float f = mc == -INFINITY ? 0.f : ptx::ex2_approx(mc - ms);
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        acc[4 * v + 0] += f * x[v].x;
-        acc[4 * v + 1] += f * x[v].y;
-        acc[4 * v + 2] += f * x[v].z;
-        acc[4 * v + 3] += f * x[v].w;
-      }
-    }
-    uint4* dst = reinterpret_cast<uint4*>(p.out + row * 64 + 32 * hh);
-#pragma unroll
-    for (int v8 = 0; v8 < 4; ++v8) {
-      uint4 u;
-      u.x = pack_bf16x2(acc[v8 * 8 + 0] * inv, acc[v8 * 8 + 1] * inv);
-      u.y = pack_bf16x2(acc[v8 * 8 + 2] * inv, acc[v8 * 8 + 3] * inv);
-      u.z = pack_bf16x2(acc[v8 * 8 + 4] * inv, acc[v8 * 8 + 5] * inv);
-      u.w = pack_bf16x2(acc[v8 * 8 + 6] * inv, acc[v8 * 8 + 7] * inv);
-      dst[v8] = u;
-    }
-  }
-  p.lse[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
-}
-
-// Epilogue of a finished tile: normalise O and store it with lse (or the split
-// chunk's partial record, merging when last).  Kept out of line: it runs once per
-// tile and would otherwise crowd the chunk loop's registers.
-__device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& td, const ItemStage& st, uint32_t bars,
-                                           uint32_t obase, int warp, int lane, volatile int* abort_flag,
-                                           volatile uint32_t* last_flag, uint32_t* n_epi) {
+// Epilogue of a finished tile: normalise O and store it with lse (or, for a chunk
+// of a split tile, its partial record).  Kept out of line: it runs once per tile
+// and would otherwise crowd the chunk loop's registers.
+__device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& td, const ItemStage& st,
+                                           const Slot& sl, uint32_t bars,
+                                           uint32_t obase, int warp, int lane, volatile int* abort_flag) {
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   const int r = (warp & 3) * 32 + lane;
   const int half = r >> 6;
-  auto epi_sync = [&]() -> bool {
-    ptx::mbar_arrive(bar(kBarEpi));
-    const bool ok = wait_warp(bar(kBarEpi), *n_epi & 1u, abort_flag, p.timeout_ns);
-    ++*n_epi;
-    return ok;
-  };
   const int tb = st.b;
   const WorkItem& tw = st.w;
   const int tqa = st.qa, tqb = st.qb;
@@ -559,13 +497,35 @@ __device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& t
   const int qblk = half ? tqb : tqa;
   const size_t row = static_cast<size_t>(tbh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
   if (tw.split < 0) {
-    if (row_active) {
-      store_row_bf16(p.out + row * 64, o, l > 0.f ? 1.f / l : 0.f);
+    if (row_active) {  // warp-uniform: a warp's 32 rows lie in one half
+      // O rows through this warp's staging buffer (128-byte swizzle: 16-byte
+      // chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)), then one TMA store of
+      // the warp's 32 x 64 tile.
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      uint8_t* stg = sl.ostage + (warp & 3) * kOStageBytes;
+      if (lane == 0) ptx::bulk_wait_read_all();  // the previous tile's store has read it
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        uint4 u;
+        u.x = pack_bf16x2(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
+        u.y = pack_bf16x2(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
+        u.z = pack_bf16x2(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
+        u.w = pack_bf16x2(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+        *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) = u;
+      }
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::tma_store_2d(&p.tm_o, sl.sO + (warp & 3) * kOStageBytes, 0,
+                          static_cast<int>(row - static_cast<size_t>(r & 31)));
+        ptx::bulk_commit_group();
+      }
       p.lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
     return true;
   }
-  // ---- split chunk: store the partial record, then the last arriver merges
+  // ---- split chunk: its partial record (unnormalised O, m, l)
   float* rec = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec) * kRecFloats;
   float4* orow = reinterpret_cast<float4*>(rec + r * 64);
 #pragma unroll
@@ -573,22 +533,12 @@ __device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& t
     orow[v4] = make_float4(o[v4 * 4 + 0], o[v4 * 4 + 1], o[v4 * 4 + 2], o[v4 * 4 + 3]);
   rec[kTileRows * 64 + r] = l > 0.f ? m : -INFINITY;
   rec[kTileRows * 64 + kTileRows + r] = l;
-  __threadfence();
-  if (!epi_sync()) return false;
-  int* ticket = p.tickets + static_cast<size_t>(tb) * p.n_split + tw.split;
-  if (r == 0) *last_flag = (atomicAdd(ticket, 1) == tw.nchunks - 1) ? 1u : 0u;
-  if (!epi_sync()) return false;
-  if (!*last_flag) return true;
-  __threadfence();
-  if (row_active) merge_split_row(p, tw, tb, r, row);
-  if (r == 0) *ticket = 0;  // leave the workspace clean for the next call
   return true;
 }
 
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl, int warp, int lane,
                                              volatile int* abort_flag) {
   const uint32_t bars = sl.bars, tmem = sl.tmem;
-  volatile uint32_t* last_flag = sl.last_flag;
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
   const int r = (warp & 3) * 32 + lane;  // tile row == TMEM lane (warp w reaches lanes 32 (w % 4)..)
   const int half = r >> 6;               // warp-uniform: a warp's 32 rows lie in one half
@@ -596,7 +546,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
   const uint32_t obase = tmem + lane_addr + kTmemO;
   const float sl2 = p.scale_log2;
   uint32_t g = 0;
-  uint32_t n_epi = 0;  // uses of the epilogue barrier
   bool alive = true;
 
   TileDone pend{};
@@ -715,8 +664,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       ptx::mbar_arrive(bar(kBarPFull + static_cast<int>(sb)));
       if (n == 0 && have_pend) {  // the previous tile's epilogue, one chunk late
         have_pend = false;
-        if (!tile_epilogue(p, pend, sl.items[pend.k % kItemRing], bars, obase, warp, lane, abort_flag,
-                           last_flag, &n_epi)) {
+        if (!tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, bars, obase, warp, lane, abort_flag)) {
           alive = false;
           break;
         }
@@ -728,8 +676,9 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
     have_pend = true;
   }
   if (alive && have_pend &&
-      tile_epilogue(p, pend, sl.items[pend.k % kItemRing], bars, obase, warp, lane, abort_flag, last_flag, &n_epi))
+      tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, bars, obase, warp, lane, abort_flag))
     release_item_warp(sl, pend.k, lane);
+  if (lane == 0) ptx::bulk_wait_all();  // O stores complete before the CTA exits
 }
 
 __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -745,12 +694,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
       const uint32_t bars = base + s * kSlotBytes + kSmemBar;
       for (int i = 0; i < kNumBars; ++i) {
         uint32_t count = 1;
-        if ((i >= kBarPFull && i < kBarPFull + static_cast<int>(kSBufs)) || i == kBarOFree || i == kBarEpi)
-          count = kSoftmaxThreads;
+        if ((i >= kBarPFull && i < kBarPFull + static_cast<int>(kSBufs)) || i == kBarOFree) count = kSoftmaxThreads;
         if (i >= kBarItemEmpty && i < kBarItemEmpty + kItemRing) count = kItemReaders;
         ptx::mbar_init(bars + 8u * i, count);
       }
-      *reinterpret_cast<volatile uint32_t*>(smem + s * kSlotBytes + kSmemLast) = 0;
     }
     misc[1] = 0;
     ptx::fence_barrier_init();
@@ -759,6 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
     ptx::prefetch_tensormap(&p.tm_q);
     ptx::prefetch_tensormap(&p.tm_k);
     ptx::prefetch_tensormap(&p.tm_v);
+    ptx::prefetch_tensormap(&p.tm_o);
   }
   if (warp == kMmaWarp) {
     ptx::tmem_alloc(ptx::smem_addr(const_cast<uint32_t*>(&misc[0])), kTmemCols);
@@ -776,7 +724,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   sl.sV = base + slot * kSlotBytes + kSmemV;
   sl.bars = base + slot * kSlotBytes + kSmemBar;
   sl.items = reinterpret_cast<ItemStage*>(smem + slot * kSlotBytes + kSmemItems);
-  sl.last_flag = reinterpret_cast<volatile uint32_t*>(smem + slot * kSlotBytes + kSmemLast);
+  sl.ostage = smem + slot * kSlotBytes + kSmemOStage;
+  sl.sO = base + slot * kSlotBytes + kSmemOStage;
   sl.tmem = misc[0] + static_cast<uint32_t>(slot) * kSlotCols;
 
   if (warp < 8) {
@@ -796,6 +745,66 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == kMmaWarp) ptx::tmem_dealloc(misc[0], kTmemCols);
+}
+
+// Merge of split tiles: one warp per (batch element, split tile, tile row).  The
+// row's records were written by the forward's chunks of that tile: unnormalised O
+// relative to the chunk's max m (log2 units), m (-inf: the row attended nothing in
+// the chunk) and l.  O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c with M the
+// largest m_c; lse = (M + log2 of that sum) ln 2.  Lane x reduces records x, x + 32,
+// ... for M and the sum, then owns output columns 2x, 2x + 1, reading each record
+// row as one coalesced 256-byte line.
+struct MergeParams {
+  const float* partials;
+  const SplitTile* splits;
+  __nv_bfloat16* out;
+  float* lse;
+  int B, H, L, n_split, n_records;
+};
+
+__global__ void __launch_bounds__(128) bsa_merge_kernel(const __grid_constant__ MergeParams p) {
+  const int lane = threadIdx.x & 31;
+  const int task = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int per_b = p.n_split * kTileRows;
+  if (task >= p.B * per_b) return;
+  const int b = task / per_b, rem = task - b * per_b;
+  const int s = rem / kTileRows, r = rem - s * kTileRows;
+  const SplitTile st = p.splits[s];
+  const int qblk = (r >> 6) ? st.qb : st.qa;
+  if (qblk < 0) return;  // the unused half of a single-block tile
+  const size_t row = static_cast<size_t>(b * p.H + st.h) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
+  const float* base = p.partials + (static_cast<size_t>(b) * p.n_records + st.rec_base) * kRecFloats;
+  constexpr int kM = kTileRows * 64, kL = kTileRows * 64 + kTileRows;
+  const int nc = st.nchunks;
+  float ms = -INFINITY;
+  for (int x = lane; x < nc; x += 32) ms = fmaxf(ms, __ldcg(base + static_cast<size_t>(x) * kRecFloats + kM + r));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+  float lsum = 0.f;
+  if (ms != -INFINITY) {
+    for (int x = lane; x < nc; x += 32) {
+      const float* rc = base + static_cast<size_t>(x) * kRecFloats;
+      const float mc = __ldcg(rc + kM + r);
+      if (mc != -INFINITY) lsum += __ldcg(rc + kL + r) * ptx::ex2_approx(mc - ms);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  float2 acc = make_float2(0.f, 0.f);
+  if (ms != -INFINITY) {
+#pragma unroll 8
+    for (int x = 0; x < nc; ++x) {
+      const float* rc = base + static_cast<size_t>(x) * kRecFloats;
+      const float mc = __ldcg(rc + kM + r);
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(rc + r * 64) + lane);
+      const float f = mc == -INFINITY ? 0.f : ptx::ex2_approx(mc - ms);  // such a record's O is 0
+      acc.x += f * v.x;
+      acc.y += f * v.y;
+    }
+  }
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  reinterpret_cast<uint32_t*>(p.out + row * 64)[lane] = pack_bf16x2(acc.x * inv, acc.y * inv);
+  if (lane == 0) p.lse[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
 }
 
 // Per (b, key block): bit c set when key 64*j + c is kept by the padding mask.
@@ -842,12 +851,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows) {
+// [rows, 64] bf16 row-major tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
   auto fn = get_encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[2] = {64, rows};
   cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {64, 64};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -897,11 +907,13 @@ void free_device(bsa_layout* lay) {
     cudaFree(lay->d_pair_q);
     cudaFree(lay->d_pair_ent);
     cudaFree(lay->d_items);
+    cudaFree(lay->d_splits);
   }
   if (have_cur) cudaSetDevice(cur);
   lay->d_pair_q = nullptr;
   lay->d_pair_ent = nullptr;
   lay->d_items = nullptr;
+  lay->d_splits = nullptr;
   lay->device = -1;
 }
 
@@ -920,9 +932,11 @@ int bsa_layout_upload(bsa_layout* lay, void* stream) {
   const size_t bq = lay->pair_q.size() * sizeof(int32_t);
   const size_t be = lay->pair_ent.size() * sizeof(uint32_t);
   const size_t bi = lay->items.size() * sizeof(WorkItem);
+  const size_t bs = lay->splits.size() * sizeof(SplitTile);
   if (cudaMalloc(&lay->d_pair_q, std::max<size_t>(bq, 16)) != cudaSuccess ||
       cudaMalloc(&lay->d_pair_ent, std::max<size_t>(be, 16)) != cudaSuccess ||
-      cudaMalloc(&lay->d_items, std::max<size_t>(bi, 32)) != cudaSuccess) {
+      cudaMalloc(&lay->d_items, std::max<size_t>(bi, 32)) != cudaSuccess ||
+      cudaMalloc(&lay->d_splits, std::max<size_t>(bs, 32)) != cudaSuccess) {
     lay->device = dev;
     free_device(lay);
     return BSA_ERR_OOM;
@@ -931,6 +945,7 @@ int bsa_layout_upload(bsa_layout* lay, void* stream) {
   if (cudaMemcpyAsync(lay->d_pair_q, lay->pair_q.data(), bq, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(lay->d_pair_ent, lay->pair_ent.data(), be, cudaMemcpyHostToDevice, s) != cudaSuccess ||
       cudaMemcpyAsync(lay->d_items, lay->items.data(), bi, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      (bs > 0 && cudaMemcpyAsync(lay->d_splits, lay->splits.data(), bs, cudaMemcpyHostToDevice, s) != cudaSuccess) ||
       cudaStreamSynchronize(s) != cudaSuccess) {
     free_device(lay);
     return BSA_ERR_CUDA;
@@ -963,7 +978,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
 
   FwdParams prm{};
   const uint64_t rows = static_cast<uint64_t>(B) * H * L;
-  if (!make_map(&prm.tm_q, q, rows) || !make_map(&prm.tm_k, k, rows) || !make_map(&prm.tm_v, v, rows))
+  if (!make_map(&prm.tm_q, q, rows, 64) || !make_map(&prm.tm_k, k, rows, 64) ||
+      !make_map(&prm.tm_v, v, rows, 64) || !make_map(&prm.tm_o, out, rows, 32))
     return BSA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   prm.out = static_cast<__nv_bfloat16*>(out);
@@ -973,8 +989,7 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
   prm.pair_ent = lay->d_pair_ent;
   prm.keybits = key_mask ? reinterpret_cast<const unsigned long long*>(ws + plan.keybits_off) : nullptr;
   prm.partials = reinterpret_cast<float*>(ws + plan.partials_off);
-  prm.sched = reinterpret_cast<int*>(ws + plan.tickets_off);
-  prm.tickets = reinterpret_cast<int*>(ws + plan.tickets_off + kSchedBytes);
+  prm.sched = reinterpret_cast<int*>(ws + plan.sched_off);
   prm.B = B;
   prm.H = H;
   prm.L = L;
@@ -982,6 +997,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
   prm.items_per_batch = static_cast<int>(lay->items.size());
   prm.n_split = lay->n_split;
   prm.n_records = lay->n_records;
+  prm.split_items = static_cast<int>(std::count_if(lay->items.begin(), lay->items.end(),
+                                                   [](const WorkItem& it) { return it.split >= 0; }));
   const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(d));
   prm.scale_log2 = sc * kLog2e;
   prm.timeout_ns = kDefaultTimeoutNs;
@@ -999,6 +1016,21 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
   if (grid < 1) return BSA_OK;
   bsa_fwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  if (lay->n_split > 0) {
+    MergeParams mp{};
+    mp.partials = prm.partials;
+    mp.splits = lay->d_splits;
+    mp.out = prm.out;
+    mp.lse = lse;
+    mp.B = B;
+    mp.H = H;
+    mp.L = L;
+    mp.n_split = lay->n_split;
+    mp.n_records = lay->n_records;
+    const int64_t tasks = static_cast<int64_t>(B) * lay->n_split * kTileRows;
+    bsa_merge_kernel<<<static_cast<int>((tasks + 3) / 4), 128, 0, s>>>(mp);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  }
   return BSA_OK;
 }
 
@@ -1069,8 +1101,8 @@ extern "C" int bsa_forward_static_ws(const void* q, const void* k, const void* v
   });
   if (g_static_ws_err[dev] != cudaSuccess || g_static_ws_addr[dev] == nullptr) return BSA_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(g_static_ws_addr[dev]);
-  // the arrival tickets must start at zero; the other regions are written before read
-  if (cudaMemsetAsync(ws + plan.tickets_off, 0, plan.tickets_bytes, static_cast<cudaStream_t>(stream)) !=
+  // the schedule counters must start at zero; the other regions are written before read
+  if (cudaMemsetAsync(ws + plan.sched_off, 0, plan.sched_bytes, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return BSA_ERR_CUDA;
   return bsa_forward(q, k, v, B, H, L, d, lay, key_mask, scale, out, lse, ws, BSA_STATIC_WORKSPACE_BYTES,

@@ -154,9 +154,9 @@ namespace bsa {
 WorkspacePlan plan_workspace(const bsa_layout& lay, int B) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   WorkspacePlan p{};
-  p.tickets_off = 0;
-  p.tickets_bytes = up(kSchedBytes + sizeof(int32_t) * static_cast<size_t>(B) * lay.n_split);
-  p.keybits_off = p.tickets_off + p.tickets_bytes;
+  p.sched_off = 0;
+  p.sched_bytes = up(2 * sizeof(int32_t));
+  p.keybits_off = p.sched_off + p.sched_bytes;
   p.keybits_bytes = up(sizeof(uint64_t) * static_cast<size_t>(B) * lay.nb);
   p.partials_off = p.keybits_off + p.keybits_bytes;
   p.partials_bytes =
@@ -226,12 +226,12 @@ void build_tiles(bsa_layout* lay) {
       lay->pair_ptr.push_back(static_cast<int32_t>(lay->pair_ent.size()));
     }
   }
-  // Work items of one batch element, in the order they are handed out (the
-  // forward draws item i for every batch element before item i + 1): first the
-  // chunks of split tiles -- the longest items, and the ones whose last chunk
-  // merges the others -- then the other tiles, head-major so that items running
-  // at the same time share the head's K/V in L2.
+  // Work items of one batch element: first the chunks of split tiles (the forward
+  // hands these out first, for the whole batch: they are the longest items, and
+  // the last chunk of each merges the others), then the other tiles, head-major
+  // so that items running at the same time share the head's K/V in L2.
   lay->items.clear();
+  lay->splits.clear();
   lay->n_split = 0;
   lay->n_records = 0;
   for (const bool split_pass : {true, false}) {
@@ -249,6 +249,7 @@ void build_tiles(bsa_layout* lay) {
         const int slot = lay->n_split++;
         const int base = lay->n_records;
         lay->n_records += nch;
+        lay->splits.push_back(bsa::SplitTile{h, lay->pair_q[2 * p], lay->pair_q[2 * p + 1], base, nch, {0, 0, 0}});
         for (int c = 0; c < nch; ++c) {
           const int cs = c * bsa::kSplitChunk;
           lay->items.push_back(bsa::WorkItem{h, p, s + cs, std::min(bsa::kSplitChunk, U - cs),

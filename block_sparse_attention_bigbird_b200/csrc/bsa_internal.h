@@ -17,11 +17,11 @@ constexpr int kHeadDim = 64;
 constexpr int kTileRows = 128;
 
 // A tile whose key-block union is longer than kSplitThreshold is cut into
-// chunks of kSplitChunk union entries (even, so only a tile's last chunk can
-// hold a single key block).  Each chunk writes a partial (O, m, l) record; the
-// last chunk to finish merges them.
-constexpr int kSplitThreshold = 48;
-constexpr int kSplitChunk = 32;
+// chunks of kSplitChunk union entries, each run as its own work item.  Each chunk
+// writes a partial (O, m, l) record; a second kernel merges a split tile's records
+// into its output rows.
+constexpr int kSplitThreshold = BSA_SPLIT_THRESHOLD;
+constexpr int kSplitChunk = BSA_SPLIT_CHUNK;
 
 // Partial record of one split chunk: O[128][64] fp32 (unnormalised, relative to
 // the chunk's running max), then m[128] (log2 units, scaled) and l[128].
@@ -33,12 +33,20 @@ struct WorkItem {
   int32_t pair;      // tile (query-block pair) index within the head
   int32_t start;     // first entry in pair_ent (absolute index)
   int32_t count;     // number of union entries processed by this item (>= 1)
-  int32_t split;     // -1: whole tile; otherwise split-tile slot within a batch element
+  int32_t split;     // -1: whole tile; otherwise split-tile index within a batch element
   int32_t rec;       // partial record index within a batch element (split only)
   int32_t nchunks;   // number of chunks of the split tile
   int32_t rec_base;  // first record of the split tile within a batch element
 };
 static_assert(sizeof(WorkItem) == 32, "WorkItem must stay 32 bytes");
+
+// A split tile, for the merge: its head, query blocks (qb = -1: single block) and
+// its records [rec_base, rec_base + nchunks) within a batch element.
+struct SplitTile {
+  int32_t h, qa, qb, rec_base, nchunks;
+  int32_t pad[3];
+};
+static_assert(sizeof(SplitTile) == 32, "SplitTile must stay 32 bytes");
 
 constexpr uint32_t kEntColMask = 0x00FFFFFFu;
 constexpr int kEntBitsShift = 24;
@@ -57,6 +65,7 @@ struct bsa_layout {
   std::vector<int32_t> pair_ptr;    // H*n_pairs + 1
   std::vector<uint32_t> pair_ent;   // union entries
   std::vector<bsa::WorkItem> items; // schedule for ONE batch element (head-major)
+  std::vector<bsa::SplitTile> splits;  // the split tiles of one batch element
   int n_split = 0;                  // split tiles per batch element
   int n_records = 0;                // partial records per batch element
   // device copies (bsa_layout_upload)
@@ -64,20 +73,20 @@ struct bsa_layout {
   int32_t* d_pair_q = nullptr;
   uint32_t* d_pair_ent = nullptr;
   bsa::WorkItem* d_items = nullptr;
+  bsa::SplitTile* d_splits = nullptr;
 };
 
 namespace bsa {
 // Workspace carve-up for batch size B (all offsets 256-byte aligned).
 struct WorkspacePlan {
-  // [tickets_off, +tickets_bytes): the area that must be zero before a call and is
+  // [sched_off, +sched_bytes): the area that must be zero before a call and is
   // zero again after one: the work-item counter and finished-slot counter of the
-  // dynamic schedule (kSchedBytes), then one arrival ticket per split tile.
-  size_t tickets_off, tickets_bytes;
+  // dynamic schedule.
+  size_t sched_off, sched_bytes;
   size_t keybits_off, keybits_bytes;
   size_t partials_off, partials_bytes;
   size_t total;
 };
-constexpr size_t kSchedBytes = 16;
 WorkspacePlan plan_workspace(const bsa_layout& lay, int B);
 void free_device(bsa_layout* lay);
 }  // namespace bsa

@@ -113,6 +113,11 @@ int bsa_layout_globals(const bsa_layout* layout, const int32_t** globals, int* n
  *             ascending.
  * Any output may be NULL.
  */
+/* Tiles whose union has more than BSA_SPLIT_THRESHOLD entries (global rows) are
+ * cut into chunks of BSA_SPLIT_CHUNK entries; bsa_forward runs the chunks as
+ * separate work items and merges their partial results in a second kernel. */
+#define BSA_SPLIT_THRESHOLD 48
+#define BSA_SPLIT_CHUNK 32
 int bsa_layout_tiles(const bsa_layout* layout, const int32_t** pair_q, int* n_pairs,
                      const int32_t** pair_ptr, const uint32_t** pair_ent, int64_t* n_ent);
 
@@ -129,11 +134,12 @@ void bsa_layout_free(bsa_layout* layout);
 
 /*
  * bsa_workspace_bytes -- device scratch bytes bsa_forward needs for batch size
- * B: split-row partial results, their arrival tickets and the per-key-block
- * padding bits.  The workspace must be ZERO-FILLED before its first use; every
- * call that completes without a device error leaves the ticket area zero again,
- * so it can be reused without clearing.  After a call that ended in a device
- * error, clear it again.
+ * B: the counters of the dynamic work schedule, the per-key-block padding bits
+ * and the partial results of split rows (global rows whose key-block list is cut
+ * into chunks that run as separate work items).  The workspace must be
+ * ZERO-FILLED before its first use; every call that completes without a device
+ * error leaves the counters zero again, so it can be reused without clearing.
+ * After a call that ended in a device error, clear it again.
  */
 int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
 
@@ -150,6 +156,8 @@ int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
  *             attended set is empty.
  *   workspace device, at least bsa_workspace_bytes(layout, B) bytes, 256-byte
  *             aligned, zero-filled before first use (see above).
+ * Enqueues up to three kernels on `stream`: the key-padding bits (with a key
+ * mask), the forward, and the merge of split rows (when the layout has any).
  * Returns after enqueueing (no synchronisation, no allocation).  A device-side
  * timeout is reported later by bsa_sync_status.
  */
@@ -163,8 +171,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
  * memory: code running where cudaMalloc is unavailable or forbidden, e.g. inside
  * a host runtime that owns every allocation, a plugin with no allocator hook, or
  * a path where an allocation would synchronise the device.  It allocates
- * nothing: the scratch (split-row partials, their arrival tickets, key-padding
- * bits) lives in one buffer of BSA_STATIC_WORKSPACE_BYTES (32 MiB) compiled into
+ * nothing: the scratch (schedule counters, key-padding bits, split-row partials)
+ * lives in one buffer of BSA_STATIC_WORKSPACE_BYTES (32 MiB) compiled into
  * the library, which every GPU that loads the library holds until process exit.
  * The pages define no such entry point; it has no counterpart there.
  *
@@ -174,7 +182,7 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
  *   - The first call on a device looks up the buffer's device address for that
  *     device (cudaGetSymbolAddress, no allocation); make that first call before
  *     any stream capture.
- *   - Every call clears the buffer's ticket area with cudaMemsetAsync on
+ *   - Every call clears the buffer's schedule counters with cudaMemsetAsync on
  *     `stream`, then enqueues the forward.  All calls on a device share the one
  *     buffer, which keeps the last call's contents: calls whose execution
  *     overlaps on the GPU (different streams, no ordering between them) race on

@@ -20,6 +20,16 @@ def test_exports_every_header_symbol():
         assert f" T {n}\n" in dyn, n
 
 
+def test_binding_constants_match_header():
+    import os
+    import re
+    hdr = open(os.path.join(os.path.dirname(bsa.LIB_PATH), "..", "include", "bsa.h")).read()
+    defs = dict(re.findall(r"#define (BSA_\w+) \(?(\d+)u?", hdr))
+    assert int(defs["BSA_SPLIT_THRESHOLD"]) == bsa.SPLIT_THRESHOLD
+    m = re.search(r"#define BSA_STATIC_WORKSPACE_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", hdr)
+    assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == bsa.STATIC_WORKSPACE_BYTES
+
+
 def test_strerror_covers_codes():
     for code in range(0, -8, -1):
         assert bsa.bsa_strerror(code) != "unknown status"

@@ -150,7 +150,7 @@ def test_deterministic_and_workspace_left_clean(bsa):
     o2, l2 = bsa.bsa_forward(q, k, v, lay, workspace=ws)
     assert bsa.bsa_sync_status() == 0
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
-    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0   # tickets back at zero
+    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0   # schedule counters back at zero
 
 
 def test_bounded_wait_reports_timeout_and_context_survives(bsa):

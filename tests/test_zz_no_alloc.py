@@ -33,7 +33,7 @@ def test_static_entry_rejects_bad_arguments_without_a_gpu():
 @pytest.mark.gpu
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 def test_static_workspace_matches_workspace_forward_on_two_calls():
-    # global rows split across chunks (tickets + partial records) and partial key
+    # global rows split across chunks (partial records + merge) and partial key
     # padding (key bits): every region of the scratch buffer is exercised
     w = workloads.custom(2, 3, 64 * 64, 1, 2, 3, seed=1, key_pad_tail=100)
     q, k, v = [t.cuda() for t in workloads.make_qkv(w)]
