@@ -751,9 +751,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
 // row's records were written by the forward's chunks of that tile: unnormalised O
 // relative to the chunk's max m (log2 units), m (-inf: the row attended nothing in
 // the chunk) and l.  O = sum_c 2^(m_c - M) O_c / sum_c 2^(m_c - M) l_c with M the
-// largest m_c; lse = (M + log2 of that sum) ln 2.  Lane x reduces records x, x + 32,
-// ... for M and the sum, then owns output columns 2x, 2x + 1, reading each record
-// row as one coalesced 256-byte line.
+// largest m_c; lse = (M + log2 of that sum) ln 2.  The records are read in groups
+// of eight with every load of a group in flight at once, and folded into a running
+// (M, sum, O) -- the same rescaling the forward applies between chunks.  Lane x
+// owns output columns 2x, 2x + 1, so each record row is one coalesced 256-byte line.
 struct MergeParams {
   const float* partials;
   const SplitTile* splits;
@@ -763,6 +764,7 @@ struct MergeParams {
 };
 
 __global__ void __launch_bounds__(128) bsa_merge_kernel(const __grid_constant__ MergeParams p) {
+  constexpr int kGroup = 8;
   const int lane = threadIdx.x & 31;
   const int task = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int per_b = p.n_split * kTileRows;
@@ -776,35 +778,42 @@ __global__ void __launch_bounds__(128) bsa_merge_kernel(const __grid_constant__ 
   const float* base = p.partials + (static_cast<size_t>(b) * p.n_records + st.rec_base) * kRecFloats;
   constexpr int kM = kTileRows * 64, kL = kTileRows * 64 + kTileRows;
   const int nc = st.nchunks;
-  float ms = -INFINITY;
-  for (int x = lane; x < nc; x += 32) ms = fmaxf(ms, __ldcg(base + static_cast<size_t>(x) * kRecFloats + kM + r));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
-  float lsum = 0.f;
-  if (ms != -INFINITY) {
-    for (int x = lane; x < nc; x += 32) {
-      const float* rc = base + static_cast<size_t>(x) * kRecFloats;
-      const float mc = __ldcg(rc + kM + r);
-      if (mc != -INFINITY) lsum += __ldcg(rc + kL + r) * ptx::ex2_approx(mc - ms);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  float M = -INFINITY, lsum = 0.f;
   float2 acc = make_float2(0.f, 0.f);
-  if (ms != -INFINITY) {
-#pragma unroll 8
-    for (int x = 0; x < nc; ++x) {
+  for (int x0 = 0; x0 < nc; x0 += kGroup) {
+    float mg[kGroup], lg[kGroup];
+    float2 og[kGroup];
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      const int x = x0 + j < nc ? x0 + j : nc - 1;  // a repeated record gets weight 0 below
       const float* rc = base + static_cast<size_t>(x) * kRecFloats;
-      const float mc = __ldcg(rc + kM + r);
-      const float2 v = __ldcg(reinterpret_cast<const float2*>(rc + r * 64) + lane);
-      const float f = mc == -INFINITY ? 0.f : ptx::ex2_approx(mc - ms);  // such a record's O is 0
-      acc.x += f * v.x;
-      acc.y += f * v.y;
+      mg[j] = __ldcg(rc + kM + r);
+      lg[j] = __ldcg(rc + kL + r);
+      og[j] = __ldcg(reinterpret_cast<const float2*>(rc + r * 64) + lane);
     }
+    float gm = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j)
+      if (x0 + j < nc) gm = fmaxf(gm, mg[j]);
+    if (gm == -INFINITY) continue;  // no record of the group attended anything
+    const float Mn = fmaxf(M, gm);
+    const float a = M == -INFINITY ? 0.f : ptx::ex2_approx(M - Mn);
+    lsum *= a;
+    acc.x *= a;
+    acc.y *= a;
+#pragma unroll
+    for (int j = 0; j < kGroup; ++j) {
+      // a record whose row attended nothing has m = -inf and O = 0: weight 0
+      const float f = (x0 + j < nc && mg[j] != -INFINITY) ? ptx::ex2_approx(mg[j] - Mn) : 0.f;
+      lsum += f * lg[j];
+      acc.x += f * og[j].x;
+      acc.y += f * og[j].y;
+    }
+    M = Mn;
   }
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
   reinterpret_cast<uint32_t*>(p.out + row * 64)[lane] = pack_bf16x2(acc.x * inv, acc.y * inv);
-  if (lane == 0) p.lse[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
+  if (lane == 0) p.lse[row] = lsum > 0.f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
 }
 
 // Per (b, key block): bit c set when key 64*j + c is kept by the padding mask.

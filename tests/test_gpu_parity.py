@@ -66,6 +66,9 @@ SMALL = [
     ("all_global", workloads.custom(1, 1, 64 * 70, 0, 70, 0), 0, None),
     ("explicit_scale_sharp", workloads.custom(1, 2, 64 * 16, 1, 1, 2, k_mul=2.0), 0, 0.3),
     ("no_random_no_global", workloads.custom(2, 2, 64 * 9, 0, 0, 0), 0, None),
+    ("single_block", workloads.custom(1, 1, 64, 0, 1, 0), 0, None),
+    # logits with std ~16 (scale 1): later chunks often exceed the running max by far
+    ("huge_logits", workloads.custom(2, 2, 64 * 24, 2, 2, 3, seed=6, k_mul=2.0), 0, 1.0),
 ]
 
 
@@ -75,6 +78,23 @@ def test_parity_small_full(bsa, name, w, pad, scale):
     (q, k, v), _, ref_lay, o, lse = _run(bsa, w, key_mask=km, scale=scale)
     o_ref, lse_ref = OA.attention(q, k, v, ref_lay, key_mask=km, scale=scale)
     _check(o, lse, o_ref, lse_ref)
+
+
+def test_rising_scores_raise_the_running_max(bsa):
+    # Key norms grow by 2^4 along the sequence, so later chunks of a row keep
+    # exceeding the running max: the path that redoes a chunk with the larger max
+    # and rescales l and O runs many times per row.
+    w = workloads.custom(2, 2, 64 * 40, 2, 1, 3, seed=7)
+    q, k, v = workloads.make_qkv(w)
+    ramp = torch.exp2(4.0 * torch.arange(w.L, dtype=torch.float32) / w.L).view(1, 1, w.L, 1)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    lay = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(lay)
+    out, lse = bsa.bsa_forward(q.cuda(), k.cuda(), v.cuda(), lay, scale=0.5)
+    assert bsa.bsa_sync_status() == 0
+    ref = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    o_ref, lse_ref = OA.attention(q, k, v, ref, scale=0.5)
+    _check(out.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref)
 
 
 def test_fully_masked_rows_give_zero_and_neg_inf(bsa):
