@@ -91,6 +91,18 @@ def _has_split_rows(lay) -> bool:
     return bool(np.any(np.diff(pair_ptr) > bsa.SPLIT_THRESHOLD))
 
 
+def _ex2_ceiling(nnz_eff, kernel_ms, dev, peaks) -> dict:
+    """The second ceiling of this d = 64 forward: one ex2 per attended score (64 x 64
+    per non-zero block) on an ex2 unit that retires 16 results per clock per SM,
+    taken at the GPU's maximum SM clock."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    peak = 16.0 * sms * mhz * 1e6 / 1e9          # G ex2 / s
+    achieved = nnz_eff * 64 * 64 / (kernel_ms * 1e-3) / 1e9
+    return {"bound": "alu (ex2 unit)", "achieved": achieved, "peak": peak, "unit": "Gex2/s",
+            "frac": achieved / peak, "peak_source": f"16 per clock per SM x {sms} SMs x {mhz:.0f} MHz"}
+
+
 def _nnz_eff(w, row_ptr, col_idx) -> int:
     """Blocks over all (b, h, i, j), minus those whose 64 keys are all padded."""
     per_batch = int(len(col_idx))
@@ -389,8 +401,10 @@ def run_ours(args, w, world, rank, local):
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "bsa_fwd_kernel", "peak_source": f"{peak_src} bf16 burst",
-                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak))},
+                     "kernel": "bsa_fwd_kernel (+ bsa_merge_kernel when the layout has split rows)",
+                     "peak_source": f"{peak_src} bf16 burst",
+                     "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                     "ex2": _ex2_ceiling(nnz_eff, kernel_ms, dev, peaks)},
         "e2e": {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": launches_per_step * args.steps,
