@@ -33,6 +33,9 @@ _SIGNATURES = {
                                         ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
                                         ctypes.POINTER(ctypes.c_int32),
                                         ctypes.POINTER(ctypes.c_void_p)]),
+    "bsa_layout_from_csr": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
+                                           ctypes.POINTER(ctypes.c_void_p)]),
     "bsa_layout_csr": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p),
                                       ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int64),
                                       ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
@@ -130,6 +133,21 @@ def bsa_layout_build(H: int, L: int, block: int = 64, window: int = 1, n_global:
     _check(lib.bsa_layout_build(H, L, block, window, n_global, n_random,
                                 ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), gptr, ctypes.byref(out)),
            "bsa_layout_build")
+    return Layout(out.value, H, L)
+
+
+def bsa_layout_from_csr(H: int, L: int, row_ptr, col_idx, block: int = 64) -> Layout:
+    """Layout from a caller's block CSR (rows head-major; see bsa_layout_from_csr in bsa.h)."""
+    rp = np.ascontiguousarray(np.asarray(row_ptr, dtype=np.int32))
+    ci = np.ascontiguousarray(np.asarray(col_idx, dtype=np.int32))
+    if rp.ndim != 1 or rp.size != H * (L // block if block > 0 else 0) + 1:
+        raise BsaError(BSA_ERR_INVALID_ARG, "bsa_layout_from_csr: row_ptr must hold H * L / block + 1 entries")
+    if int(rp[-1]) > ci.size:
+        raise BsaError(BSA_ERR_INVALID_ARG, "bsa_layout_from_csr: col_idx is shorter than row_ptr[-1]")
+    out = ctypes.c_void_p()
+    cptr = ci.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)) if ci.size else None
+    _check(lib.bsa_layout_from_csr(H, L, block, rp.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cptr,
+                                   ctypes.byref(out)), "bsa_layout_from_csr")
     return Layout(out.value, H, L)
 
 

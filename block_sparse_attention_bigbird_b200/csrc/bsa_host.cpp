@@ -223,6 +223,10 @@ void build_tiles(bsa_layout* lay) {
         if (x < only_a.size()) lay->pair_ent.push_back(only_a[x]);
         if (x < only_b.size()) lay->pair_ent.push_back(only_b[x]);
       }
+      // A tile whose rows are all empty (possible in a caller's CSR) still runs one
+      // entry so that its output rows get written (O = 0, lse = -inf): key block 0
+      // with no membership bit, which neither half attends.
+      if (both.empty() && only_a.empty() && only_b.empty()) lay->pair_ent.push_back(0u);
       lay->pair_ptr.push_back(static_cast<int32_t>(lay->pair_ent.size()));
     }
   }
@@ -321,6 +325,70 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
         lay->row_ptr.push_back(static_cast<int32_t>(lay->col_idx.size()));
       }
     }
+    build_tiles(lay);
+    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
+      delete lay;
+      return BSA_ERR_INVALID_ARG;
+    }
+  } catch (const std::bad_alloc&) {
+    delete lay;
+    return BSA_ERR_OOM;
+  } catch (...) {
+    delete lay;
+    return BSA_ERR_INVALID_ARG;
+  }
+  *out = lay;
+  return BSA_OK;
+}
+
+int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const int32_t* col_idx,
+                        bsa_layout** out) {
+  if (out == nullptr) return BSA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (block != bsa::kBlock) return BSA_ERR_UNSUPPORTED;
+  if (H < 1 || L < 1 || L % block != 0 || row_ptr == nullptr) return BSA_ERR_INVALID_ARG;
+  const int nb = L / block;
+  if (nb > static_cast<int>(bsa::kEntColMask) || static_cast<int64_t>(H) * nb > (1 << 30))
+    return BSA_ERR_INVALID_ARG;
+  const size_t n_rows = static_cast<size_t>(H) * nb;
+  // row_ptr: starts at 0, never decreases; col_idx may be NULL only if it is empty
+  if (row_ptr[0] != 0) return BSA_ERR_INVALID_ARG;
+  for (size_t x = 0; x < n_rows; ++x)
+    if (row_ptr[x + 1] < row_ptr[x]) return BSA_ERR_INVALID_ARG;
+  const int64_t nnz_in = row_ptr[n_rows];
+  if (nnz_in > 0 && col_idx == nullptr) return BSA_ERR_INVALID_ARG;
+  for (int64_t x = 0; x < nnz_in; ++x)
+    if (col_idx[x] < 0 || col_idx[x] >= nb) return BSA_ERR_INVALID_ARG;
+  bsa_layout* lay = new (std::nothrow) bsa_layout();
+  if (lay == nullptr) return BSA_ERR_OOM;
+  try {
+    lay->H = H;
+    lay->L = L;
+    lay->block = block;
+    lay->nb = nb;
+    lay->window = -1;  // not a generated layout
+    lay->n_random = -1;
+    // rows sorted ascending and deduplicated
+    lay->row_ptr.reserve(n_rows + 1);
+    lay->row_ptr.push_back(0);
+    lay->col_idx.reserve(static_cast<size_t>(nnz_in));
+    std::vector<int32_t> row;
+    // dense[i]: query block i lists every key block in every head
+    std::vector<uint8_t> dense(static_cast<size_t>(nb), 1);
+    for (size_t x = 0; x < n_rows; ++x) {
+      row.assign(col_idx + row_ptr[x], col_idx + row_ptr[x + 1]);
+      std::sort(row.begin(), row.end());
+      row.erase(std::unique(row.begin(), row.end()), row.end());
+      if (static_cast<int>(row.size()) != nb) dense[x % static_cast<size_t>(nb)] = 0;
+      lay->col_idx.insert(lay->col_idx.end(), row.begin(), row.end());
+      lay->row_ptr.push_back(static_cast<int32_t>(lay->col_idx.size()));
+    }
+    // The dense query blocks play the part of BigBird's global blocks in the
+    // pairing: they pair with each other, so that no sparse row is paired with a
+    // full one.
+    for (int i = 0; i < nb; ++i)
+      if (dense[static_cast<size_t>(i)]) lay->globals.push_back(i);
+    lay->n_global = static_cast<int>(lay->globals.size());
     build_tiles(lay);
     if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
       delete lay;

@@ -91,6 +91,38 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
                      uint64_t seed, const int32_t* globals, bsa_layout** out);
 
 /*
+ * bsa_layout_from_csr -- host only, no GPU needed.
+ *
+ * Builds a layout from a caller's block mask instead of the BigBird rule.
+ * The pages keep the attention mask as a 0/1 matrix over 64x64 blocks
+ * ("Transformer计算效率优化：SQA稀疏注意力机制详解", 3.1), and that is the CSR
+ * form taken here.
+ *   row_ptr  host, H*nb+1 int32 (nb = L / block): row (h, i), the key blocks
+ *            query block i of head h attends, is col_idx[row_ptr[h*nb+i] ..
+ *            row_ptr[h*nb+i+1]).  Rows are head-major.  row_ptr[0] must be 0
+ *            and row_ptr must never decrease.
+ *   col_idx  host, row_ptr[H*nb] int32 key block indices in [0, nb).  Within a
+ *            row: any order, duplicates allowed; the layout keeps each row
+ *            sorted and duplicate-free (bsa_layout_csr returns that form).
+ *            May be NULL when row_ptr[H*nb] == 0.
+ * A row may be empty: its query tokens get O = 0 and lse = -inf.  Rows may
+ * differ between heads.  A query block that lists every key block in every
+ * head is paired with other such blocks in the tile decomposition; such
+ * blocks are what bsa_layout_globals returns for this layout.
+ *
+ * Rows that list every key block are how caller-chosen global query rows are
+ * expressed, e.g. the top-k queries an SQA router picks for global attention
+ * ("Transformer计算效率优化：SQA稀疏注意力机制详解", 2.1), the others keeping a
+ * local window.
+ *
+ * block must be 64 (else BSA_ERR_UNSUPPORTED).  BSA_ERR_INVALID_ARG for
+ * H < 1, L < 1, L % block != 0, a NULL row_ptr, a bad row_ptr or a column
+ * out of range.  The arrays are copied; the caller keeps ownership.
+ */
+int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const int32_t* col_idx,
+                        bsa_layout** out);
+
+/*
  * bsa_layout_csr -- host views of the CSR: row_ptr has H*nb+1 int32 entries,
  * col_idx has nnz int32 entries (key block indices).  Any output pointer may be
  * NULL.  The views stay valid until bsa_layout_free.

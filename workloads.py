@@ -110,3 +110,48 @@ def make_key_mask(w: Workload) -> Optional[torch.Tensor]:
     m = torch.ones((w.B, w.L), dtype=torch.uint8)
     m[:, w.L - w.key_pad_tail:] = 0
     return m
+
+
+def make_block_csr(H: int, nb: int, seed: int, p_empty: float = 0.1, p_full: float = 0.05,
+                   max_len: Optional[int] = None, full_blocks=()):
+    """A caller's block mask in CSR form (rows head-major), seeded.
+
+    Each row (h, i) is empty with probability ``p_empty``, lists every key block
+    with probability ``p_full`` and otherwise holds 1..max_len blocks drawn with
+    replacement, in the drawn order (so rows come unsorted and may repeat a
+    block).  Query blocks in ``full_blocks`` list every key block in every head.
+    Returns (row_ptr int32 [H*nb+1], col_idx int32 [nnz]).
+    """
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    max_len = max_len or max(1, nb // 3)
+    full = set(int(x) for x in full_blocks)
+    row_ptr, cols = [0], []
+    for _h in range(H):
+        for i in range(nb):
+            u = rng.random()
+            if i in full or (u >= p_empty and u < p_empty + p_full):
+                row = list(rng.permutation(nb))
+            elif u < p_empty:
+                row = []
+            else:
+                row = list(rng.integers(0, nb, size=int(rng.integers(1, max_len + 1))))
+            cols.extend(int(c) for c in row)
+            row_ptr.append(len(cols))
+    return np.asarray(row_ptr, dtype=np.int32), np.asarray(cols, dtype=np.int32)
+
+
+def make_router_csr(H: int, nb: int, k_global: int, window: int, seed: int):
+    """Block CSR of a router-style layout, seeded: in each head ``k_global`` query
+    blocks drawn at random list every key block; every other query block i
+    lists the blocks j with |i - j| <= window.  Rows head-major, ascending."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    row_ptr, cols = [0], []
+    for _h in range(H):
+        chosen = set(int(x) for x in rng.choice(nb, size=min(k_global, nb), replace=False))
+        for i in range(nb):
+            row = range(nb) if i in chosen else range(max(0, i - window), min(nb, i + window + 1))
+            cols.extend(row)
+            row_ptr.append(len(cols))
+    return np.asarray(row_ptr, dtype=np.int32), np.asarray(cols, dtype=np.int32)
