@@ -1,0 +1,87 @@
+"""Oracle gradients of the block-sparse attention in fp64 (numpy).  TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg
+may import this module.  It shares no code with the CUDA library.
+
+What is differentiated: the forward of ``oracle.attention``, i.e. the masked
+attention Softmax(Q K^T / sqrt(d_k) (.) M) V of "Adapt or Perish: 新手入门指南 –
+Adaptive Sparse Transformer 核心原理与实战" (sparse-attention formula), with
+(.) M read as restricting the softmax to M and a key-padding mask removing keys.
+The pages train these models ("BERT 稀疏注意力机制入门指南", 生产环境部署建议:
+mixed-precision training, gradient checkpointing; "BigBird 稀疏注意力机制解析",
+避坑指南: mixed precision, gradient checkpointing) but print no gradient
+formula, so the gradient is the plain derivative of that forward.
+
+For a loss whose gradient with respect to O is dO, with S = Q K^T * scale
+restricted to the attended keys and P = softmax(S) row by row:
+    dV  = P^T dO
+    dP  = dO V^T
+    dS  = P (.) (dP - D),   D = rowsum(P (.) dP)        (the softmax Jacobian)
+    dQ  = dS K * scale,     dK = dS^T Q * scale
+Entries outside the attended set have P = 0 and hence dS = 0; a row with no
+attended key has P = 0 and contributes nothing.
+
+The computation is masked-dense like the forward: for each query block the
+scores against all L keys are formed, the excluded entries get P = 0, and the
+four products above are taken over the full key range.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from .attention import _as_f64, token_mask_row
+
+
+def attention_backward(q, k, v, dout, layout: dict, key_mask=None, scale=None,
+                       with_magnitude: bool = False):
+    """dq, dk, dv [B,H,L,d] in fp64 for the loss gradient ``dout`` = dL/dO.
+
+    With ``with_magnitude`` also returns, per output element, the sum of the
+    absolute values of the terms it is summed from (same shapes):
+      |dq|-terms  scale * (P (.) (|dP| + |D|)) |K|
+      |dk|-terms  scale * (P (.) (|dP| + |D|))^T |Q|
+      |dv|-terms  P^T |dO|
+    These bound the effect of rounding P, dS or D by a relative amount on the
+    result, which is what a tolerance needs.
+    """
+    q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    B, H, L, d = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    km = None if key_mask is None else _as_f64(key_mask) != 0
+    block, nb = layout["block"], layout["nb"]
+    assert layout["H"] == H and layout["L"] == L
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    if with_magnitude:
+        mq, mk, mv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            kb, vb = k[b, h], v[b, h]
+            for i in range(nb):
+                rows = slice(i * block, (i + 1) * block)
+                allowed = token_mask_row(layout, h, i, L)
+                if km is not None:
+                    allowed = allowed & km[b]
+                s = np.where(allowed, (q[b, h, rows] @ kb.T) * scale, -np.inf)
+                mx = s.max(axis=-1, keepdims=True)
+                empty = ~np.isfinite(mx)
+                e = np.exp(s - np.where(empty, 0.0, mx))          # 0 where excluded
+                den = e.sum(axis=-1, keepdims=True)
+                p = np.where(empty, 0.0, e / np.where(empty, 1.0, den))
+                dp = do[b, h, rows] @ vb.T
+                D = (p * dp).sum(axis=-1, keepdims=True)
+                ds = p * (dp - D)
+                dq[b, h, rows] = (ds @ kb) * scale
+                dk[b, h] += (ds.T @ q[b, h, rows]) * scale
+                dv[b, h] += p.T @ do[b, h, rows]
+                if with_magnitude:
+                    w = p * (np.abs(dp) + np.abs(D))
+                    mq[b, h, rows] = (w @ np.abs(kb)) * scale
+                    mk[b, h] += (w.T @ np.abs(q[b, h, rows])) * scale
+                    mv[b, h] += p.T @ np.abs(do[b, h, rows])
+    if with_magnitude:
+        return dq, dk, dv, (mq, mk, mv)
+    return dq, dk, dv
