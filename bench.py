@@ -54,12 +54,18 @@ def _peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+# The sources the forward kernel is compiled from (its own file and what it includes).
+FWD_SOURCES = ("bsa_fwd_sm100.cu", "bsa_internal.h", "bsa_wait.cuh", "bsa_host_cuda.h", "sm100_ptx.cuh")
+
+
 def _source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_attention_bigbird_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in FWD_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
+    with open(os.path.join(ROOT, "include", "bsa.h"), "rb") as f:
+        h.update(b"bsa.h" + f.read())
     return h.hexdigest()[:16]
 
 

@@ -56,6 +56,16 @@ _SIGNATURES = {
                                              ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                              ctypes.c_void_p]),
+    "bsa_layout_key_tiles": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p),
+                                            ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_void_p),
+                                            ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int64)]),
+    "bsa_backward_workspace_bytes": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int,
+                                                    ctypes.POINTER(ctypes.c_size_t)]),
+    "bsa_backward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_size_t, ctypes.c_void_p]),
     "bsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p]),
@@ -186,6 +196,20 @@ def bsa_layout_tiles(layout: Layout):
     return pair_q.reshape(P, 2), pair_ptr, pair_ent
 
 
+def bsa_layout_key_tiles(layout: Layout):
+    """(pair_k [n_pairs, 2], pair_ptr [H*n_pairs+1], pair_ent [n_ent] uint32) of the key-major tiles."""
+    pq, pp, pe = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+    n_pairs, n_ent = ctypes.c_int(), ctypes.c_int64()
+    _check(lib.bsa_layout_key_tiles(layout.handle, ctypes.byref(pq), ctypes.byref(n_pairs), ctypes.byref(pp),
+                                    ctypes.byref(pe), ctypes.byref(n_ent)), "bsa_layout_key_tiles")
+    P = n_pairs.value
+    pair_k = np.ctypeslib.as_array(ctypes.cast(pq, ctypes.POINTER(ctypes.c_int32)), (2 * P,)).copy()
+    pair_ptr = np.ctypeslib.as_array(ctypes.cast(pp, ctypes.POINTER(ctypes.c_int32)),
+                                     (layout.H * P + 1,)).copy()
+    pair_ent = np.ctypeslib.as_array(ctypes.cast(pe, ctypes.POINTER(ctypes.c_uint32)), (n_ent.value,)).copy()
+    return pair_k.reshape(P, 2), pair_ptr, pair_ent
+
+
 def bsa_layout_upload(layout: Layout, stream=None) -> None:
     _check(lib.bsa_layout_upload(layout.handle, ctypes.c_void_p(_stream_ptr(stream))), "bsa_layout_upload")
     layout._workspaces.clear()
@@ -264,6 +288,53 @@ def bsa_forward_static_ws(q, k, v, layout: Layout, key_mask=None, scale: Optiona
                                      lse.data_ptr(), ctypes.c_void_p(_stream_ptr(stream)))
     _check(code, "bsa_forward_static_ws")
     return out, lse
+
+
+def bsa_backward_workspace_bytes(layout: Layout, B: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib.bsa_backward_workspace_bytes(layout.handle, B, ctypes.byref(n)), "bsa_backward_workspace_bytes")
+    return n.value
+
+
+def bsa_backward(q, k, v, out, dout, lse, layout: Layout, key_mask=None, scale: Optional[float] = None,
+                 dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dq, dk, dv (bf16 [B,H,L,64]) of the block-sparse attention for dL/dO = ``dout``.
+
+    q, k, v, out, dout: contiguous bf16 CUDA tensors [B, H, L, 64]; out and lse
+    (fp32 [B, H, L]) are the forward's results for the same inputs, layout,
+    key_mask and scale.  workspace: optional uint8 CUDA tensor of at least
+    bsa_backward_workspace_bytes(layout, B) bytes (no clearing needed); when
+    omitted a cached one of the layout is used.
+    """
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 4:
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor [B, H, L, d]")
+        if t.shape != q.shape:
+            raise ValueError(f"{name} shape differs from q")
+    B, H, L, d = q.shape
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, L) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 tensor [B, H, L]")
+    if key_mask is not None:
+        if key_mask.dtype != torch.uint8 or tuple(key_mask.shape) != (B, L) or not key_mask.is_contiguous():
+            raise ValueError("key_mask must be a contiguous uint8 tensor [B, L]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        key = ("bwd", str(q.device), B)
+        workspace = layout._workspaces.get(key)
+        if workspace is None:
+            workspace = torch.empty(bsa_backward_workspace_bytes(layout, B), dtype=torch.uint8, device=q.device)
+            layout._workspaces[key] = workspace
+    code = lib.bsa_backward(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(),
+                            lse.data_ptr(), B, H, L, d, layout.handle,
+                            key_mask.data_ptr() if key_mask is not None else None,
+                            ctypes.c_float(scale if scale is not None else 0.0), dq.data_ptr(), dk.data_ptr(),
+                            dv.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                            ctypes.c_void_p(_stream_ptr(stream)))
+    _check(code, "bsa_backward")
+    return dq, dk, dv
 
 
 def bsa_sync_status(stream=None) -> int:

@@ -46,6 +46,8 @@
 
 #include "bsa_internal.h"
 #include "sm100_ptx.cuh"
+#include "bsa_wait.cuh"
+#include "bsa_host_cuda.h"
 
 namespace bsa {
 
@@ -66,11 +68,6 @@ constexpr uint32_t kSBufs = 3;               // S buffers of 64 columns at +0, +
 constexpr uint32_t kTmemS = 0;
 constexpr uint32_t kTmemO = 192;             // O at +192
 constexpr float kLazyBound = 4096.0f;  // 2^kLazyLog2, kLazyLog2 = 12: bound on a chunk's sum of p
-constexpr float kLn2 = 0.69314718055994530942f;
-constexpr float kLog2e = 1.44269504088896340736f;
-constexpr uint32_t kMaxSpin = 1u << 24;
-constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
-constexpr uint32_t kWaitSleepNs = 20000;  // upper bound on one sleep inside a barrier wait
 
 // shared memory map of one slot (offsets from its 1024-aligned base)
 constexpr uint32_t kSmemQ = 0;
@@ -147,54 +144,6 @@ struct FwdParams {
   float scale_log2;
   unsigned long long timeout_ns;
 };
-
-__device__ int g_bsa_status;
-
-// ------------------------------------------------------------ bounded waits
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       uint64_t timeout_ns, bool honor_abort) {
-  const uint64_t t0 = ptx::globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    // sleeping in the barrier instead of spinning leaves issue slots to the
-    // warps that share this SM sub-partition
-    if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
-    if ((it & 15u) == 0) {
-      if (honor_abort && *abort_flag) return false;
-      if (ptx::globaltimer_ns() - t0 > timeout_ns || it > kMaxSpin) {
-        *abort_flag = 1;
-        atomicCAS(&g_bsa_status, 0, static_cast<int>(BSA_ERR_DEVICE_TIMEOUT));
-        return false;
-      }
-    }
-  }
-}
-
-// Whole-warp wait; the result is warp-uniform.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint64_t timeout_ns) {
-  bool ok = ptx::mbar_try_wait(bar, parity);
-  if (__all_sync(0xffffffffu, ok)) return true;
-  ok = wait_slow(bar, parity, abort_flag, timeout_ns, true);
-  return __all_sync(0xffffffffu, ok);
-}
-
-__device__ __forceinline__ void wait_force(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                           uint64_t timeout_ns) {
-  if (!ptx::mbar_try_wait(bar, parity)) wait_slow(bar, parity, abort_flag, timeout_ns, false);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// ------------------------------------------------------------ roles
-// Single-thread wait (the TMA and MMA roles run on one elected lane).
-__device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                         uint64_t timeout_ns) {
-  if (ptx::mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, abort_flag, timeout_ns, true);
-}
 
 constexpr int kItemNone = -1;   // no work left
 constexpr int kItemAbort = -2;  // a wait gave up
@@ -860,6 +809,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // [rows, 64] bf16 row-major tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
   auto fn = get_encode_fn();
@@ -872,6 +823,15 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows)
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+cudaError_t launch_keybits(const uint8_t* key_mask, unsigned long long* bits, int B, int L, int nb,
+                           cudaStream_t s) {
+  const int n = B * nb;
+  bsa_keybits_kernel<<<(n + 255) / 256, 256, 0, s>>>(key_mask, bits, B, L, nb);
+  return cudaGetLastError();
+}
+
+namespace {
 
 struct DeviceInfo {
   int sms = 0;
@@ -917,12 +877,24 @@ void free_device(bsa_layout* lay) {
     cudaFree(lay->d_pair_ent);
     cudaFree(lay->d_items);
     cudaFree(lay->d_splits);
+    cudaFree(lay->d_kpair_q);
+    cudaFree(lay->d_kpair_ent);
+    cudaFree(lay->d_dq_items);
+    cudaFree(lay->d_dkv_items);
+    cudaFree(lay->d_dq_splits);
+    cudaFree(lay->d_dkv_splits);
   }
   if (have_cur) cudaSetDevice(cur);
   lay->d_pair_q = nullptr;
   lay->d_pair_ent = nullptr;
   lay->d_items = nullptr;
   lay->d_splits = nullptr;
+  lay->d_kpair_q = nullptr;
+  lay->d_kpair_ent = nullptr;
+  lay->d_dq_items = nullptr;
+  lay->d_dkv_items = nullptr;
+  lay->d_dq_splits = nullptr;
+  lay->d_dkv_splits = nullptr;
   lay->device = -1;
 }
 
@@ -938,24 +910,44 @@ int bsa_layout_upload(bsa_layout* lay, void* stream) {
   if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
   free_device(lay);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t bq = lay->pair_q.size() * sizeof(int32_t);
-  const size_t be = lay->pair_ent.size() * sizeof(uint32_t);
-  const size_t bi = lay->items.size() * sizeof(WorkItem);
-  const size_t bs = lay->splits.size() * sizeof(SplitTile);
-  if (cudaMalloc(&lay->d_pair_q, std::max<size_t>(bq, 16)) != cudaSuccess ||
-      cudaMalloc(&lay->d_pair_ent, std::max<size_t>(be, 16)) != cudaSuccess ||
-      cudaMalloc(&lay->d_items, std::max<size_t>(bi, 32)) != cudaSuccess ||
-      cudaMalloc(&lay->d_splits, std::max<size_t>(bs, 32)) != cudaSuccess) {
-    lay->device = dev;
-    free_device(lay);
-    return BSA_ERR_OOM;
-  }
+  // (device pointer, host data, bytes) of every table the kernels read
+  struct Table {
+    void** dst;
+    const void* src;
+    size_t bytes;
+  };
+  const Table tables[] = {
+      {reinterpret_cast<void**>(&lay->d_pair_q), lay->pair_q.data(), lay->pair_q.size() * sizeof(int32_t)},
+      {reinterpret_cast<void**>(&lay->d_pair_ent), lay->pair_ent.data(), lay->pair_ent.size() * sizeof(uint32_t)},
+      {reinterpret_cast<void**>(&lay->d_items), lay->items.data(), lay->items.size() * sizeof(WorkItem)},
+      {reinterpret_cast<void**>(&lay->d_splits), lay->splits.data(), lay->splits.size() * sizeof(SplitTile)},
+      {reinterpret_cast<void**>(&lay->d_kpair_q), lay->ktiles.pair_q.data(),
+       lay->ktiles.pair_q.size() * sizeof(int32_t)},
+      {reinterpret_cast<void**>(&lay->d_kpair_ent), lay->ktiles.pair_ent.data(),
+       lay->ktiles.pair_ent.size() * sizeof(uint32_t)},
+      {reinterpret_cast<void**>(&lay->d_dq_items), lay->dq_plan.items.data(),
+       lay->dq_plan.items.size() * sizeof(BwdItem)},
+      {reinterpret_cast<void**>(&lay->d_dkv_items), lay->dkv_plan.items.data(),
+       lay->dkv_plan.items.size() * sizeof(BwdItem)},
+      {reinterpret_cast<void**>(&lay->d_dq_splits), lay->dq_plan.splits.data(),
+       lay->dq_plan.splits.size() * sizeof(SplitTile)},
+      {reinterpret_cast<void**>(&lay->d_dkv_splits), lay->dkv_plan.splits.data(),
+       lay->dkv_plan.splits.size() * sizeof(SplitTile)},
+  };
   lay->device = dev;
-  if (cudaMemcpyAsync(lay->d_pair_q, lay->pair_q.data(), bq, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(lay->d_pair_ent, lay->pair_ent.data(), be, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(lay->d_items, lay->items.data(), bi, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      (bs > 0 && cudaMemcpyAsync(lay->d_splits, lay->splits.data(), bs, cudaMemcpyHostToDevice, s) != cudaSuccess) ||
-      cudaStreamSynchronize(s) != cudaSuccess) {
+  for (const Table& t : tables) {
+    if (cudaMalloc(t.dst, std::max<size_t>(t.bytes, 32)) != cudaSuccess) {
+      free_device(lay);
+      return BSA_ERR_OOM;
+    }
+  }
+  for (const Table& t : tables) {
+    if (t.bytes > 0 && cudaMemcpyAsync(*t.dst, t.src, t.bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+      free_device(lay);
+      return BSA_ERR_CUDA;
+    }
+  }
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
     free_device(lay);
     return BSA_ERR_CUDA;
   }
@@ -1013,12 +1005,10 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
   prm.timeout_ns = kDefaultTimeoutNs;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (key_mask != nullptr) {
-    const int n = B * lay->nb;
-    bsa_keybits_kernel<<<(n + 255) / 256, 256, 0, s>>>(
-        key_mask, reinterpret_cast<unsigned long long*>(ws + plan.keybits_off), B, L, lay->nb);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
-  }
+  if (key_mask != nullptr &&
+      launch_keybits(key_mask, reinterpret_cast<unsigned long long*>(ws + plan.keybits_off), B, L, lay->nb, s) !=
+          cudaSuccess)
+    return BSA_ERR_CUDA;
   const int64_t total = static_cast<int64_t>(B) * prm.items_per_batch;
   // two slots per CTA; items are drawn dynamically
   const int grid = static_cast<int>(std::min<int64_t>((total + kSlots - 1) / kSlots, info.sms));
@@ -1051,7 +1041,8 @@ int bsa_sync_status(void* stream) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_bsa_status, &zero, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
   }
-  return st;
+  const int st_bwd = bwd_take_status();  // the backward kernels' status word
+  return st != 0 ? st : st_bwd;
 }
 
 int bsa_debug_wait_timeout(uint64_t timeout_ns, void* stream) {

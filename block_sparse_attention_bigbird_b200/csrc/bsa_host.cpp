@@ -165,46 +165,59 @@ WorkspacePlan plan_workspace(const bsa_layout& lay, int B) {
   return p;
 }
 
+BwdWorkspacePlan plan_bwd_workspace(const bsa_layout& lay, int B) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t rows = static_cast<size_t>(B) * lay.H * lay.L;
+  BwdWorkspacePlan p{};
+  p.keybits_off = 0;
+  p.dsum_off = up(sizeof(uint64_t) * static_cast<size_t>(B) * lay.nb);
+  p.lse2_off = p.dsum_off + up(sizeof(float) * rows);
+  p.dq_rec_off = p.lse2_off + up(sizeof(float) * rows);
+  p.dkv_rec_off = p.dq_rec_off + up(sizeof(float) * kBwdDqRecFloats * static_cast<size_t>(B) * lay.dq_plan.n_records);
+  p.total = p.dkv_rec_off + up(sizeof(float) * kBwdDkvRecFloats * static_cast<size_t>(B) * lay.dkv_plan.n_records);
+  return p;
+}
+
 }  // namespace bsa
 
 namespace {
 
-void build_tiles(bsa_layout* lay) {
-  const int nb = lay->nb, H = lay->H;
-  std::vector<uint8_t> is_global(static_cast<size_t>(nb), 0);
-  for (int g : lay->globals) is_global[static_cast<size_t>(g)] = 1;
-  // Pairs: global blocks with global blocks, the others with the others, in
-  // ascending order; an odd one out forms a single-block tile.
+// Tiles of 128 rows over a block CSR (H x nb rows, head-major): rows paired in
+// ascending order, the dense ones (flagged) with each other and the others with
+// each other; an odd one out forms a single-row tile.  Per tile and head the
+// entries are the union of the two rows with membership bits: the blocks in both
+// rows, then the blocks in one row only, alternating first/second, each group
+// ascending.  The order is free (one softmax over the union), and this one keeps
+// the two halves of the tile -- whose warps skip the work of a block their half
+// does not take part in -- doing equal work chunk by chunk.
+void make_tiles(int H, int nb, const std::vector<int32_t>& row_ptr, const std::vector<int32_t>& col_idx,
+                const std::vector<uint8_t>& dense, std::vector<int32_t>* pair_q, int* n_pairs,
+                std::vector<int32_t>* pair_ptr, std::vector<uint32_t>* pair_ent) {
   std::vector<int32_t> gl, ng;
-  for (int i = 0; i < nb; ++i) (is_global[static_cast<size_t>(i)] ? gl : ng).push_back(i);
-  lay->pair_q.clear();
+  for (int i = 0; i < nb; ++i) (dense[static_cast<size_t>(i)] ? gl : ng).push_back(i);
+  pair_q->clear();
   for (const auto* lst : {&gl, &ng}) {
     for (size_t x = 0; x < lst->size(); x += 2) {
-      lay->pair_q.push_back((*lst)[x]);
-      lay->pair_q.push_back(x + 1 < lst->size() ? (*lst)[x + 1] : -1);
+      pair_q->push_back((*lst)[x]);
+      pair_q->push_back(x + 1 < lst->size() ? (*lst)[x + 1] : -1);
     }
   }
-  lay->n_pairs = static_cast<int>(lay->pair_q.size() / 2);
-  const int P = lay->n_pairs;
-  lay->pair_ptr.assign(1, 0);
-  lay->pair_ent.clear();
+  *n_pairs = static_cast<int>(pair_q->size() / 2);
+  const int P = *n_pairs;
+  pair_ptr->assign(1, 0);
+  pair_ent->clear();
   std::vector<uint32_t> both, only_a, only_b;
   for (int h = 0; h < H; ++h) {
     for (int p = 0; p < P; ++p) {
-      const int qa = lay->pair_q[2 * p], qb = lay->pair_q[2 * p + 1];
-      const int32_t* ra = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qa];
-      const int32_t* ra_end = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qa + 1];
+      const int qa = (*pair_q)[2 * p], qb = (*pair_q)[2 * p + 1];
+      const int32_t* ra = col_idx.data() + row_ptr[static_cast<size_t>(h) * nb + qa];
+      const int32_t* ra_end = col_idx.data() + row_ptr[static_cast<size_t>(h) * nb + qa + 1];
       const int32_t* rb = ra_end;
       const int32_t* rb_end = ra_end;
       if (qb >= 0) {
-        rb = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qb];
-        rb_end = lay->col_idx.data() + lay->row_ptr[static_cast<size_t>(h) * nb + qb + 1];
+        rb = col_idx.data() + row_ptr[static_cast<size_t>(h) * nb + qb];
+        rb_end = col_idx.data() + row_ptr[static_cast<size_t>(h) * nb + qb + 1];
       }
-      // Union entries: the blocks both query blocks attend, then the blocks only one
-      // of them attends, alternating first/second; each group ascending.  The order
-      // is free (one softmax over the union), and this one keeps the two halves of
-      // the tile -- whose warps skip the exponentials of a block their half does not
-      // attend -- doing equal work chunk by chunk.
       both.clear();
       only_a.clear();
       only_b.clear();
@@ -218,22 +231,63 @@ void build_tiles(bsa_layout* lay) {
           ++rb;
         }
       }
-      lay->pair_ent.insert(lay->pair_ent.end(), both.begin(), both.end());
+      pair_ent->insert(pair_ent->end(), both.begin(), both.end());
       for (size_t x = 0; x < std::max(only_a.size(), only_b.size()); ++x) {
-        if (x < only_a.size()) lay->pair_ent.push_back(only_a[x]);
-        if (x < only_b.size()) lay->pair_ent.push_back(only_b[x]);
+        if (x < only_a.size()) pair_ent->push_back(only_a[x]);
+        if (x < only_b.size()) pair_ent->push_back(only_b[x]);
       }
       // A tile whose rows are all empty (possible in a caller's CSR) still runs one
-      // entry so that its output rows get written (O = 0, lse = -inf): key block 0
-      // with no membership bit, which neither half attends.
-      if (both.empty() && only_a.empty() && only_b.empty()) lay->pair_ent.push_back(0u);
-      lay->pair_ptr.push_back(static_cast<int32_t>(lay->pair_ent.size()));
+      // entry so that its output rows get written (zeros): block 0 with no
+      // membership bit, which neither half takes part in.
+      if (both.empty() && only_a.empty() && only_b.empty()) pair_ent->push_back(0u);
+      pair_ptr->push_back(static_cast<int32_t>(pair_ent->size()));
     }
   }
+}
+
+// Work list of a backward kernel: first the chunks of the tiles whose union is
+// longer than kSplitThreshold (kSplitChunk entries each, every one writing a
+// partial record), then the other tiles, longest first.
+void make_bwd_plan(int H, const std::vector<int32_t>& pair_q, int P, const std::vector<int32_t>& pair_ptr,
+                   bsa::BwdPlan* plan) {
+  plan->items.clear();
+  plan->splits.clear();
+  plan->n_records = 0;
+  std::vector<bsa::BwdItem> whole;
+  for (int h = 0; h < H; ++h) {
+    for (int p = 0; p < P; ++p) {
+      const int32_t s = pair_ptr[static_cast<size_t>(h) * P + p];
+      const int32_t U = pair_ptr[static_cast<size_t>(h) * P + p + 1] - s;
+      if (U <= bsa::kSplitThreshold) {
+        whole.push_back(bsa::BwdItem{h, p, s, U, -1, {0, 0, 0}});
+        continue;
+      }
+      const int nch = (U + bsa::kSplitChunk - 1) / bsa::kSplitChunk;
+      const int base = plan->n_records;
+      plan->n_records += nch;
+      plan->splits.push_back(bsa::SplitTile{h, pair_q[2 * p], pair_q[2 * p + 1], base, nch, {0, 0, 0}});
+      for (int c = 0; c < nch; ++c) {
+        const int cs = c * bsa::kSplitChunk;
+        plan->items.push_back(bsa::BwdItem{h, p, s + cs, std::min(bsa::kSplitChunk, U - cs), base + c, {0, 0, 0}});
+      }
+    }
+  }
+  std::stable_sort(whole.begin(), whole.end(),
+                   [](const bsa::BwdItem& a, const bsa::BwdItem& b) { return a.count > b.count; });
+  plan->items.insert(plan->items.end(), whole.begin(), whole.end());
+}
+
+void build_tiles(bsa_layout* lay) {
+  const int nb = lay->nb, H = lay->H;
+  std::vector<uint8_t> is_global(static_cast<size_t>(nb), 0);
+  for (int g : lay->globals) is_global[static_cast<size_t>(g)] = 1;
+  make_tiles(H, nb, lay->row_ptr, lay->col_idx, is_global, &lay->pair_q, &lay->n_pairs, &lay->pair_ptr,
+             &lay->pair_ent);
+  const int P = lay->n_pairs;
   // Work items of one batch element: first the chunks of split tiles (the forward
-  // hands these out first, for the whole batch: they are the longest items, and
-  // the last chunk of each merges the others), then the other tiles, head-major
-  // so that items running at the same time share the head's K/V in L2.
+  // hands these out first, for the whole batch: they are the longest items), then
+  // the other tiles, head-major so that items running at the same time share the
+  // head's K/V in L2.
   lay->items.clear();
   lay->splits.clear();
   lay->n_split = 0;
@@ -262,6 +316,32 @@ void build_tiles(bsa_layout* lay) {
       }
     }
   }
+  // Backward.  dQ runs over the same query tiles.  dK and dV run over key tiles:
+  // the transposed CSR (row (h, j) = the query blocks whose row holds key block j,
+  // ascending) cut into tiles the same way, the key blocks every query block
+  // attends in every head (BigBird's globals) paired with each other.
+  make_bwd_plan(H, lay->pair_q, P, lay->pair_ptr, &lay->dq_plan);
+  std::vector<int32_t> t_ptr(static_cast<size_t>(H) * nb + 1, 0), t_col(lay->col_idx.size());
+  for (int h = 0; h < H; ++h)
+    for (int i = 0; i < nb; ++i)
+      for (int32_t x = lay->row_ptr[static_cast<size_t>(h) * nb + i];
+           x < lay->row_ptr[static_cast<size_t>(h) * nb + i + 1]; ++x)
+        ++t_ptr[static_cast<size_t>(h) * nb + lay->col_idx[static_cast<size_t>(x)] + 1];
+  for (size_t x = 0; x + 1 < t_ptr.size(); ++x) t_ptr[x + 1] += t_ptr[x];
+  std::vector<int32_t> fill(t_ptr.begin(), t_ptr.end() - 1);
+  for (int h = 0; h < H; ++h)
+    for (int i = 0; i < nb; ++i)
+      for (int32_t x = lay->row_ptr[static_cast<size_t>(h) * nb + i];
+           x < lay->row_ptr[static_cast<size_t>(h) * nb + i + 1]; ++x)
+        t_col[static_cast<size_t>(fill[static_cast<size_t>(h) * nb + lay->col_idx[static_cast<size_t>(x)]]++)] = i;
+  std::vector<uint8_t> kdense(static_cast<size_t>(nb), 1);
+  for (int h = 0; h < H; ++h)
+    for (int j = 0; j < nb; ++j)
+      if (t_ptr[static_cast<size_t>(h) * nb + j + 1] - t_ptr[static_cast<size_t>(h) * nb + j] != nb)
+        kdense[static_cast<size_t>(j)] = 0;
+  make_tiles(H, nb, t_ptr, t_col, kdense, &lay->ktiles.pair_q, &lay->ktiles.n_pairs, &lay->ktiles.pair_ptr,
+             &lay->ktiles.pair_ent);
+  make_bwd_plan(H, lay->ktiles.pair_q, lay->ktiles.n_pairs, lay->ktiles.pair_ptr, &lay->dkv_plan);
 }
 
 }  // namespace
@@ -326,7 +406,8 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
       }
     }
     build_tiles(lay);
-    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
+    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX) ||
+        lay->ktiles.pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
       delete lay;
       return BSA_ERR_INVALID_ARG;
     }
@@ -390,7 +471,8 @@ int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const i
       if (dense[static_cast<size_t>(i)]) lay->globals.push_back(i);
     lay->n_global = static_cast<int>(lay->globals.size());
     build_tiles(lay);
-    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
+    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX) ||
+        lay->ktiles.pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
       delete lay;
       return BSA_ERR_INVALID_ARG;
     }
@@ -431,6 +513,23 @@ int bsa_layout_tiles(const bsa_layout* lay, const int32_t** pair_q, int* n_pairs
   if (pair_ptr) *pair_ptr = lay->pair_ptr.data();
   if (pair_ent) *pair_ent = lay->pair_ent.data();
   if (n_ent) *n_ent = static_cast<int64_t>(lay->pair_ent.size());
+  return BSA_OK;
+}
+
+int bsa_layout_key_tiles(const bsa_layout* lay, const int32_t** pair_k, int* n_pairs,
+                         const int32_t** pair_ptr, const uint32_t** pair_ent, int64_t* n_ent) {
+  if (lay == nullptr) return BSA_ERR_INVALID_ARG;
+  if (pair_k) *pair_k = lay->ktiles.pair_q.data();
+  if (n_pairs) *n_pairs = lay->ktiles.n_pairs;
+  if (pair_ptr) *pair_ptr = lay->ktiles.pair_ptr.data();
+  if (pair_ent) *pair_ent = lay->ktiles.pair_ent.data();
+  if (n_ent) *n_ent = static_cast<int64_t>(lay->ktiles.pair_ent.size());
+  return BSA_OK;
+}
+
+int bsa_backward_workspace_bytes(const bsa_layout* lay, int B, size_t* bytes) {
+  if (lay == nullptr || bytes == nullptr || B < 1) return BSA_ERR_INVALID_ARG;
+  *bytes = bsa::plan_bwd_workspace(*lay, B).total;
   return BSA_OK;
 }
 

@@ -48,6 +48,31 @@ struct SplitTile {
 };
 static_assert(sizeof(SplitTile) == 32, "SplitTile must stay 32 bytes");
 
+// One work item of the backward kernels: a whole tile, or one chunk of a split
+// tile (rec >= 0: its partial record index within a batch element).
+struct BwdItem {
+  int32_t h, pair, start, count, rec;
+  int32_t pad[3];
+};
+static_assert(sizeof(BwdItem) == 32, "BwdItem must stay 32 bytes");
+
+// Tiles of 128 rows over a block CSR: pair_q (2 per tile), pair_ptr (H*n_pairs+1),
+// pair_ent (key block | membership << 24).
+struct TileSet {
+  std::vector<int32_t> pair_q;
+  int n_pairs = 0;
+  std::vector<int32_t> pair_ptr;
+  std::vector<uint32_t> pair_ent;
+};
+
+// Work list of a backward kernel over a TileSet: split-tile chunks first, then
+// whole tiles, longest first; the split tiles for the merge.
+struct BwdPlan {
+  std::vector<BwdItem> items;
+  std::vector<SplitTile> splits;
+  int n_records = 0;
+};
+
 constexpr uint32_t kEntColMask = 0x00FFFFFFu;
 constexpr int kEntBitsShift = 24;
 
@@ -68,12 +93,22 @@ struct bsa_layout {
   std::vector<bsa::SplitTile> splits;  // the split tiles of one batch element
   int n_split = 0;                  // split tiles per batch element
   int n_records = 0;                // partial records per batch element
+  // backward: key-major tiles (pairs of key blocks over the union of the query
+  // blocks that attend them) and the work lists of its two kernels
+  bsa::TileSet ktiles;
+  bsa::BwdPlan dq_plan, dkv_plan;
   // device copies (bsa_layout_upload)
   int device = -1;
   int32_t* d_pair_q = nullptr;
   uint32_t* d_pair_ent = nullptr;
   bsa::WorkItem* d_items = nullptr;
   bsa::SplitTile* d_splits = nullptr;
+  int32_t* d_kpair_q = nullptr;
+  uint32_t* d_kpair_ent = nullptr;
+  bsa::BwdItem* d_dq_items = nullptr;
+  bsa::BwdItem* d_dkv_items = nullptr;
+  bsa::SplitTile* d_dq_splits = nullptr;
+  bsa::SplitTile* d_dkv_splits = nullptr;
 };
 
 namespace bsa {
@@ -88,5 +123,14 @@ struct WorkspacePlan {
   size_t total;
 };
 WorkspacePlan plan_workspace(const bsa_layout& lay, int B);
+// Backward workspace for batch size B: key-padding bits, D = rowsum(dO * O) and
+// lse in log2 units per row, and the partial records of split tiles (dQ: 128 x 64
+// floats each; dK and dV: 2 x 128 x 64 floats each).
+struct BwdWorkspacePlan {
+  size_t keybits_off, dsum_off, lse2_off, dq_rec_off, dkv_rec_off, total;
+};
+BwdWorkspacePlan plan_bwd_workspace(const bsa_layout& lay, int B);
+constexpr int kBwdDqRecFloats = kTileRows * kHeadDim;
+constexpr int kBwdDkvRecFloats = 2 * kTileRows * kHeadDim;
 void free_device(bsa_layout* lay);
 }  // namespace bsa

@@ -1,4 +1,4 @@
-// Thin inline-PTX wrappers for the sm_100a features the forward kernel uses:
+// Thin inline-PTX wrappers for the sm_100a features the kernels use:
 // mbarriers, TMA tile loads, tcgen05 MMA / commit / TMEM load-store / alloc.
 // Written from the PTX ISA (tcgen05, cp.async.bulk.tensor, mbarrier sections).
 #pragma once
@@ -74,6 +74,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint3
       " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+// Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from global to shared memory, completing on `bar` (tx bytes).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
 }
 // TMA tile store from shared memory (bulk-group completion).
 __device__ __forceinline__ void tma_store_2d(const void* map, uint32_t src, int x, int y) {

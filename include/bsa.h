@@ -1,7 +1,8 @@
 /*
- * bsa.h -- C ABI of the B200 (sm_100a) BigBird block-sparse attention forward.
+ * bsa.h -- C ABI of the B200 (sm_100a) BigBird block-sparse attention forward
+ * and its gradients (bsa_backward).
  *
- * What is computed (forward pass only), for every batch element b, head h and
+ * What the forward computes, for every batch element b, head h and
  * query token t of query block i = t / 64:
  *
  *     O[b,h,t,:] = softmax_{p in A(h,i)} ( q_t . k_p * scale ) . V[b,h,p,:]
@@ -154,6 +155,24 @@ int bsa_layout_tiles(const bsa_layout* layout, const int32_t** pair_q, int* n_pa
                      const int32_t** pair_ptr, const uint32_t** pair_ent, int64_t* n_ent);
 
 /*
+ * bsa_layout_key_tiles -- host views of the key-major tiles the backward's dK/dV
+ * kernel runs: the transposed layout (row (h, j) = the query blocks whose row
+ * holds key block j, ascending) cut into 128-row tiles exactly as
+ * bsa_layout_tiles describes for query rows.
+ *   pair_k:   2*n_pairs int32, (first, second) key block; second = -1 for a
+ *             single-block tile.  Key blocks that every query block attends in
+ *             every head pair with each other.
+ *   pair_ptr: H*n_pairs+1 int32 offsets into pair_ent, head-major.
+ *   pair_ent: query block | (membership << 24): bit 0 = the query block attends
+ *             the first key block, bit 1 = the second.  Order as in
+ *             bsa_layout_tiles; a tile no query block attends holds one entry
+ *             (block 0, no bits).
+ * Any output may be NULL.
+ */
+int bsa_layout_key_tiles(const bsa_layout* layout, const int32_t** pair_k, int* n_pairs,
+                         const int32_t** pair_ptr, const uint32_t** pair_ent, int64_t* n_ent);
+
+/*
  * bsa_layout_upload -- copies the tile tables and work list to the CURRENT
  * device (cudaMemcpyAsync on `stream`, then a stream synchronize).  Must
  * precede bsa_forward on that device.  Calling it again re-uploads to the
@@ -224,6 +243,47 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
 int bsa_forward_static_ws(const void* q, const void* k, const void* v, int B, int H, int L, int d,
                           const bsa_layout* layout, const uint8_t* key_mask, float scale,
                           void* out, float* lse, void* stream);
+
+/*
+ * bsa_backward_workspace_bytes -- device scratch bytes bsa_backward needs for
+ * batch size B: key-padding bits, two fp32 values per query row (D and lse in
+ * log2 units) and the fp32 partial sums of split tiles.  Unlike the forward's
+ * workspace it needs no clearing: every byte is written before it is read.
+ */
+int bsa_backward_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
+
+/*
+ * bsa_backward -- enqueues the gradients of bsa_forward on `stream`.
+ *
+ * For a loss L with dO = dL/dO, with P the attention weights of the forward
+ * (P = exp(scale q_t . k_p - lse_t) on the attended keys, 0 elsewhere):
+ *     D_t  = sum_c dO[t,c] O[t,c]
+ *     dS   = P (.) (dO V^T - D)                 (the softmax Jacobian)
+ *     dQ   = scale dS K,   dK = scale dS^T Q,   dV = P^T dO
+ * This is the derivative of the forward's masked attention ("Adapt or Perish:
+ * 新手入门指南 – Adaptive Sparse Transformer 核心原理与实战", sparse-attention
+ * formula), the training the pages describe ("BERT 稀疏注意力机制入门指南",
+ * 生产环境部署建议; "BigBird 稀疏注意力机制解析", 避坑指南) needing it.
+ *   q, k, v   device, bf16, [B, H, L, d] contiguous, 16-byte aligned: the
+ *             forward's inputs.
+ *   out, lse  device: the forward's O (bf16 [B, H, L, d]) and lse (fp32
+ *             [B, H, L]) for the same inputs, layout, key_mask and scale.
+ *   dout      device, bf16, [B, H, L, d]: dL/dO.
+ *   key_mask  device uint8 [B, L] (1 = keep) or NULL, as in the forward.
+ *   scale     as in the forward (<= 0 selects 1/sqrt(d)).
+ *   dq, dk, dv device, bf16, [B, H, L, d], written in full (zeros for keys no
+ *             query attends and for query rows that attend no key).
+ *   workspace device, at least bsa_backward_workspace_bytes(layout, B) bytes,
+ *             256-byte aligned; no clearing needed.
+ * d must be 64 (else BSA_ERR_UNSUPPORTED).  Enqueues up to seven kernels (key
+ * bits, D and lse, dQ, dK/dV, and the sums of split tiles for dQ, dK and dV); no
+ * synchronisation, no allocation.  A device-side timeout is reported later by
+ * bsa_sync_status.
+ */
+int bsa_backward(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                 const float* lse, int B, int H, int L, int d, const bsa_layout* layout,
+                 const uint8_t* key_mask, float scale, void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, void* stream);
 
 /*
  * bsa_sync_status -- synchronises `stream`, then returns and clears the

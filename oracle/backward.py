@@ -39,13 +39,14 @@ def attention_backward(q, k, v, dout, layout: dict, key_mask=None, scale=None,
                        with_magnitude: bool = False):
     """dq, dk, dv [B,H,L,d] in fp64 for the loss gradient ``dout`` = dL/dO.
 
-    With ``with_magnitude`` also returns, per output element, the sum of the
-    absolute values of the terms it is summed from (same shapes):
-      |dq|-terms  scale * (P (.) (|dP| + |D|)) |K|
-      |dk|-terms  scale * (P (.) (|dP| + |D|))^T |Q|
+    With ``with_magnitude`` also returns, per output element, a sum of absolute
+    values that bounds the terms it is summed from (same shapes):
+      |dq|-terms  scale * (P (.) (|dP| + Dabs)) |K|
+      |dk|-terms  scale * (P (.) (|dP| + Dabs))^T |Q|
       |dv|-terms  P^T |dO|
-    These bound the effect of rounding P, dS or D by a relative amount on the
-    result, which is what a tolerance needs.
+    with Dabs = rowsum(|dO| (.) |O|) >= |D|.  A relative error e in P, in dS or in
+    the factors of D moves the result by at most e times this sum, which is what
+    a tolerance needs.
     """
     q, k, v, do = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
     B, H, L, d = q.shape
@@ -78,7 +79,8 @@ def attention_backward(q, k, v, dout, layout: dict, key_mask=None, scale=None,
                 dk[b, h] += (ds.T @ q[b, h, rows]) * scale
                 dv[b, h] += p.T @ do[b, h, rows]
                 if with_magnitude:
-                    w = p * (np.abs(dp) + np.abs(D))
+                    dabs = (np.abs(do[b, h, rows]) * np.abs(p @ vb)).sum(axis=-1, keepdims=True)
+                    w = p * (np.abs(dp) + dabs)
                     mq[b, h, rows] = (w @ np.abs(kb)) * scale
                     mk[b, h] += (w.T @ np.abs(q[b, h, rows])) * scale
                     mv[b, h] += p.T @ np.abs(do[b, h, rows])

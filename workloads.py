@@ -103,6 +103,13 @@ def make_qkv(w: Workload, data_seed: int = 0):
             v.to(torch.bfloat16).contiguous())
 
 
+def make_grad(w: Workload, seed: int = 1) -> torch.Tensor:
+    """A loss gradient dL/dO for the backward: fp32 randn(B, H, L, d) from
+    ``torch.Generator().manual_seed(seed)``, rounded to bf16."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn((w.B, w.H, w.L, w.d), generator=g, dtype=torch.float32).to(torch.bfloat16).contiguous()
+
+
 def make_key_mask(w: Workload) -> Optional[torch.Tensor]:
     """uint8 [B, L] key-padding mask (1 = keep), or None when the shape has none."""
     if w.key_pad_tail <= 0:
