@@ -90,6 +90,11 @@ def _dead_from(w):
     return (w.L - w.key_pad_tail + 63) // 64
 
 
+METRIC_BWD = ("block-sparse attn bwd TFLOP/s (non-zero blocks, five 64x64x64 products each) "
+              "and % of B200 bf16 peak")
+FLOP_PER_BLOCK_BWD = 5 * 2 * 64 * 64 * 64  # S, dP, dV, dK, dQ: 2.5x the forward's
+
+
 def _has_split_rows(lay) -> bool:
     """Whether bsa_forward launches its split-row merge for this layout."""
     from block_sparse_attention_bigbird_b200 import bsa
@@ -270,18 +275,25 @@ def run_reference(args, w, world, rank):
     km = workloads.make_key_mask(w)
     nb = w.nb
     n_blocks = max(1, min(nb, int(os.environ.get("BSA_REF_BLOCKS", "8"))))
+    backward = args.pass_ == "backward"
+    if backward:
+        do = workloads.make_grad(w, seed=100)
+        sample_fn = lambda h: _oracle_bwd_sample(w, lay, q, k, v, do, km, h, n_blocks)  # noqa: E731
+    else:
+        sample_fn = lambda h: _oracle_sample(w, lay, q, k, v, km, h, n_blocks)  # noqa: E731
     for s in range(args.warmup):
-        _oracle_sample(w, lay, q, k, v, km, s % w.H, n_blocks)
+        sample_fn(s % w.H)
     tot_t = tot_f = 0.0
     for s in range(args.steps):
-        dt, fl = _oracle_sample(w, lay, q, k, v, km, s % w.H, n_blocks)
+        dt, fl = sample_fn(s % w.H)
         tot_t += dt
         tot_f += fl
     val = tot_f / tot_t / 1e12
     cores = _oracle_cores()
-    sample = (f"per step: query blocks 0..{n_blocks - 1} of batch 0, head step%H "
-              f"({n_blocks * 64} of {w.L} query rows), fp64 masked-dense")
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+    sample = (f"per step: {'gradients from ' if backward else ''}query blocks 0..{n_blocks - 1} of batch 0, "
+              f"head step%H ({n_blocks * 64} of {w.L} query rows), fp64 masked-dense")
+    line = {"impl": "reference", "metric": METRIC_BWD if backward else METRIC, "value": val, "unit": UNIT,
+            "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": _config(w, None, world),
@@ -451,6 +463,155 @@ def run_ours(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+def _bwd_launches(lay, masked: bool) -> int:
+    """Kernels one bsa_backward call enqueues: key bits (with a mask), D and lse,
+    dQ, dK/dV, and the split-tile sums of dQ and of dK and dV when there are any."""
+    from block_sparse_attention_bigbird_b200 import bsa
+    _, qp, _ = bsa.bsa_layout_tiles(lay)
+    _, kp, _ = bsa.bsa_layout_key_tiles(lay)
+    n = 3 + (1 if masked else 0)
+    n += 1 if np.any(np.diff(qp) > bsa.SPLIT_THRESHOLD) else 0
+    n += 2 if np.any(np.diff(kp) > bsa.SPLIT_THRESHOLD) else 0
+    return n
+
+
+def _oracle_bwd_sample(w, lay, q, k, v, do, km, h, n_blocks):
+    """Oracle gradients from query blocks [0, n_blocks) of (b=0, head h); (seconds, flop)."""
+    from oracle import backward as OB
+    view = _head_view(lay, h)
+    rp, ci = view["row_ptr"], view["col_idx"]
+    nnz = int(rp[n_blocks])
+    dead = _dead_from(w)
+    if dead is not None:
+        nnz -= int(np.count_nonzero(ci[:rp[n_blocks]] >= dead))
+    sl = slice(h, h + 1)
+    kmask = None if km is None else km[0:1]
+    t0 = time.perf_counter()
+    OB.attention_backward(q[0:1, sl], k[0:1, sl], v[0:1, sl], do[0:1, sl], view, key_mask=kmask,
+                          query_blocks=range(n_blocks))
+    return time.perf_counter() - t0, nnz * FLOP_PER_BLOCK_BWD
+
+
+def run_backward(args, w, world, rank, local):
+    """Backward pass: one bsa_backward call per step on inputs resident in HBM."""
+    from block_sparse_attention_bigbird_b200 import bsa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    q, k, v = workloads.make_qkv(w, data_seed=rank)
+    do = workloads.make_grad(w, seed=100 + rank)
+    km = workloads.make_key_mask(w)
+    lay = bsa.bsa_layout_build(w.H, w.L, w.block, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(lay)
+    row_ptr, col_idx = bsa.bsa_layout_csr(lay)
+    nnz_eff = _nnz_eff(w, row_ptr, col_idx)
+    flop_step = nnz_eff * FLOP_PER_BLOCK_BWD
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    kmd = km.to(dev) if km is not None else None
+    out, lse = bsa.bsa_forward(qd, kd, vd, lay, key_mask=kmd, stream=stream)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(bsa.bsa_backward_workspace_bytes(lay, w.B), dtype=torch.uint8, device=dev)
+    launches_per_step = _bwd_launches(lay, km is not None)
+
+    def step(qs=qd, ks=kd, vs=vd, outs=out, dos=dod, lses=lse, gq=dq, gk=dk, gv=dv):
+        bsa.bsa_backward(qs, ks, vs, outs, dos, lses, lay, key_mask=kmd, dq=gq, dk=gk, dv=gv, workspace=ws,
+                         stream=stream)
+
+    sampler = ClockSampler(local).start() if rank == 0 else None
+    for _ in range(max(3, args.warmup)):
+        step()
+    _barrier(world)
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error during warm-up")
+    t_settle = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    per = max(e0.elapsed_time(e1), 1e-3)
+    for _ in range(int(min(2000, 1500.0 / per))):
+        step()
+    _barrier(world)
+    t_timed0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    _barrier(world)
+    t_timed1 = time.time()
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error in the timed region")
+    total_ms = sharding.max_over_ranks(start.elapsed_time(end), world)
+    clocks = sampler.summary(t_settle, t_timed1, t_timed0) if sampler else None
+    if sampler:
+        sampler.stop()
+
+    # end to end through the public API, one step after another on one stream:
+    # the step's six inputs from pinned host memory, the backward, the three
+    # gradients back to pinned host memory
+    e2e_steps = max(3, min(args.steps, 10))
+    hosts = [t.detach().to("cpu").pin_memory() for t in (qd, kd, vd, out, dod, lse)]
+    outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in hosts) + (km.numel() if km is not None else 0)
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    devs = [torch.empty_like(t) for t in (qd, kd, vd, out, dod, lse)]
+    _barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        for dst, src in zip(devs, hosts):
+            dst.copy_(src, non_blocking=True)
+        step(*devs)
+        for dst, src in zip(outs_h, (dq, dk, dv)):
+            dst.copy_(src, non_blocking=True)
+    b.record(stream)
+    _barrier(world)
+    e2e_ms = sharding.max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error in the end-to-end run")
+
+    ms_per_step = total_ms / args.steps
+    value = world * flop_step / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = _peaks()
+    achieved = flop_step / (ms_per_step * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        lay_o = _oracle_heads(w)
+        budget = float(os.environ.get("BSA_CPU_BUDGET_S", "12"))
+        tot_t = tot_f = 0.0
+        n_blocks, h = min(w.nb, 8), 0
+        while tot_t < budget and h < w.H:
+            dt, fl = _oracle_bwd_sample(w, lay_o, q, k, v, do, km, h, n_blocks)
+            tot_t, tot_f, h = tot_t + dt, tot_f + fl, h + 1
+        cpu = {"value": tot_f / tot_t / 1e12, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
+               "sample": f"gradients from query blocks 0..{n_blocks - 1} of batch 0, heads 0..{h - 1} "
+                         f"({tot_t:.1f} s of fp64 masked-dense)"}
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC_BWD, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded randn, see workloads.py)",
+        "config": dict(_config(w, nnz_eff, world), **{"pass": "backward"}),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "the whole bsa_backward step (prep, dQ, dK/dV and split-tile sums)",
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "e2e": {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "pipelining": "none: copies in, backward, copies out on one stream"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def _cpu_baseline(w):
     lay = _oracle_heads(w)
     q, k, v = workloads.make_qkv(w, 0)
@@ -477,6 +638,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
+                    help="forward (the default benchmark) or the backward pass")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -489,7 +652,7 @@ def main():
         return
     world, rank, local = _dist_setup(args)
     try:
-        run_ours(args, w, world, rank, local)
+        (run_backward if args.pass_ == "backward" else run_ours)(args, w, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist

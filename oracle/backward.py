@@ -36,8 +36,12 @@ from .attention import _as_f64, token_mask_row
 
 
 def attention_backward(q, k, v, dout, layout: dict, key_mask=None, scale=None,
-                       with_magnitude: bool = False):
+                       with_magnitude: bool = False, query_blocks=None):
     """dq, dk, dv [B,H,L,d] in fp64 for the loss gradient ``dout`` = dL/dO.
+
+    ``query_blocks`` optionally restricts the sums to those query blocks (dq of
+    the other rows stays zero, dk and dv hold only their contributions); the
+    arithmetic is unchanged.
 
     With ``with_magnitude`` also returns, per output element, a sum of absolute
     values that bounds the terms it is summed from (same shapes):
@@ -61,7 +65,7 @@ def attention_backward(q, k, v, dout, layout: dict, key_mask=None, scale=None,
     for b in range(B):
         for h in range(H):
             kb, vb = k[b, h], v[b, h]
-            for i in range(nb):
+            for i in (range(nb) if query_blocks is None else query_blocks):
                 rows = slice(i * block, (i + 1) * block)
                 allowed = token_mask_row(layout, h, i, L)
                 if km is not None:
