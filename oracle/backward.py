@@ -91,3 +91,58 @@ def attention_backward(q, k, v, dout, layout: dict, key_mask=None, scale=None,
     if with_magnitude:
         return dq, dk, dv, (mq, mk, mv)
     return dq, dk, dv
+
+
+def attention_backward_rows(q, k, v, dout, layout: dict, b: int, h: int, query_tokens=(), key_tokens=(),
+                            key_mask=None, scale=None):
+    """Selected rows of the gradients of one (b, h), in fp64, with their magnitudes.
+
+    Returns (dq [nq, d], dk [nk, d], dv [nk, d], (mq, mk, mv)) for the query
+    tokens ``query_tokens`` and the key tokens ``key_tokens``: the same
+    definition as ``attention_backward``, evaluated only on the query rows that
+    the requested outputs depend on (for a key p, every query row whose block
+    attends p's block), block by block over all L keys as in the masked-dense
+    form.
+    """
+    qb, kb, vb, dob = (_as_f64(x[b, h]) for x in (q, k, v, dout))
+    L, d = kb.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    block, nb = layout["block"], layout["nb"]
+    km = None if key_mask is None else _as_f64(key_mask[b]) != 0
+    key_tokens = np.asarray([int(p) for p in key_tokens], dtype=np.int64)
+    query_tokens = [int(t) for t in query_tokens]
+    kblocks = sorted({int(p) // block for p in key_tokens})
+    dq = np.zeros((len(query_tokens), d))
+    dk = np.zeros((len(key_tokens), d))
+    dv = np.zeros((len(key_tokens), d))
+    mq, mk, mv = np.zeros_like(dq), np.zeros_like(dk), np.zeros_like(dv)
+    for i in range(nb):
+        allowed = token_mask_row(layout, h, i, L)
+        whole = any(allowed[j * block] for j in kblocks)  # the block's rows reach a requested key
+        mine = [(n, t) for n, t in enumerate(query_tokens) if t // block == i]
+        if not whole and not mine:
+            continue
+        if km is not None:
+            allowed = allowed & km
+        rows = np.arange(i * block, (i + 1) * block) if whole else np.asarray([t for _, t in mine])
+        s = np.where(allowed, (qb[rows] @ kb.T) * scale, -np.inf)
+        mx = s.max(axis=-1, keepdims=True)
+        empty = ~np.isfinite(mx)
+        e = np.exp(s - np.where(empty, 0.0, mx))
+        p = np.where(empty, 0.0, e / np.where(empty, 1.0, e.sum(axis=-1, keepdims=True)))
+        dp = dob[rows] @ vb.T
+        D = (p * dp).sum(axis=-1, keepdims=True)
+        ds = p * (dp - D)
+        dabs = (np.abs(dob[rows]) * np.abs(p @ vb)).sum(axis=-1, keepdims=True)
+        w = p * (np.abs(dp) + dabs)
+        for n, t in mine:
+            r = int(np.nonzero(rows == t)[0][0])
+            dq[n] = (ds[r] @ kb) * scale
+            mq[n] = (w[r] @ np.abs(kb)) * scale
+        if whole and len(key_tokens):
+            dk += (ds[:, key_tokens].T @ qb[rows]) * scale
+            mk += (w[:, key_tokens].T @ np.abs(qb[rows])) * scale
+            dv += p[:, key_tokens].T @ dob[rows]
+            mv += p[:, key_tokens].T @ np.abs(dob[rows])
+    return dq, dk, dv, (mq, mk, mv)

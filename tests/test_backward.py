@@ -110,7 +110,9 @@ def test_backward_workspace_grows_with_batch():
 
 # ------------------------------------------------------------------ GPU parity
 
-def _gpu_grads(w, lay, key_mask, scale, data_seed=0):
+def _gpu_grads(w, lay, key_mask, scale, data_seed=0, to_numpy=True):
+    """Forward then backward on the GPU with the inputs bench.py's rank 0 uses
+    (data seed 0, gradient seed 100)."""
     q, k, v = workloads.make_qkv(w, data_seed)
     do = workloads.make_grad(w, seed=data_seed + 100)
     dev = torch.device("cuda")
@@ -119,7 +121,8 @@ def _gpu_grads(w, lay, key_mask, scale, data_seed=0):
     out, lse = bsa.bsa_forward(qd, kd, vd, lay, key_mask=kmd, scale=scale)
     dq, dk, dv = bsa.bsa_backward(qd, kd, vd, out, dod, lse, lay, key_mask=kmd, scale=scale)
     assert bsa.bsa_sync_status() == 0
-    return (q, k, v, do), [t.float().cpu().numpy() for t in (dq, dk, dv)]
+    grads = (dq, dk, dv)
+    return (q, k, v, do), ([t.float().cpu().numpy() for t in grads] if to_numpy else grads)
 
 
 def _check_grads(gpu, ref, mags):
@@ -186,3 +189,40 @@ def test_backward_repeatable_and_workspace_reusable():
     _, g2 = _gpu_grads(w, lay, None, None)
     for a, b in zip(g1, g2):
         assert np.array_equal(a, b)
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+@pytest.mark.parametrize("name", ["c3", "c5"])
+def test_backward_full_size_sampled(name):
+    """Full benchmark shapes in the launch configuration ``bench.py --pass backward``
+    times, checked on sampled rows: query rows (first, last, global, random) and key
+    rows (random non-global ones; for long_b4h12l16384 also the global key blocks'
+    first and last keys, which every query block attends; for genomic_b1h8l131072
+    padded keys, whose gradients are zero)."""
+    w = workloads.get(name)
+    lay = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(lay)
+    km = workloads.make_key_mask(w)
+    (q, k, v, do), (dq, dk, dv) = _gpu_grads(w, lay, km, None, to_numpy=False)
+    ref_lay = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    g = ref_lay["globals"]
+    rng = np.random.default_rng(7)
+    non_global = np.setdiff1d(np.arange(w.nb), g)
+    if w.key_pad_tail:
+        non_global = non_global[non_global * 64 + 63 < w.L - w.key_pad_tail]
+    for n, (b, h) in enumerate([(0, 0), (w.B - 1, w.H - 1)]):
+        qt = {0, 63, 64, w.L - 1, g[0] * 64 + 5, g[-1] * 64 + 60}
+        qt.update(int(x) * 64 + int(rng.integers(0, 64)) for x in rng.choice(non_global, 4, replace=False))
+        kt = {int(x) * 64 + int(rng.integers(0, 64)) for x in rng.choice(non_global, 5, replace=False)}
+        if name == "c3" and n == 0:
+            kt.update({g[0] * 64, g[-1] * 64 + 63})
+        if w.key_pad_tail:
+            kt.update({w.L - 1, w.L - w.key_pad_tail})
+        qt, kt = sorted(qt), sorted(kt)
+        rq, rk, rv, (mq, mk, mv) = OB.attention_backward_rows(q, k, v, do, ref_lay, b, h, qt, kt, key_mask=km)
+        got = [t[b, h, idx].float().cpu().numpy() for t, idx in ((dq, qt), (dk, kt), (dv, kt))]
+        _check_grads(got, (rq, rk, rv), (mq, mk, mv))
+        if w.key_pad_tail:
+            padded = [x for x, p in enumerate(kt) if p >= w.L - w.key_pad_tail]
+            assert np.all(got[1][padded] == 0) and np.all(got[2][padded] == 0)

@@ -143,3 +143,21 @@ def test_magnitudes_bound_the_results():
     _, _, dv2 = OB.attention_backward(q, k, v, do, lay)
     assert np.array_equal(dv, dv2)
     assert math.isfinite(float(mq.max()))
+
+
+def test_rows_api_matches_full():
+    B, H, L, d = 2, 2, 64 * 7, 8
+    lay = OL.build_layout(H, L, 64, 1, 1, 2, 4)
+    q, k, v, do = (_rand((B, H, L, d), s) for s in (41, 42, 43, 44))
+    km = np.ones((B, L), dtype=np.uint8)
+    km[1, -50:] = 0
+    dq, dk, dv, (mq, mk, mv) = OB.attention_backward(q, k, v, do, lay, key_mask=km, with_magnitude=True)
+    qt, kt = [0, 5, 63, 64, 200, 447], [1, 64, 130, 300, 420, 446]
+    for b in range(B):
+        for h in range(H):
+            rq, rk, rv, (sq, sk, sv) = OB.attention_backward_rows(q, k, v, do, lay, b, h, qt, kt, key_mask=km)
+            assert np.abs(rq - dq[b, h, qt]).max() < 1e-12
+            assert np.abs(rk - dk[b, h, kt]).max() < 1e-12
+            assert np.abs(rv - dv[b, h, kt]).max() < 1e-12
+            for a, m in ((sq, mq[b, h, qt]), (sk, mk[b, h, kt]), (sv, mv[b, h, kt])):
+                assert np.abs(a - m).max() < 1e-12
