@@ -9,25 +9,35 @@
 //   D  = rowsum(dO * O)                               bsa_bwd_prep_kernel
 //   P  = 2^(S * scale * log2 e - lse * log2 e),  S = Q K^T on the attended keys
 //   dP = dO V^T,  dS = P * (dP - D)
-//   dQ = scale * dS K                                 bsa_bwd_dq_kernel
-//   dK = scale * dS^T Q,  dV = P^T dO                 bsa_bwd_dkv_kernel
+//   dQ = scale * dS K                                 bsa_bwd_kernel<false>
+//   dK = scale * dS^T Q,  dV = P^T dO                 bsa_bwd_kernel<true>
 // P is rebuilt from lse, so no softmax statistics are recomputed.
 //
-// Both main kernels run one 128-row tile per CTA (128 threads; thread r owns tile
-// row r = TMEM lane r) and walk the tile's entries one 64-block at a time:
-//   dQ kernel   tile = two query blocks (the forward's tiles), entries = key blocks.
-//               S = Q K_j^T and dP = dO V_j^T (tcgen05, A and B from shared
-//               memory), dS (bf16) written over the S columns, dQ += dS K_j
-//               (A = dS from TMEM).
-//   dKV kernel  tile = two key blocks (tiles of the transposed layout), entries =
-//               the query blocks that attend them.  S^T = K Q_i^T, dP^T = V dO_i^T,
-//               P^T and dS^T (bf16) over their columns, dV += P^T dO_i and
-//               dK += dS^T Q_i (A from TMEM).
-// One thread issues the TMA loads and the MMAs; the next entry's blocks load
-// while the current one is processed.  Tiles with long unions are cut into chunks
-// whose partial sums (fp32) bsa_bwd_merge_kernel adds up.  Every wait is bounded;
-// on expiry the CTA records BSA_ERR_DEVICE_TIMEOUT, lets its copies and MMAs
-// finish, frees TMEM and returns.
+// bsa_bwd_kernel runs persistent CTAs (one per SM, 352 threads) over a list of
+// 128-row tiles, each CTA taking items blockIdx.x, blockIdx.x + gridDim.x, ...
+// of a list sorted longest first.  A tile walks its entries one 64-block at a time:
+//   dQ   tile = two query blocks (the forward's tiles), entries = key blocks j.
+//        S = Q K_j^T, dP = dO V_j^T; dS (bf16) over S; dQ += dS K_j.
+//   dKV  tile = two key blocks (tiles of the transposed layout), entries = the
+//        query blocks i attending them.  S^T = K Q_i^T, dP^T = V dO_i^T; P^T and
+//        dS^T (bf16) over them; dV += P^T dO_i, dK += dS^T Q_i.
+// Roles:
+//   warps 0-7  compute: warp w owns TMEM lanes 32 (w % 4) .. + 31 (tile rows) and
+//              score columns 32 (w / 4) .. + 31; it writes its 32 bf16 results
+//              packed into the first 16 of those columns (columns it has read).
+//              They also run each tile's epilogue, one entry into the next tile.
+//   warp 8     TMA producer: the tile's two resident operands (2 stages, so the
+//              next tile loads during this one) and each entry's two blocks (and,
+//              for dKV, the entry's 64 values of lse * log2 e and D) into a
+//              4-stage ring.
+//   warp 9     score issuer: S and dP of entry g into TMEM score stage g % 2 --
+//              one entry ahead of the compute warps.  Allocates TMEM.
+//   warp 10    accumulate issuer: once dS of entry g is written, the accumulating
+//              MMAs of entry g into TMEM accumulator stage (tile % 2), so the
+//              epilogue of a tile overlaps the next one.
+// Tiles with long unions are cut into chunks whose partial sums (fp32)
+// bsa_bwd_merge_kernel adds up.  Every wait is bounded; on expiry the CTA records
+// BSA_ERR_DEVICE_TIMEOUT, lets its copies and MMAs finish, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -44,41 +54,43 @@
 namespace bsa {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr uint32_t kBlkBytes = 64 * 128;  // one 64 x 64 bf16 block
-constexpr uint32_t kTmemCols = 256;
-// TMEM columns: two 64-column score buffers, two 64-column accumulators
-constexpr uint32_t kTmemA = 0;    // S (dQ) or S^T (dKV); bf16 dS / P^T over its first 32
-constexpr uint32_t kTmemB = 64;   // dP (dQ) or dP^T (dKV); bf16 dS^T over its first 32 (dKV)
-constexpr uint32_t kTmemC = 128;  // dQ accumulator (dQ) or dV (dKV)
-constexpr uint32_t kTmemD = 192;  // dK accumulator (dKV)
-
-// shared memory (offsets from the 1024-aligned base).  The tile's own two 64-row
-// blocks of two operands (Q and dO, or K and V) stay resident; the entry's two
-// blocks (K_j and V_j, or Q_i and dO_i) cycle through two stages.
-constexpr uint32_t kSmemTileA = 0;                       // 2 blocks
-constexpr uint32_t kSmemTileB = kSmemTileA + 2 * kBlkBytes;  // 2 blocks
-constexpr uint32_t kSmemEntA = kSmemTileB + 2 * kBlkBytes;   // 2 stages
-constexpr uint32_t kSmemEntB = kSmemEntA + 2 * kBlkBytes;    // 2 stages
-constexpr uint32_t kSmemVec = kSmemEntB + 2 * kBlkBytes;     // dKV: lse2 and D of the entry, 2 stages
+constexpr int kComputeWarps = 8;
+constexpr int kComputeThreads = 32 * kComputeWarps;
+constexpr int kProducerWarp = 8;
+constexpr int kScoreWarp = 9;
+constexpr int kAccWarp = 10;
+constexpr int kThreads = 352;
+constexpr int kEStages = 4;                   // entry ring
+constexpr uint32_t kBlkBytes = 64 * 128;      // one 64 x 64 bf16 block
+constexpr uint32_t kOpBytes = 2 * kBlkBytes;  // a 128-row tile operand
 constexpr uint32_t kVecBytes = 64 * 4;
-constexpr uint32_t kSmemBar = kSmemVec + 4 * kVecBytes;
+constexpr uint32_t kTmemCols = 512;
+// TMEM: score stage s at 128 s (S or S^T at +0, dP or dP^T at +64); accumulator
+// stage a at 256 + kAccCols a (dQ; or dV at +0 and dK at +64)
+constexpr uint32_t kTmemScore = 0;
+constexpr uint32_t kTmemAcc = 256;
+
+// shared memory (offsets from the 1024-aligned base)
+constexpr uint32_t kSmemTile = 0;                                // [2 stages][operand A | operand B]
+constexpr uint32_t kSmemEnt = kSmemTile + 2 * 2 * kOpBytes;      // [4 stages][block A | block B]
+constexpr uint32_t kSmemVec = kSmemEnt + kEStages * 2 * kBlkBytes;  // [4 stages][lse2 | D] (dKV)
+constexpr uint32_t kSmemBar = kSmemVec + kEStages * 2 * kVecBytes;
 enum : int {
-  kBarTile = 0,      // the tile's resident blocks landed
-  kBarEnt = 1,       // [2 stages] the entry's blocks landed
-  kBarSdp = 3,       // MMA commit: S and dP (or S^T and dP^T) are in TMEM
-  kBarDs = 4,        // 128 arrivals: dS (and P^T) written to TMEM
-  kBarAcc = 5,       // MMA commit: the accumulating MMAs of the entry are done
-  kBarFinal = 6,     // MMA commit of an aborting CTA
-  kNumBars = 7
+  kBarTileFull = 0,                      // [2] the tile's operands landed
+  kBarTileEmpty = 2,                     // [2] the tile's last score MMAs are done
+  kBarEntFull = 4,                       // [4] the entry's blocks (and vectors) landed
+  kBarEntEmpty = kBarEntFull + kEStages,      // [4] the entry's accumulating MMAs are done
+  kBarScoreFull = kBarEntEmpty + kEStages,    // [2] S and dP of the entry are in TMEM
+  kBarScoreFree = kBarScoreFull + 2,          // [2] the entry's accumulating MMAs read its dS
+  kBarDsFull = kBarScoreFree + 2,             // [2] 256 arrivals: dS (and P^T) written
+  kBarAccFull = kBarDsFull + 2,               // [2] the tile's last accumulating MMAs are done
+  kBarAccEmpty = kBarAccFull + 2,             // [2] 256 arrivals: the epilogue read the accumulators
+  kBarFinal = kBarAccEmpty + 2,               // [2] the issuers' last commits
+  kNumBars = kBarFinal + 2
 };
 constexpr uint32_t kSmemMisc = kSmemBar + 8 * kNumBars;  // u32 TMEM base, int abort flag
-constexpr uint32_t kSmemUsed = kSmemMisc + 16;
-// Requested dynamic shared memory: the used part plus alignment slack, rounded up
-// so that at most two CTAs share an SM -- two fill its 512 TMEM columns.
-constexpr uint32_t kSmemAlloc = 96 * 1024;
-static_assert(kSmemUsed + 1024 <= kSmemAlloc, "shared memory budget");
-static_assert(3 * (kSmemAlloc + 1024) > 228 * 1024, "at most two CTAs per SM");
+constexpr uint32_t kSmemAlloc = kSmemMisc + 16 + 1024;   // + slack for 1024-byte alignment
+static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
 
 struct BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;
@@ -92,7 +104,7 @@ struct BwdParams {
   const uint32_t* pair_ent;  // entries: block | membership << 24
   const unsigned long long* keybits;  // [B, nb] or null
   float* records;  // partial sums of split tiles, per batch element n_records of them
-  int B, H, L, nb, n_records;
+  int B, H, L, nb, n_items, n_records;
   float scale, scale_log2;
   unsigned long long timeout_ns;
 };
@@ -100,93 +112,62 @@ struct BwdParams {
 constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, 64, false);  // B K-major
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 64, true);   // B MN-major
 
-// Issues A (128 rows, K-major, at smem a) times B^T (64 rows, K-major, at smem b)
-// into TMEM column d: head dim 64 = 4 steps of K = 16, +32 bytes each.
+// A (128 rows, K-major, at smem a) times B^T (64 rows, K-major, at smem b) into
+// TMEM column d: head dim 64 = 4 steps of K = 16, +32 bytes each.
 __device__ __forceinline__ void mma_rows_x_rows(uint32_t d, uint32_t a, uint32_t b) {
   const uint64_t da = ptx::smem_desc_sw128(a, 16), db = ptx::smem_desc_sw128(b, 16);
 #pragma unroll
   for (uint32_t kk = 0; kk < 4; ++kk) ptx::mma_ss(d, da + 2 * kk, db + 2 * kk, kIdescQK, kk > 0 ? 1u : 0u);
 }
 
-// Issues D (+)= A (128 x 64, bf16 in TMEM column a) times B (a 64 x 64 row-major
-// block at smem b, read MN-major): 4 steps of K = 16 rows of B, +2048 bytes each.
+// D (+)= A times B: A is 128 x 64 bf16 in TMEM starting at column a, packed two
+// per column, keys 0-31 in columns a .. a + 15 and keys 32-63 in a + 32 .. a + 47
+// (each compute warp packs its 32 columns into the first half of them); B is a
+// 64 x 64 row-major block at smem b, read MN-major, 16 rows (2048 bytes) per step.
 __device__ __forceinline__ void mma_tmem_x_block(uint32_t d, uint32_t a, uint32_t b, bool accumulate) {
   const uint64_t db = ptx::smem_desc_sw128(b, 0);
 #pragma unroll
   for (uint32_t kk = 0; kk < 4; ++kk)
-    ptx::mma_ts(d, a + 8u * kk, db + kk * (2048u >> 4), kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+    ptx::mma_ts(d, a + 8u * kk + (kk >= 2 ? 16u : 0u), db + kk * (2048u >> 4), kIdescPV,
+                (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// Bookkeeping of the issuing thread, for draining after an abort.
-struct IssueState {
-  uint32_t ent_issued = 0, ent_waited = 0;  // entry loads
-  bool tile_issued = false, tile_waited = false;
-  bool mma_issued = false;
+struct ItemRef {
+  BwdItem w;
+  int b, ta, tb, row0;
 };
 
-// After an abort: wait (bounded) for this thread's copies and MMAs so that nothing
-// lands in shared memory or TMEM after the CTA has left.
-__device__ void drain(const IssueState& is, uint32_t bars, volatile int* abort_flag, uint64_t timeout_ns) {
-  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  if (is.tile_issued && !is.tile_waited) wait_force(bar(kBarTile), 0, abort_flag, timeout_ns);
-  for (uint32_t x = is.ent_waited; x < is.ent_issued; ++x)
-    wait_force(bar(kBarEnt + static_cast<int>(x & 1u)), (x >> 1) & 1u, abort_flag, timeout_ns);
-  if (is.mma_issued) {
-    ptx::mma_commit(bar(kBarFinal));
-    wait_force(bar(kBarFinal), 0, abort_flag, timeout_ns);
-  }
+__device__ __forceinline__ ItemRef item_at(const BwdParams& p, int it) {
+  ItemRef r;
+  const int i = it / p.B;
+  r.b = it - i * p.B;
+  r.w = p.items[i];
+  r.ta = p.pair[2 * r.w.pair];
+  r.tb = p.pair[2 * r.w.pair + 1];
+  r.row0 = (r.b * p.H + r.w.h) * p.L;
+  return r;
 }
 
-// Common prologue: barriers, TMEM.  Returns the TMEM base.
-__device__ __forceinline__ uint32_t cta_setup(uint8_t* smem, uint32_t base) {
-  const uint32_t bars = base + kSmemBar;
-  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kSmemMisc);
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i)
-      ptx::mbar_init(bars + 8u * static_cast<uint32_t>(i), i == kBarDs ? static_cast<uint32_t>(kThreads) : 1u);
-    misc[1] = 0;
-    ptx::fence_barrier_init();
-  }
-  if ((threadIdx.x >> 5) == 0) {
-    ptx::tmem_alloc(ptx::smem_addr(const_cast<uint32_t*>(&misc[0])), kTmemCols);
-    ptx::tmem_relinquish();
-  }
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  return misc[0];
-}
-
-__device__ __forceinline__ void cta_teardown(uint32_t tmem) {
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  if ((threadIdx.x >> 5) == 0) ptx::tmem_dealloc(tmem, kTmemCols);
-}
-
-// 64 fp32 values of this thread's row from TMEM column `col` (lane offset included).
-__device__ __forceinline__ void load_row64(uint32_t taddr, float (&v)[64]) {
-  uint32_t raw[2][32];
-  ptx::tmem_ld32(taddr, raw[0]);
-  ptx::tmem_ld32(taddr + 32u, raw[1]);
+// 32 fp32 values of this thread's lane from TMEM column taddr.
+__device__ __forceinline__ void load32(uint32_t taddr, float (&v)[32]) {
+  uint32_t raw[32];
+  ptx::tmem_ld32(taddr, raw);
   ptx::tmem_wait_ld();
-  ptx::reg_fence(raw[0]);
-  ptx::reg_fence(raw[1]);
+  ptx::reg_fence(raw);
 #pragma unroll
-  for (int c = 0; c < 64; ++c) v[c] = __uint_as_float(raw[c >> 5][c & 31]);
+  for (int c = 0; c < 32; ++c) v[c] = __uint_as_float(raw[c]);
 }
 
-// Stores a row of 64 values times f: bf16 to `out` (a whole tile) or fp32 to `rec`
-// (a chunk of a split tile).
-__device__ __forceinline__ void store_row64(const float (&v)[64], float f, __nv_bfloat16* out, float* rec) {
+// Stores 32 values times f: bf16 to `out` or fp32 to `rec` (a chunk of a split tile).
+__device__ __forceinline__ void store32(const float (&v)[32], float f, __nv_bfloat16* out, float* rec) {
   if (rec != nullptr) {
     float4* o = reinterpret_cast<float4*>(rec);
 #pragma unroll
-    for (int x = 0; x < 16; ++x) o[x] = make_float4(v[4 * x] * f, v[4 * x + 1] * f, v[4 * x + 2] * f, v[4 * x + 3] * f);
+    for (int x = 0; x < 8; ++x) o[x] = make_float4(v[4 * x] * f, v[4 * x + 1] * f, v[4 * x + 2] * f, v[4 * x + 3] * f);
   } else {
     uint4* o = reinterpret_cast<uint4*>(out);
 #pragma unroll
-    for (int x = 0; x < 8; ++x) {
+    for (int x = 0; x < 4; ++x) {
       uint4 u;
       u.x = pack_bf16x2(v[8 * x + 0] * f, v[8 * x + 1] * f);
       u.y = pack_bf16x2(v[8 * x + 2] * f, v[8 * x + 3] * f);
@@ -197,300 +178,305 @@ __device__ __forceinline__ void store_row64(const float (&v)[64], float f, __nv_
   }
 }
 
-// ------------------------------------------------------------------ dQ
-__global__ void __launch_bounds__(kThreads, 1) bsa_bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+template <bool kDkv>
+__global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
   const uint32_t bars = base + kSmemBar;
   auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  const uint32_t tmem = cta_setup(smem, base);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemMisc + 4);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const bool leader = tid == 0;
-
-  const int it = blockIdx.x / p.B, b = blockIdx.x - it * p.B;
-  const BwdItem w = p.items[it];
-  const int qa = p.pair[2 * w.pair], qb = p.pair[2 * w.pair + 1];
-  const int row0 = (b * p.H + w.h) * p.L;
-  const int half = tid >> 6;
-  const bool row_active = half == 0 || qb >= 0;
-  const size_t grow = static_cast<size_t>(row0) + static_cast<size_t>(half ? qb : qa) * 64 + (tid & 63);
-  const float lse2 = row_active ? p.lse2[grow] : INFINITY;
-  const float drow = row_active ? p.dsum[grow] : 0.f;
-  const float sl2 = p.scale_log2;
-  const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t sQ = base + kSmemTileA, sDO = base + kSmemTileB, sK = base + kSmemEntA, sV = base + kSmemEntB;
-
-  IssueState is;
-  bool ok = true;
-  const uint64_t pol = ptx::policy_evict_last();
-  auto issue_entry = [&](int n) {  // K_j and V_j of entry n into stage n % 2
-    const int j = static_cast<int>(p.pair_ent[w.start + n] & kEntColMask);
-    const uint32_t st = static_cast<uint32_t>(n) & 1u;
-    ptx::mbar_arrive_expect_tx(bar(kBarEnt + static_cast<int>(st)), 2 * kBlkBytes);
-    ptx::tma_load_2d(sK + st * kBlkBytes, &p.tm_k, bar(kBarEnt + static_cast<int>(st)), 0, row0 + j * 64, pol);
-    ptx::tma_load_2d(sV + st * kBlkBytes, &p.tm_v, bar(kBarEnt + static_cast<int>(st)), 0, row0 + j * 64, pol);
-    ++is.ent_issued;
-  };
-  if (leader) {
-    const int qb_ld = qb >= 0 ? qb : qa;  // a single-block tile loads its block twice
-    ptx::mbar_arrive_expect_tx(bar(kBarTile), 4 * kBlkBytes);
-    ptx::tma_load_2d(sQ, &p.tm_q, bar(kBarTile), 0, row0 + qa * 64, pol);
-    ptx::tma_load_2d(sQ + kBlkBytes, &p.tm_q, bar(kBarTile), 0, row0 + qb_ld * 64, pol);
-    ptx::tma_load_2d(sDO, &p.tm_do, bar(kBarTile), 0, row0 + qa * 64, pol);
-    ptx::tma_load_2d(sDO + kBlkBytes, &p.tm_do, bar(kBarTile), 0, row0 + qb_ld * 64, pol);
-    is.tile_issued = true;
-    issue_entry(0);
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kSmemMisc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNumBars; ++i) {
+      const bool many = (i >= kBarDsFull && i < kBarDsFull + 2) || (i >= kBarAccEmpty && i < kBarAccEmpty + 2);
+      ptx::mbar_init(bar(i), many ? static_cast<uint32_t>(kComputeThreads) : 1u);
+    }
+    misc[1] = 0;
+    ptx::fence_barrier_init();
   }
+  if (warp == kScoreWarp) {
+    ptx::tmem_alloc(ptx::smem_addr(const_cast<uint32_t*>(&misc[0])), kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = misc[0];
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
+  const int total = p.B * p.n_items;
+  constexpr uint32_t kAccCols = kDkv ? 128u : 64u;
+  auto tile_op = [&](uint32_t ts, int op) { return base + kSmemTile + ts * 2 * kOpBytes + op * kOpBytes; };
+  auto ent_op = [&](uint32_t es, int op) { return base + kSmemEnt + es * 2 * kBlkBytes + op * kBlkBytes; };
 
-  for (int n = 0; n < w.count && ok; ++n) {
-    const uint32_t e = p.pair_ent[w.start + n];
-    const uint32_t st = static_cast<uint32_t>(n) & 1u;
-    const uint32_t ph = static_cast<uint32_t>(n) & 1u;  // phase of the once-per-entry barriers
-    if (leader) {
-      // stage st ^ 1 last served entry n - 1, whose MMAs are done (waited below)
-      if (n + 1 < w.count) issue_entry(n + 1);
-      if (n == 0) {
-        ok = wait_one(bar(kBarTile), 0, abort_flag, p.timeout_ns);
-        is.tile_waited = ok;
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      const uint64_t pol = ptx::policy_evict_last();
+      const CUtensorMap* tmA = kDkv ? &p.tm_k : &p.tm_q;   // tile operands
+      const CUtensorMap* tmB = kDkv ? &p.tm_v : &p.tm_do;
+      const CUtensorMap* emA = kDkv ? &p.tm_q : &p.tm_k;   // entry operands
+      const CUtensorMap* emB = kDkv ? &p.tm_do : &p.tm_v;
+      const uint32_t ent_tx = 2 * kBlkBytes + (kDkv ? 2 * kVecBytes : 0u);
+      uint32_t k = 0, g = 0, tiles = 0;  // tiles: tile loads issued; g: entry loads issued
+      bool ok = true;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x, ++k) {
+        const ItemRef r = item_at(p, it);
+        const uint32_t ts = k & 1u;
+        if (!wait_one(bar(kBarTileEmpty + static_cast<int>(ts)), ((k >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        ++tiles;
+        const int tb = r.tb >= 0 ? r.tb : r.ta;  // a single-block tile loads its block twice
+        ptx::mbar_arrive_expect_tx(bar(kBarTileFull + static_cast<int>(ts)), 2 * kOpBytes);
+        ptx::tma_load_2d(tile_op(ts, 0), tmA, bar(kBarTileFull + ts), 0, r.row0 + r.ta * 64, pol);
+        ptx::tma_load_2d(tile_op(ts, 0) + kBlkBytes, tmA, bar(kBarTileFull + ts), 0, r.row0 + tb * 64, pol);
+        ptx::tma_load_2d(tile_op(ts, 1), tmB, bar(kBarTileFull + ts), 0, r.row0 + r.ta * 64, pol);
+        ptx::tma_load_2d(tile_op(ts, 1) + kBlkBytes, tmB, bar(kBarTileFull + ts), 0, r.row0 + tb * 64, pol);
+        for (int n = 0; n < r.w.count; ++n) {
+          const int blk = static_cast<int>(p.pair_ent[r.w.start + n] & kEntColMask);
+          const uint32_t es = g % kEStages;
+          if (!wait_one(bar(kBarEntEmpty + static_cast<int>(es)), ((g / kEStages) & 1u) ^ 1u, abort_flag,
+                        p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          ++g;
+          const uint32_t eb = bar(kBarEntFull + static_cast<int>(es));
+          ptx::mbar_arrive_expect_tx(eb, ent_tx);
+          ptx::tma_load_2d(ent_op(es, 0), emA, eb, 0, r.row0 + blk * 64, pol);
+          ptx::tma_load_2d(ent_op(es, 1), emB, eb, 0, r.row0 + blk * 64, pol);
+          if constexpr (kDkv) {
+            const uint32_t sv = base + kSmemVec + es * 2 * kVecBytes;
+            const size_t off = static_cast<size_t>(r.row0) + static_cast<size_t>(blk) * 64;
+            ptx::bulk_load(sv, p.lse2 + off, kVecBytes, eb);
+            ptx::bulk_load(sv + kVecBytes, p.dsum + off, kVecBytes, eb);
+          }
+        }
       }
-      ok = ok && wait_one(bar(kBarEnt + static_cast<int>(st)), (static_cast<uint32_t>(n) >> 1) & 1u, abort_flag,
-                          p.timeout_ns);
-      if (ok) {
-        ++is.ent_waited;
+      if (!ok) {
+        // let every copy this thread issued land before the CTA exits: the last
+        // issue into ring slot s of a ring of R had index s + R floor((n - 1 - s) / R)
+        auto drain = [&](int first_bar, uint32_t n, uint32_t ring) {
+          for (uint32_t s = 0; s < ring; ++s)
+            if (n > s) {
+              const uint32_t last = s + ring * ((n - 1u - s) / ring);
+              wait_force(bar(first_bar + static_cast<int>(s)), (last / ring) & 1u, abort_flag, p.timeout_ns);
+            }
+        };
+        drain(kBarTileFull, tiles, 2u);
+        drain(kBarEntFull, g, static_cast<uint32_t>(kEStages));
+      }
+    }
+  } else if (warp == kScoreWarp) {
+    if (lane == 0) {
+      // ---------------- score issuer: S and dP of entry g into score stage g % 2
+      uint32_t k = 0, g = 0;
+      bool ok = true, issued = false;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x, ++k) {
+        const ItemRef r = item_at(p, it);
+        const uint32_t ts = k & 1u;
+        if (!wait_one(bar(kBarTileFull + static_cast<int>(ts)), (k >> 1) & 1u, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        for (int n = 0; n < r.w.count; ++n, ++g) {
+          const uint32_t es = g % kEStages, ss = g & 1u;
+          if (!wait_one(bar(kBarEntFull + static_cast<int>(es)), (g / kEStages) & 1u, abort_flag, p.timeout_ns) ||
+              !wait_one(bar(kBarScoreFree + static_cast<int>(ss)), ((g >> 1) & 1u) ^ 1u, abort_flag,
+                        p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t d = tmem + kTmemScore + 128u * ss;
+          mma_rows_x_rows(d, tile_op(ts, 0), ent_op(es, 0));        // S  (or S^T)
+          mma_rows_x_rows(d + 64u, tile_op(ts, 1), ent_op(es, 1));  // dP (or dP^T)
+          ptx::mma_commit(bar(kBarScoreFull + static_cast<int>(ss)));
+          issued = true;
+        }
+        if (ok) ptx::mma_commit(bar(kBarTileEmpty + static_cast<int>(ts)));
+      }
+      if (issued) {  // every MMA of this thread done before TMEM is released
+        ptx::mma_commit(bar(kBarFinal));
+        wait_force(bar(kBarFinal), 0, abort_flag, p.timeout_ns);
+      }
+    }
+  } else if (warp == kAccWarp) {
+    if (lane == 0) {
+      // ---------------- accumulate issuer
+      uint32_t k = 0, g = 0;
+      bool ok = true, issued = false;
+      for (int it = blockIdx.x; it < total && ok; it += gridDim.x, ++k) {
+        const ItemRef r = item_at(p, it);
+        const uint32_t as = k & 1u;
+        if (!wait_one(bar(kBarAccEmpty + static_cast<int>(as)), ((k >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const uint32_t acc = tmem + kTmemAcc + kAccCols * as;
+        for (int n = 0; n < r.w.count; ++n, ++g) {
+          const uint32_t es = g % kEStages, ss = g & 1u;
+          if (!wait_one(bar(kBarDsFull + static_cast<int>(ss)), (g >> 1) & 1u, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sc = tmem + kTmemScore + 128u * ss;
+          if constexpr (kDkv) {
+            mma_tmem_x_block(acc, sc, ent_op(es, 1), n > 0);              // dV += P^T dO_i
+            mma_tmem_x_block(acc + 64u, sc + 64u, ent_op(es, 0), n > 0);  // dK += dS^T Q_i
+          } else {
+            mma_tmem_x_block(acc, sc, ent_op(es, 0), n > 0);  // dQ += dS K_j
+          }
+          ptx::mma_commit(bar(kBarScoreFree + static_cast<int>(ss)));
+          ptx::mma_commit(bar(kBarEntEmpty + static_cast<int>(es)));
+          issued = true;
+        }
+        if (ok) ptx::mma_commit(bar(kBarAccFull + static_cast<int>(as)));
+      }
+      if (issued) {
+        ptx::mma_commit(bar(kBarFinal + 1));
+        wait_force(bar(kBarFinal + 1), 0, abort_flag, p.timeout_ns);
+      }
+    }
+  } else {
+    // ---------------- compute warps (the single-lane roles above rejoin their
+    // warps below)
+    const int quad = warp & 3, ch = warp >> 2;  // TMEM lane quadrant, column half
+    const int r = quad * 32 + lane;               // tile row
+    const int half = r >> 6;                      // which block of the tile
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    const float sl2 = p.scale_log2;
+    uint32_t k = 0, g = 0;
+    bool ok = true;
+    // the previous tile, whose epilogue runs after this tile's first entry
+    bool have_pend = false;
+    uint32_t pend_k = 0;
+    ItemRef pend{};
+    auto epilogue = [&](uint32_t kt, const ItemRef& t) -> bool {
+      const uint32_t as = kt & 1u;
+      if (!wait_warp(bar(kBarAccFull + static_cast<int>(as)), (kt >> 1) & 1u, abort_flag, p.timeout_ns)) return false;
+      ptx::tc_fence_after();
+      const bool active = half == 0 || t.tb >= 0;
+      const size_t grow =
+          static_cast<size_t>(t.row0) + static_cast<size_t>(half ? t.tb : t.ta) * 64 + static_cast<size_t>(r & 63);
+      const uint32_t acc = tmem + lane_addr + kTmemAcc + kAccCols * as + 32u * ch;
+      float* rec = nullptr;
+      if (t.w.rec >= 0)
+        rec = p.records + (static_cast<size_t>(t.b) * p.n_records + t.w.rec) * (kDkv ? kBwdDkvRecFloats : kBwdDqRecFloats) +
+              static_cast<size_t>(r) * 64 + 32 * ch;
+      float v[32];
+      if constexpr (kDkv) {
+        load32(acc + 64u, v);  // dK
+        if (active) store32(v, p.scale, p.dk + grow * 64 + 32 * ch, rec);
+        load32(acc, v);  // dV
+        if (active) store32(v, 1.f, p.dv + grow * 64 + 32 * ch, rec != nullptr ? rec + kTileRows * 64 : nullptr);
+      } else {
+        load32(acc, v);
+        if (active) store32(v, p.scale, p.dq + grow * 64 + 32 * ch, rec);
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(bar(kBarAccEmpty + static_cast<int>(as)));
+      return true;
+    };
+    for (int it = blockIdx.x; it < total && ok; it += gridDim.x, ++k) {
+      const ItemRef t = item_at(p, it);
+      const bool active = half == 0 || t.tb >= 0;
+      const int blk = half ? t.tb : t.ta;
+      // dQ: this row's lse (log2) and D; dKV: whether this key is kept by the padding mask
+      float lse2 = INFINITY, drow = 0.f;
+      bool key_kept = false;
+      if constexpr (kDkv) {
+        key_kept = active && (p.keybits == nullptr ||
+                              ((p.keybits[static_cast<size_t>(t.b) * p.nb + blk] >> (r & 63)) & 1ull));
+      } else if (active) {
+        const size_t grow = static_cast<size_t>(t.row0) + static_cast<size_t>(blk) * 64 + (r & 63);
+        lse2 = p.lse2[grow];
+        drow = p.dsum[grow];
+      }
+      for (int n = 0; n < t.w.count; ++n, ++g) {
+        const uint32_t e = p.pair_ent[t.w.start + n];
+        const uint32_t ss = g & 1u, es = g % kEStages;
+        if (!wait_warp(bar(kBarScoreFull + static_cast<int>(ss)), (g >> 1) & 1u, abort_flag, p.timeout_ns)) {
+          ok = false;
+          break;
+        }
+        if constexpr (kDkv) {  // the entry's lse2 and D vectors are read from its stage
+          if (!wait_warp(bar(kBarEntFull + static_cast<int>(es)), (g / kEStages) & 1u, abort_flag, p.timeout_ns)) {
+            ok = false;
+            break;
+          }
+        }
         ptx::tc_fence_after();
-        mma_rows_x_rows(tmem + kTmemA, sQ, sK + st * kBlkBytes);    // S = Q K_j^T
-        mma_rows_x_rows(tmem + kTmemB, sDO, sV + st * kBlkBytes);   // dP = dO V_j^T
-        ptx::mma_commit(bar(kBarSdp));
-        is.mma_issued = true;
-      }
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) break;
-    if (!wait_warp(bar(kBarSdp), ph, abort_flag, p.timeout_ns)) {
-      ok = false;
-      break;
-    }
-    ptx::tc_fence_after();
-    // this half's keys of block j: membership bit, then key padding
-    unsigned long long mk = 0ull;
-    if (row_active && ((e >> (kEntBitsShift + half)) & 1u))
-      mk = p.keybits != nullptr ? p.keybits[static_cast<size_t>(b) * p.nb + (e & kEntColMask)] : ~0ull;
-    uint32_t pk[32];
-    if (mk != 0ull) {  // warp-uniform
-#pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
+        const uint32_t sc = tmem + lane_addr + kTmemScore + 128u * ss + 32u * ch;
         uint32_t s_raw[32], dp_raw[32];
-        ptx::tmem_ld32(tmem + lane_addr + kTmemA + 32u * hc, s_raw);
-        ptx::tmem_ld32(tmem + lane_addr + kTmemB + 32u * hc, dp_raw);
+        ptx::tmem_ld32(sc, s_raw);
+        ptx::tmem_ld32(sc + 64u, dp_raw);
         ptx::tmem_wait_ld();
         ptx::reg_fence(s_raw);
         ptx::reg_fence(dp_raw);
+        const bool member = active && ((e >> (kEntBitsShift + half)) & 1u);
+        if constexpr (kDkv) {
+          const bool take = member && key_kept;
+          const float* vec = reinterpret_cast<const float*>(smem + kSmemVec + es * 2 * kVecBytes) + 32 * ch;
+          uint32_t ppk[16], dpk[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int c0 = 32 * hc + 2 * c;
-          const float p0 = ((mk >> c0) & 1ull) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - lse2) : 0.f;
-          const float p1 =
-              ((mk >> (c0 + 1)) & 1ull) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - lse2) : 0.f;
-          pk[16 * hc + c] = pack_bf16x2(p0 * (__uint_as_float(dp_raw[2 * c]) - drow),
-                                        p1 * (__uint_as_float(dp_raw[2 * c + 1]) - drow));
+          for (int c = 0; c < 16; ++c) {
+            const float2 l2 = *reinterpret_cast<const float2*>(vec + 2 * c);
+            const float2 dd = *reinterpret_cast<const float2*>(vec + 64 + 2 * c);
+            const float p0 = take ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - l2.x) : 0.f;
+            const float p1 = take ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - l2.y) : 0.f;
+            ppk[c] = pack_bf16x2(p0, p1);
+            dpk[c] = pack_bf16x2(p0 * (__uint_as_float(dp_raw[2 * c]) - dd.x),
+                                 p1 * (__uint_as_float(dp_raw[2 * c + 1]) - dd.y));
+          }
+          ptx::tmem_st16(sc, ppk);         // P^T over S^T columns this warp has read
+          ptx::tmem_st16(sc + 64u, dpk);   // dS^T over dP^T columns this warp has read
+        } else {
+          unsigned long long mk = 0ull;
+          if (member)
+            mk = p.keybits != nullptr ? p.keybits[static_cast<size_t>(t.b) * p.nb + (e & kEntColMask)] : ~0ull;
+          const uint32_t mh = static_cast<uint32_t>(mk >> (32 * ch));  // this warp's 32 keys
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float p0 = ((mh >> (2 * c)) & 1u) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - lse2) : 0.f;
+            const float p1 =
+                ((mh >> (2 * c + 1)) & 1u) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - lse2) : 0.f;
+            pk[c] = pack_bf16x2(p0 * (__uint_as_float(dp_raw[2 * c]) - drow),
+                                p1 * (__uint_as_float(dp_raw[2 * c + 1]) - drow));
+          }
+          ptx::tmem_st16(sc, pk);  // dS over S columns this warp has read
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(bar(kBarDsFull + static_cast<int>(ss)));
+        if (n == 0 && have_pend) {
+          have_pend = false;
+          if (!epilogue(pend_k, pend)) {
+            ok = false;
+            break;
+          }
         }
       }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = 0u;
-    }
-    ptx::tmem_st32(tmem + lane_addr + kTmemA, pk);  // dS over S columns already read
-    ptx::tmem_wait_st();
-    ptx::tc_fence_before();
-    ptx::mbar_arrive(bar(kBarDs));
-    if (leader) {
-      ok = wait_one(bar(kBarDs), ph, abort_flag, p.timeout_ns);
-      if (ok) {
-        ptx::tc_fence_after();
-        mma_tmem_x_block(tmem + kTmemC, tmem + kTmemA, sK + st * kBlkBytes, n > 0);  // dQ += dS K_j
-        ptx::mma_commit(bar(kBarAcc));
-        ok = wait_one(bar(kBarAcc), ph, abort_flag, p.timeout_ns);
-      }
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);  // keep the loop warp-uniform
-  }
-  ok = __syncthreads_and(ok ? 1 : 0) != 0;
-  if (ok && w.count > 0) {
-    if (!wait_warp(bar(kBarAcc), static_cast<uint32_t>(w.count - 1) & 1u, abort_flag, p.timeout_ns)) ok = false;
-  }
-  if (ok) {
-    ptx::tc_fence_after();
-    float v[64];
-    load_row64(tmem + lane_addr + kTmemC, v);
-    if (row_active) {
-      float* rec = w.rec >= 0 ? p.records + (static_cast<size_t>(b) * p.n_records + w.rec) * kBwdDqRecFloats +
-                                    static_cast<size_t>(tid) * 64
-                              : nullptr;
-      store_row64(v, p.scale, p.dq + grow * 64, rec);
-    }
-  } else if (leader) {
-    drain(is, bars, abort_flag, p.timeout_ns);
-  }
-  cta_teardown(tmem);
-}
-
-// ------------------------------------------------------------------ dK, dV
-__global__ void __launch_bounds__(kThreads, 1) bsa_bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = ptx::smem_addr(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* smem = smem_raw + (base - raw);
-  const uint32_t bars = base + kSmemBar;
-  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  const uint32_t tmem = cta_setup(smem, base);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemMisc + 4);
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const bool leader = tid == 0;
-
-  const int it = blockIdx.x / p.B, b = blockIdx.x - it * p.B;
-  const BwdItem w = p.items[it];
-  const int ka = p.pair[2 * w.pair], kb = p.pair[2 * w.pair + 1];
-  const int row0 = (b * p.H + w.h) * p.L;
-  const int half = tid >> 6;
-  const bool row_active = half == 0 || kb >= 0;
-  const int kblk = half ? kb : ka;
-  const size_t grow = static_cast<size_t>(row0) + static_cast<size_t>(kblk) * 64 + (tid & 63);
-  // this key row takes part at all: its key is not dropped by the padding mask
-  const bool key_kept =
-      row_active && (p.keybits == nullptr || ((p.keybits[static_cast<size_t>(b) * p.nb + kblk] >> (tid & 63)) & 1ull));
-  const float sl2 = p.scale_log2;
-  const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-  const uint32_t sK = base + kSmemTileA, sV = base + kSmemTileB, sQ = base + kSmemEntA, sDO = base + kSmemEntB;
-  const float* vec = reinterpret_cast<const float*>(smem + kSmemVec);  // [stage][lse2 64, D 64]
-
-  IssueState is;
-  bool ok = true;
-  const uint64_t pol = ptx::policy_evict_last();
-  auto issue_entry = [&](int n) {  // Q_i, dO_i, lse2 and D of query block i into stage n % 2
-    const int i = static_cast<int>(p.pair_ent[w.start + n] & kEntColMask);
-    const uint32_t st = static_cast<uint32_t>(n) & 1u;
-    const uint32_t eb = bar(kBarEnt + static_cast<int>(st));
-    ptx::mbar_arrive_expect_tx(eb, 2 * kBlkBytes + 2 * kVecBytes);
-    ptx::tma_load_2d(sQ + st * kBlkBytes, &p.tm_q, eb, 0, row0 + i * 64, pol);
-    ptx::tma_load_2d(sDO + st * kBlkBytes, &p.tm_do, eb, 0, row0 + i * 64, pol);
-    const uint32_t sv = base + kSmemVec + st * 2 * kVecBytes;
-    ptx::bulk_load(sv, p.lse2 + static_cast<size_t>(row0) + static_cast<size_t>(i) * 64, kVecBytes, eb);
-    ptx::bulk_load(sv + kVecBytes, p.dsum + static_cast<size_t>(row0) + static_cast<size_t>(i) * 64, kVecBytes, eb);
-    ++is.ent_issued;
-  };
-  if (leader) {
-    const int kb_ld = kb >= 0 ? kb : ka;
-    ptx::mbar_arrive_expect_tx(bar(kBarTile), 4 * kBlkBytes);
-    ptx::tma_load_2d(sK, &p.tm_k, bar(kBarTile), 0, row0 + ka * 64, pol);
-    ptx::tma_load_2d(sK + kBlkBytes, &p.tm_k, bar(kBarTile), 0, row0 + kb_ld * 64, pol);
-    ptx::tma_load_2d(sV, &p.tm_v, bar(kBarTile), 0, row0 + ka * 64, pol);
-    ptx::tma_load_2d(sV + kBlkBytes, &p.tm_v, bar(kBarTile), 0, row0 + kb_ld * 64, pol);
-    is.tile_issued = true;
-    issue_entry(0);
-  }
-
-  for (int n = 0; n < w.count && ok; ++n) {
-    const uint32_t e = p.pair_ent[w.start + n];
-    const uint32_t st = static_cast<uint32_t>(n) & 1u;
-    const uint32_t ph = static_cast<uint32_t>(n) & 1u;
-    if (leader) {
-      if (n + 1 < w.count) issue_entry(n + 1);
-      if (n == 0) {
-        ok = wait_one(bar(kBarTile), 0, abort_flag, p.timeout_ns);
-        is.tile_waited = ok;
-      }
-    }
-    // every thread: the entry's stage landed (the threads read lse2 and D from it)
-    if (!wait_warp(bar(kBarEnt + static_cast<int>(st)), (static_cast<uint32_t>(n) >> 1) & 1u, abort_flag,
-                   p.timeout_ns)) {
-      ok = false;
-      break;
-    }
-    if (leader) {
-      ++is.ent_waited;
       ok = ok && !*abort_flag;
-      if (ok) {
-        ptx::tc_fence_after();
-        mma_rows_x_rows(tmem + kTmemA, sK, sQ + st * kBlkBytes);    // S^T = K Q_i^T
-        mma_rows_x_rows(tmem + kTmemB, sV, sDO + st * kBlkBytes);   // dP^T = V dO_i^T
-        ptx::mma_commit(bar(kBarSdp));
-        is.mma_issued = true;
-      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      have_pend = true;
+      pend_k = k;
+      pend = t;
     }
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) break;
-    if (!wait_warp(bar(kBarSdp), ph, abort_flag, p.timeout_ns)) {
-      ok = false;
-      break;
-    }
-    ptx::tc_fence_after();
-    const bool take = key_kept && ((e >> (kEntBitsShift + half)) & 1u);  // warp-uniform membership
-    uint32_t ppk[32], dpk[32];
-    if (__any_sync(0xffffffffu, take)) {
-      const float* l2 = vec + st * 128;
-      const float* dd = l2 + 64;
-#pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
-        uint32_t s_raw[32], dp_raw[32];
-        ptx::tmem_ld32(tmem + lane_addr + kTmemA + 32u * hc, s_raw);
-        ptx::tmem_ld32(tmem + lane_addr + kTmemB + 32u * hc, dp_raw);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence(s_raw);
-        ptx::reg_fence(dp_raw);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int c0 = 32 * hc + 2 * c;
-          const float2 lv = *reinterpret_cast<const float2*>(l2 + c0);
-          const float2 dv2 = *reinterpret_cast<const float2*>(dd + c0);
-          const float p0 = take ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - lv.x) : 0.f;
-          const float p1 = take ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - lv.y) : 0.f;
-          ppk[16 * hc + c] = pack_bf16x2(p0, p1);
-          dpk[16 * hc + c] = pack_bf16x2(p0 * (__uint_as_float(dp_raw[2 * c]) - dv2.x),
-                                         p1 * (__uint_as_float(dp_raw[2 * c + 1]) - dv2.y));
-        }
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 32; ++c) ppk[c] = dpk[c] = 0u;
-    }
-    ptx::tmem_st32(tmem + lane_addr + kTmemA, ppk);  // P^T over S^T columns already read
-    ptx::tmem_st32(tmem + lane_addr + kTmemB, dpk);  // dS^T over dP^T columns already read
-    ptx::tmem_wait_st();
-    ptx::tc_fence_before();
-    ptx::mbar_arrive(bar(kBarDs));
-    if (leader) {
-      ok = wait_one(bar(kBarDs), ph, abort_flag, p.timeout_ns);
-      if (ok) {
-        ptx::tc_fence_after();
-        mma_tmem_x_block(tmem + kTmemC, tmem + kTmemA, sDO + st * kBlkBytes, n > 0);  // dV += P^T dO_i
-        mma_tmem_x_block(tmem + kTmemD, tmem + kTmemB, sQ + st * kBlkBytes, n > 0);   // dK += dS^T Q_i
-        ptx::mma_commit(bar(kBarAcc));
-        ok = wait_one(bar(kBarAcc), ph, abort_flag, p.timeout_ns);
-      }
-    }
-    ok = __shfl_sync(0xffffffffu, ok, 0);  // keep the loop warp-uniform
+    if (ok && have_pend) epilogue(pend_k, pend);
   }
-  ok = __syncthreads_and(ok ? 1 : 0) != 0;
-  if (ok && w.count > 0) {
-    if (!wait_warp(bar(kBarAcc), static_cast<uint32_t>(w.count - 1) & 1u, abort_flag, p.timeout_ns)) ok = false;
-  }
-  if (ok) {
-    ptx::tc_fence_after();
-    float* rec = w.rec >= 0 ? p.records + (static_cast<size_t>(b) * p.n_records + w.rec) * kBwdDkvRecFloats +
-                                  static_cast<size_t>(tid) * 64
-                            : nullptr;
-    float v[64];
-    load_row64(tmem + lane_addr + kTmemD, v);
-    if (row_active) store_row64(v, p.scale, p.dk + grow * 64, rec);
-    load_row64(tmem + lane_addr + kTmemC, v);
-    if (row_active) store_row64(v, 1.f, p.dv + grow * 64, rec != nullptr ? rec + kTileRows * 64 : nullptr);
-  } else if (leader) {
-    drain(is, bars, abort_flag, p.timeout_ns);
-  }
-  cta_teardown(tmem);
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == kScoreWarp) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------ D, lse2
@@ -564,6 +550,7 @@ __global__ void __launch_bounds__(128) bsa_bwd_merge_kernel(const __grid_constan
 constexpr int kMaxDevices = 64;
 std::once_flag g_setup_once[kMaxDevices];
 int g_setup_status[kMaxDevices];
+int g_sms[kMaxDevices];
 
 int bwd_device_setup(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
@@ -578,13 +565,16 @@ int bwd_device_setup(int dev) {
       g_setup_status[dev] = BSA_ERR_UNSUPPORTED;
       return;
     }
-    if (cudaFuncSetAttribute(bsa_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaFuncSetAttribute(bsa_bwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemAlloc)) != cudaSuccess ||
-        cudaFuncSetAttribute(bsa_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(bsa_bwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemAlloc)) != cudaSuccess) {
       g_setup_status[dev] = BSA_ERR_CUDA;
       return;
     }
+    g_sms[dev] = sms;
     g_setup_status[dev] = BSA_OK;
   });
   return g_setup_status[dev];
@@ -678,9 +668,10 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   pq.pair_ent = lay->d_pair_ent;
   pq.records = reinterpret_cast<float*>(ws + plan.dq_rec_off);
   pq.n_records = lay->dq_plan.n_records;
-  const int64_t gq = static_cast<int64_t>(B) * static_cast<int64_t>(lay->dq_plan.items.size());
+  pq.n_items = static_cast<int>(lay->dq_plan.items.size());
+  const int64_t gq = std::min<int64_t>(static_cast<int64_t>(B) * pq.n_items, g_sms[dev]);
   if (gq > 0) {
-    bsa_bwd_dq_kernel<<<static_cast<unsigned>(gq), kThreads, kSmemAlloc, s>>>(pq);
+    bsa_bwd_kernel<false><<<static_cast<unsigned>(gq), kThreads, kSmemAlloc, s>>>(pq);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   // dK and dV over the key tiles
@@ -690,9 +681,10 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   pk.pair_ent = lay->d_kpair_ent;
   pk.records = reinterpret_cast<float*>(ws + plan.dkv_rec_off);
   pk.n_records = lay->dkv_plan.n_records;
-  const int64_t gk = static_cast<int64_t>(B) * static_cast<int64_t>(lay->dkv_plan.items.size());
+  pk.n_items = static_cast<int>(lay->dkv_plan.items.size());
+  const int64_t gk = std::min<int64_t>(static_cast<int64_t>(B) * pk.n_items, g_sms[dev]);
   if (gk > 0) {
-    bsa_bwd_dkv_kernel<<<static_cast<unsigned>(gk), kThreads, kSmemAlloc, s>>>(pk);
+    bsa_bwd_kernel<true><<<static_cast<unsigned>(gk), kThreads, kSmemAlloc, s>>>(pk);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   const int n_dq_split = static_cast<int>(lay->dq_plan.splits.size());
