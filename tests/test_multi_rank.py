@@ -1,9 +1,10 @@
 """Multi-rank host logic on CPU with two gloo ranks (no GPU).
 
-A forward split by batch element across ranks, each rank computing its shard
-(here with the fp64 oracle, since no GPU is present), must reproduce the
-single-process result once gathered; the timing reduction must return the
-maximum over ranks.
+A forward, and a backward, split by batch element across ranks, each rank
+computing its shard (here with the fp64 oracle, since no GPU is present), must
+reproduce the single-process result once gathered -- the gradients of one batch
+element, dK and dV included, depend on that element alone; the timing reduction
+must return the maximum over ranks.
 """
 
 import os
@@ -18,6 +19,7 @@ import torch.multiprocessing as mp
 import workloads
 from block_sparse_attention_bigbird_b200 import sharding
 from oracle import attention as OA
+from oracle import backward as OB
 from oracle import layout as OL
 
 
@@ -76,3 +78,47 @@ def test_two_gloo_ranks_reproduce_single_process():
     o = np.concatenate([s[2] for s in sorted(shards, key=lambda x: x[0])])
     lse = np.concatenate([s[3] for s in sorted(shards, key=lambda x: x[0])])
     assert np.array_equal(o, o_ref) and np.array_equal(lse, lse_ref)
+
+
+def _worker_bwd(rank, world, port, queue):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = workloads.custom(3, 2, 64 * 5, 1, 1, 1, seed=4, key_pad_tail=20)
+        q, k, v = workloads.make_qkv(w)
+        do = workloads.make_grad(w, seed=7)
+        km = workloads.make_key_mask(w)
+        lay = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+        b0, b1 = sharding.batch_shard(w.B, rank, world)
+        grads = OB.attention_backward(q[b0:b1], k[b0:b1], v[b0:b1], do[b0:b1], lay, key_mask=km[b0:b1])
+        shards = [None] * world
+        dist.all_gather_object(shards, (b0, b1, grads))
+        if rank == 0:
+            queue.put(shards)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_backward_reproduce_single_process():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_bwd, args=(r, 2, port, queue)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    shards = queue.get(timeout=120)
+    for pr in procs:
+        pr.join(timeout=120)
+        assert pr.exitcode == 0
+    w = workloads.custom(3, 2, 64 * 5, 1, 1, 1, seed=4, key_pad_tail=20)
+    q, k, v = workloads.make_qkv(w)
+    do = workloads.make_grad(w, seed=7)
+    km = workloads.make_key_mask(w)
+    lay = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    ref = OB.attention_backward(q, k, v, do, lay, key_mask=km)
+    shards = sorted(shards, key=lambda x: x[0])
+    for i in range(3):
+        got = np.concatenate([s[2][i] for s in shards])
+        assert np.array_equal(got, ref[i])
