@@ -17,27 +17,17 @@ import random
 
 import pytest
 
+from protocol_model import Bar, replay, wait
+
 E_STAGES = 4
 COMPUTE_WARPS = 8
-
-
-class _Bar:
-    def __init__(self, name, count):
-        self.name, self.count, self.arrivals, self.done = name, count, 0, 0
-
-    def arrive(self):
-        self.arrivals += 1
-        assert self.arrivals <= self.count, self.name
-        if self.arrivals == self.count:
-            self.arrivals = 0
-            self.done += 1
 
 
 def _roles(dkv, counts):
     bars = {}
 
     def bar(name, count=1):
-        bars[name] = _Bar(name, count)
+        bars[name] = Bar(name, count)
 
     for i in range(2):
         for n in ("TileFull", "TileEmpty", "ScoreFull", "ScoreFree", "AccFull"):
@@ -47,9 +37,6 @@ def _roles(dkv, counts):
     for i in range(E_STAGES):
         bar(f"EntFull{i}")
         bar(f"EntEmpty{i}")
-
-    def wait(name, phase):  # wait for the completion of phase `phase` (no-op if < 0)
-        return ("wait", name, phase) if phase >= 0 else None
 
     prod, score, acc = [], [], []
     g = 0
@@ -85,44 +72,12 @@ def _roles(dkv, counts):
         if pend is not None:
             ops += [wait(f"AccFull{pend & 1}", pend >> 1), ("arrive", f"AccEmpty{pend & 1}")]
         roles[f"compute{w}"] = ops
-    return bars, {r: [o for o in ops if o is not None] for r, ops in roles.items()}
+    return bars, roles
 
 
 def _run(dkv, counts, seed):
-    rnd = random.Random(seed)
     bars, roles = _roles(dkv, counts)
-    pc = {r: 0 for r in roles}
-    inflight = []
-    while True:
-        runnable = []
-        for r, ops in roles.items():
-            if pc[r] == len(ops):
-                continue
-            op = ops[pc[r]]
-            if op[0] == "wait":
-                b, t = bars[op[1]], op[2]
-                if (b.done & 1) != (t & 1):  # try_wait.parity: the phase of t's parity completed
-                    assert b.done == t + 1, f"{r}: {op} satisfied by a later phase (done={b.done})"
-                    runnable.append(r)
-                else:
-                    assert b.done <= t, f"{r}: {op} waits for a phase already gone (done={b.done})"
-            else:
-                runnable.append(r)
-        choices = runnable + (["async"] if inflight else [])
-        if not choices:
-            stuck = [(r, roles[r][pc[r]]) for r in roles if pc[r] < len(roles[r])]
-            assert not stuck, f"deadlock: {stuck}"
-            return
-        c = rnd.choice(choices)
-        if c == "async":
-            bars[inflight.pop(rnd.randrange(len(inflight)))].arrive()
-            continue
-        op = roles[c][pc[c]]
-        pc[c] += 1
-        if op[0] == "arrive":
-            bars[op[1]].arrive()
-        elif op[0] == "async":
-            inflight.append(op[1])
+    replay(bars, roles, seed)
 
 
 @pytest.mark.parametrize("dkv", [False, True], ids=["dq", "dkv"])
@@ -142,7 +97,7 @@ def test_the_model_catches_a_missing_release():
 
     def broken(dkv, counts):
         bars, roles = orig(dkv, counts)
-        roles["score"] = [o for o in roles["score"] if not (o[0] == "wait" and o[1].startswith("ScoreFree"))]
+        roles["score"] = [o for o in roles["score"] if not (o and o[0] == "wait" and o[1].startswith("ScoreFree"))]
         return bars, roles
 
     m._roles = broken
