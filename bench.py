@@ -309,17 +309,32 @@ def run_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
-    q, k, v = workloads.make_qkv(w, data_seed=rank)
     km = workloads.make_key_mask(w)
     lay = bsa.bsa_layout_build(w.H, w.L, w.block, w.window, w.n_global, w.n_random, w.seed)
-    bsa.bsa_layout_upload(lay)
     row_ptr, col_idx = bsa.bsa_layout_csr(lay)
+    heads = args.shard == "heads"
+    if heads:
+        # strong scaling over heads: every rank takes its heads of the same sequence
+        # (the genomic shape has one batch element) and a layout of those heads' rows
+        if world > w.H:
+            raise SystemExit(f"--shard heads needs at most {w.H} ranks")
+        h0, h1 = sharding.head_shard(w.H, rank, world)
+        total_flop = _nnz_eff(w, row_ptr, col_idx) * FLOP_PER_BLOCK
+        row_ptr, col_idx = sharding.head_rows(row_ptr, col_idx, w.nb, h0, h1)
+        lay = bsa.bsa_layout_from_csr(h1 - h0, w.L, row_ptr, col_idx)
+        q, k, v = (t[:, h0:h1].contiguous() for t in workloads.make_qkv(w, data_seed=0))
+    else:
+        q, k, v = workloads.make_qkv(w, data_seed=rank)
+    bsa.bsa_layout_upload(lay)
+    H_r = q.shape[1]
     nnz_eff = _nnz_eff(w, row_ptr, col_idx)
     flop_step = nnz_eff * FLOP_PER_BLOCK
+    # work of the whole job per step: every rank's own batch (weak), or one sequence's heads (strong)
+    job_flop = total_flop if heads else world * flop_step
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     kmd = km.to(dev) if km is not None else None
     out = torch.empty_like(qd)
-    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, H_r, w.L), dtype=torch.float32, device=dev)
     ws = torch.zeros(bsa.bsa_workspace_bytes(lay, w.B), dtype=torch.uint8, device=dev)
     # forward, plus the key-bit kernel with a key mask and the merge with split rows
     launches_per_step = 1 + (1 if km is not None else 0) + (1 if _has_split_rows(lay) else 0)
@@ -429,11 +444,11 @@ def run_ours(args, w, world, rank, local):
         raise RuntimeError("device status error in the end-to-end run")
 
     ms_per_step = total_ms / args.steps
-    value = world * flop_step / (ms_per_step * 1e-3) / 1e12
+    value = job_flop / (ms_per_step * 1e-3) / 1e12
     peaks, peak_src = _peaks()
     achieved = flop_step / (kernel_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = _traffic_for(w.name)
+    traffic = _traffic_for(w.name) if not heads or world == 1 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(w)
@@ -442,9 +457,10 @@ def run_ours(args, w, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if heads else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded randn, see workloads.py)",
-        "config": _config(w, nnz_eff, world),
+        "config": dict(_config(w, nnz_eff, world),
+                       **({"parallelism": f"heads{world}", "global_batch": w.B} if heads else {})),
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": traffic,
@@ -452,7 +468,7 @@ def run_ours(args, w, world, rank, local):
                      "peak_source": f"{peak_src} bf16 burst",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
                      "ex2": _ex2_ceiling(nnz_eff, kernel_ms, dev, peaks)},
-        "e2e": {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+        "e2e": {"value": job_flop / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "pipelining": "double-buffered device tensors; host->device copy, forward and "
                               "device->host read on three streams, overlapped across steps"},
@@ -640,6 +656,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
                     help="forward (the default benchmark) or the backward pass")
+    ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
+                    help="forward over N ranks: each rank its own batch (weak scaling, the default) "
+                         "or the heads of one batch split across ranks (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

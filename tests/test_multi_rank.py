@@ -122,3 +122,53 @@ def test_two_gloo_ranks_backward_reproduce_single_process():
     for i in range(3):
         got = np.concatenate([s[2][i] for s in shards])
         assert np.array_equal(got, ref[i])
+
+
+def _worker_heads(rank, world, port, queue):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # one long-ish sequence (B = 1), its heads split across the ranks; each rank
+        # builds its own layout from its heads' rows with the library's CSR builder
+        from block_sparse_attention_bigbird_b200 import bsa
+        w = workloads.custom(1, 5, 64 * 12, 1, 2, 2, seed=9, key_pad_tail=30)
+        q, k, v = workloads.make_qkv(w)
+        km = workloads.make_key_mask(w)
+        full = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+        rp, ci = bsa.bsa_layout_csr(full)
+        h0, h1 = sharding.head_shard(w.H, rank, world)
+        srp, sci = sharding.head_rows(rp, ci, w.nb, h0, h1)
+        mine = bsa.bsa_layout_from_csr(h1 - h0, w.L, srp, sci)
+        r2, c2 = bsa.bsa_layout_csr(mine)
+        lay = {"H": h1 - h0, "L": w.L, "block": 64, "nb": w.nb, "row_ptr": r2.astype(np.int64), "col_idx": c2}
+        o, lse = OA.attention(q[:, h0:h1], k[:, h0:h1], v[:, h0:h1], lay, key_mask=km)
+        shards = [None] * world
+        dist.all_gather_object(shards, (h0, h1, o, lse))
+        if rank == 0:
+            queue.put(shards)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_shard_rows_and_two_gloo_ranks_reproduce_single_process():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_heads, args=(r, 2, port, queue)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    shards = queue.get(timeout=120)
+    for pr in procs:
+        pr.join(timeout=120)
+        assert pr.exitcode == 0
+    w = workloads.custom(1, 5, 64 * 12, 1, 2, 2, seed=9, key_pad_tail=30)
+    q, k, v = workloads.make_qkv(w)
+    km = workloads.make_key_mask(w)
+    lay = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    o_ref, lse_ref = OA.attention(q, k, v, lay, key_mask=km)
+    shards = sorted(shards, key=lambda x: x[0])
+    assert [s[:2] for s in shards] == [(0, 3), (3, 5)]
+    assert np.array_equal(np.concatenate([s[2] for s in shards], axis=1), o_ref)
+    assert np.array_equal(np.concatenate([s[3] for s in shards], axis=1), lse_ref)
