@@ -1,7 +1,9 @@
 // Host side of the BigBird block-sparse attention library: the seeded layout
-// builder, the 128-row tile decomposition and the static work list.  Pure C++,
-// no GPU needed.  Every entry point validates its arguments and returns a
-// bsa_status; no exception crosses the C ABI.
+// builder, layouts from a caller's block CSR, the 128-row tile decomposition
+// (query-major for the forward and dQ, key-major over the transposed layout for
+// dK and dV) and the work lists.  Pure C++, no GPU needed.  Every entry point
+// validates its arguments and returns a bsa_status; no exception crosses the C
+// ABI.
 #include <algorithm>
 #include <cstring>
 #include <new>

@@ -1,5 +1,6 @@
 // Internal structures shared by the host library (bsa_host.cpp) and the CUDA
-// forward (bsa_fwd_sm100.cu).  Not part of the public ABI.
+// forward (bsa_fwd_sm100.cu) and backward (bsa_bwd_sm100.cu).  Not part of the
+// public ABI.
 #pragma once
 
 #include <cstddef>
