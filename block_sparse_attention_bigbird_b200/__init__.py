@@ -15,12 +15,14 @@ __all__ = ["bsa_layout_build", "bsa_layout_from_csr", "bsa_layout_csr", "bsa_lay
            "bsa_layout_tiles", "bsa_layout_key_tiles", "bsa_layout_upload", "bsa_workspace_bytes",
            "bsa_forward", "bsa_backward", "bsa_backward_workspace_bytes", "bsa_sync_status",
            "bsa_strerror", "bsa_debug_wait_timeout", "bsa_forward_static_ws", "Layout", "BsaError",
-           "block_sparse_attention"]
+           "block_sparse_attention", "BigBirdSelfAttention"]
 
 
 def __getattr__(name):
     if name == "block_sparse_attention":
         return getattr(importlib.import_module(".autograd", __name__), name)
+    if name == "BigBirdSelfAttention":
+        return getattr(importlib.import_module(".layer", __name__), name)
     if name in __all__:
         return getattr(importlib.import_module(".bsa", __name__), name)
     raise AttributeError(name)

@@ -1,0 +1,113 @@
+"""BigBirdSelfAttention: QKV projection, block-sparse attention, output projection.
+
+CPU: the layer with the library's kernels replaced by fakes built on the fp64
+oracle, against a dense fp64 torch implementation of the same layer (masked
+softmax attention over the expanded block mask) -- outputs and the gradients of
+the input and of both projections.  This pins the head split, the q/k/v order of
+the projection and the merge of heads.
+GPU: the layer against the same steps spelled out with the binding (the same
+arithmetic: equal up to the GEMM library's choice of algorithm, checked at 1 %
+of the output's scale -- a wrong head split or q/k/v order is off by O(1)), and
+a backward that reaches every weight.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import workloads
+from block_sparse_attention_bigbird_b200 import bsa
+from block_sparse_attention_bigbird_b200.layer import BigBirdSelfAttention
+from oracle import attention as OA
+from oracle import backward as OB
+from oracle import layout as OL
+
+
+def _dense_reference(mod, x, lay, km):
+    B, L, C = x.shape
+    H = mod.num_heads
+    q, k, v = mod.qkv(x).view(B, L, 3, H, 64).permute(2, 0, 3, 1, 4).unbind(0)
+    s = (q @ k.transpose(-1, -2)) / math.sqrt(64)
+    allowed = torch.from_numpy(np.repeat(np.repeat(OL.block_mask(lay), 64, axis=1), 64, axis=2))  # [H, L, L]
+    allowed = allowed[None].expand(B, H, L, L)
+    if km is not None:
+        allowed = allowed & (torch.as_tensor(km) != 0)[:, None, None, :]
+    p = torch.softmax(s.masked_fill(~allowed, -math.inf), dim=-1)
+    o = (p @ v).transpose(1, 2).reshape(B, L, C)
+    return mod.proj(o)
+
+
+def test_layer_plumbing_with_fake_library(monkeypatch):
+    B, H, L = 2, 2, 64 * 5
+    w = workloads.custom(B, H, L, 1, 1, 1, seed=4, key_pad_tail=30)
+    lay = OL.build_layout(H, L, 64, w.window, w.n_global, w.n_random, w.seed)
+
+    class FakeLayout:
+        def __init__(self):
+            self.H, self.L = H, L
+
+    def fake_build(H_, L_, block, window, n_global, n_random, seed, globals=None):
+        assert (H_, L_, block, window, n_global, n_random, seed) == (H, L, 64, 1, 1, 1, 4)
+        return FakeLayout()
+
+    def fake_forward(q, k, v, layout, key_mask=None, scale=None):
+        o, lse = OA.attention(q, k, v, lay, key_mask=key_mask, scale=scale)
+        return torch.from_numpy(o), torch.from_numpy(lse)
+
+    def fake_backward(q, k, v, out, dout, lse, layout, key_mask=None, scale=None):
+        return tuple(torch.from_numpy(t) for t in OB.attention_backward(q, k, v, dout, lay, key_mask=key_mask,
+                                                                          scale=scale))
+
+    monkeypatch.setattr(bsa, "bsa_layout_build", fake_build)
+    monkeypatch.setattr(bsa, "bsa_layout_upload", lambda layout, stream=None: None)
+    monkeypatch.setattr(bsa, "bsa_forward", fake_forward)
+    monkeypatch.setattr(bsa, "bsa_backward", fake_backward)
+    torch.manual_seed(0)
+    mod = BigBirdSelfAttention(H * 64, H, window=1, num_global=1, num_random=1, seed=4).double()
+    ref = BigBirdSelfAttention(H * 64, H).double()
+    ref.load_state_dict(mod.state_dict())
+    km = workloads.make_key_mask(w).numpy()
+    x = torch.randn(B, L, H * 64, dtype=torch.float64, requires_grad=True)
+    x_ref = x.detach().clone().requires_grad_(True)
+    y = mod(x, key_mask=torch.from_numpy(km))
+    y_ref = _dense_reference(ref, x_ref, lay, km)
+    assert torch.allclose(y, y_ref, rtol=0, atol=1e-10)
+    g = torch.randn_like(y)
+    y.backward(g)
+    y_ref.backward(g)
+    assert torch.allclose(x.grad, x_ref.grad, rtol=0, atol=1e-9)
+    for (n, a), (_, b) in zip(mod.named_parameters(), ref.named_parameters()):
+        assert torch.allclose(a.grad, b.grad, rtol=0, atol=1e-8), n
+
+
+def test_layer_rejects_non_64_heads():
+    with pytest.raises(ValueError):
+        BigBirdSelfAttention(100, 2)
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+def test_layer_equals_its_steps_spelled_out():
+    B, H, L = 2, 4, 64 * 24
+    dev = torch.device("cuda")
+    torch.manual_seed(1)
+    mod = BigBirdSelfAttention(H * 64, H, window=1, num_global=2, num_random=2, seed=3).to(dev, torch.bfloat16)
+    x = torch.randn(B, L, H * 64, device=dev).to(torch.bfloat16).requires_grad_(True)
+    km = torch.ones(B, L, dtype=torch.uint8, device=dev)
+    km[1, -40:] = 0
+    y = mod(x, key_mask=km)
+    # the same steps with the binding
+    lay = bsa.bsa_layout_build(H, L, 64, 1, 2, 2, 3)
+    bsa.bsa_layout_upload(lay)
+    q, k, v = F.linear(x.detach(), mod.qkv.weight, mod.qkv.bias).view(B, L, 3, H, 64).permute(2, 0, 3, 1, 4).unbind(0)
+    o, _ = bsa.bsa_forward(q.contiguous(), k.contiguous(), v.contiguous(), lay, key_mask=km)
+    y2 = F.linear(o.transpose(1, 2).reshape(B, L, H * 64), mod.proj.weight, mod.proj.bias)
+    err = (y.detach().float() - y2.float()).abs().max().item()
+    assert err <= 1e-2 * y2.float().abs().max().item(), err
+    y.float().square().sum().backward()
+    assert bsa.bsa_sync_status() == 0
+    for t in (x.grad, mod.qkv.weight.grad, mod.qkv.bias.grad, mod.proj.weight.grad):
+        assert torch.isfinite(t.float()).all() and t.float().abs().sum() > 0
