@@ -279,11 +279,11 @@ void make_bwd_plan(int H, const std::vector<int32_t>& pair_q, int P, const std::
   plan->items.insert(plan->items.end(), whole.begin(), whole.end());
 }
 
-void build_tiles(bsa_layout* lay) {
+// dense[i]: 64-key query block i lists every key block in every head (it pairs
+// with other such blocks).
+void build_tiles(bsa_layout* lay, const std::vector<uint8_t>& dense) {
   const int nb = lay->nb, H = lay->H;
-  std::vector<uint8_t> is_global(static_cast<size_t>(nb), 0);
-  for (int g : lay->globals) is_global[static_cast<size_t>(g)] = 1;
-  make_tiles(H, nb, lay->row_ptr, lay->col_idx, is_global, &lay->pair_q, &lay->n_pairs, &lay->pair_ptr,
+  make_tiles(H, nb, lay->row_ptr, lay->col_idx, dense, &lay->pair_q, &lay->n_pairs, &lay->pair_ptr,
              &lay->pair_ent);
   const int P = lay->n_pairs;
   // Work items of one batch element: first the chunks of split tiles (the forward
@@ -346,6 +346,51 @@ void build_tiles(bsa_layout* lay) {
   make_bwd_plan(H, lay->ktiles.pair_q, lay->ktiles.n_pairs, lay->ktiles.pair_ptr, &lay->dkv_plan);
 }
 
+// Expands a CSR over blocks of 64 m keys (H x nbu rows, head-major, rows
+// ascending) to 64-key blocks: row (h, m I + t) lists m J + u, u = 0 .. m - 1, for
+// every J in row (h, I).  Attention restricted to (64 m)-blocks is exactly
+// attention restricted to these 64-blocks.  False if the result would not fit
+// int32 offsets.
+bool expand_csr(int H, int nbu, int m, const std::vector<int32_t>& rp, const std::vector<int32_t>& ci,
+                std::vector<int32_t>* rp64, std::vector<int32_t>* ci64) {
+  if (static_cast<int64_t>(ci.size()) * m * m > INT32_MAX) return false;
+  rp64->assign(1, 0);
+  ci64->clear();
+  ci64->reserve(ci.size() * static_cast<size_t>(m) * m);
+  for (int h = 0; h < H; ++h)
+    for (int I = 0; I < nbu; ++I) {
+      const size_t r = static_cast<size_t>(h) * nbu + I;
+      for (int t = 0; t < m; ++t) {
+        for (int32_t x = rp[r]; x < rp[r + 1]; ++x)
+          for (int u = 0; u < m; ++u) ci64->push_back(ci[static_cast<size_t>(x)] * m + u);
+        rp64->push_back(static_cast<int32_t>(ci64->size()));
+      }
+    }
+  return true;
+}
+
+// Stores a layout given in the caller's block units (rows ascending and
+// duplicate-free) at 64-key granularity, and builds its tiles.  dense_user[I]:
+// block I's row lists every block in every head.  False on int32 overflow.
+bool set_rows(bsa_layout* lay, std::vector<int32_t> urp, std::vector<int32_t> uci,
+              const std::vector<uint8_t>& dense_user) {
+  const int m = lay->block / bsa::kBlock, nbu = lay->L / lay->block;
+  std::vector<uint8_t> dense(static_cast<size_t>(lay->nb), 0);
+  for (int I = 0; I < nbu; ++I)
+    for (int u = 0; u < m; ++u) dense[static_cast<size_t>(I) * m + u] = dense_user[static_cast<size_t>(I)];
+  if (m == 1) {
+    lay->row_ptr = std::move(urp);
+    lay->col_idx = std::move(uci);
+  } else {
+    if (!expand_csr(lay->H, nbu, m, urp, uci, &lay->row_ptr, &lay->col_idx)) return false;
+    lay->user_row_ptr = std::move(urp);
+    lay->user_col_idx = std::move(uci);
+  }
+  build_tiles(lay, dense);
+  return lay->pair_ent.size() <= static_cast<size_t>(INT32_MAX) &&
+         lay->ktiles.pair_ent.size() <= static_cast<size_t>(INT32_MAX);
+}
+
 }  // namespace
 
 extern "C" {
@@ -354,11 +399,11 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
                      uint64_t seed, const int32_t* globals, bsa_layout** out) {
   if (out == nullptr) return BSA_ERR_INVALID_ARG;
   *out = nullptr;
-  if (block != bsa::kBlock) return BSA_ERR_UNSUPPORTED;
+  if (block < bsa::kBlock || block % bsa::kBlock != 0) return BSA_ERR_UNSUPPORTED;
   if (H < 1 || L < 1 || L % block != 0 || window < 0 || n_global < 0 || n_random < 0)
     return BSA_ERR_INVALID_ARG;
-  const int nb = L / block;
-  if (nb > static_cast<int>(bsa::kEntColMask) || static_cast<int64_t>(H) * nb > (1 << 30))
+  const int nb = L / block;  // the caller's blocks; the kernels run L / 64 blocks of 64
+  if (L / bsa::kBlock > static_cast<int>(bsa::kEntColMask) || static_cast<int64_t>(H) * (L / bsa::kBlock) > (1 << 30))
     return BSA_ERR_INVALID_ARG;
   bsa_layout* lay = new (std::nothrow) bsa_layout();
   if (lay == nullptr) return BSA_ERR_OOM;
@@ -366,7 +411,7 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
     lay->H = H;
     lay->L = L;
     lay->block = block;
-    lay->nb = nb;
+    lay->nb = L / bsa::kBlock;
     lay->window = window;
     lay->n_global = n_global;
     lay->n_random = n_random;
@@ -392,24 +437,22 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
     lay->globals = g;
     std::vector<uint8_t> is_global(static_cast<size_t>(nb), 0);
     for (int x : g) is_global[static_cast<size_t>(x)] = 1;
-    // CSR rows, head-major
-    lay->row_ptr.reserve(static_cast<size_t>(H) * nb + 1);
-    lay->row_ptr.push_back(0);
-    std::vector<int32_t> row;
+    // CSR rows in the caller's block units, head-major
+    std::vector<int32_t> urp, uci, row;
+    urp.reserve(static_cast<size_t>(H) * nb + 1);
+    urp.push_back(0);
     for (int h = 0; h < H; ++h) {
       for (int i = 0; i < nb; ++i) {
         build_row(h, i, nb, window, g, is_global, n_random, seed, &row);
-        lay->col_idx.insert(lay->col_idx.end(), row.begin(), row.end());
-        if (lay->col_idx.size() > static_cast<size_t>(INT32_MAX)) {
+        uci.insert(uci.end(), row.begin(), row.end());
+        if (uci.size() > static_cast<size_t>(INT32_MAX)) {
           delete lay;
           return BSA_ERR_INVALID_ARG;
         }
-        lay->row_ptr.push_back(static_cast<int32_t>(lay->col_idx.size()));
+        urp.push_back(static_cast<int32_t>(uci.size()));
       }
     }
-    build_tiles(lay);
-    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX) ||
-        lay->ktiles.pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
+    if (!set_rows(lay, std::move(urp), std::move(uci), is_global)) {
       delete lay;
       return BSA_ERR_INVALID_ARG;
     }
@@ -428,10 +471,10 @@ int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const i
                         bsa_layout** out) {
   if (out == nullptr) return BSA_ERR_INVALID_ARG;
   *out = nullptr;
-  if (block != bsa::kBlock) return BSA_ERR_UNSUPPORTED;
+  if (block < bsa::kBlock || block % bsa::kBlock != 0) return BSA_ERR_UNSUPPORTED;
   if (H < 1 || L < 1 || L % block != 0 || row_ptr == nullptr) return BSA_ERR_INVALID_ARG;
-  const int nb = L / block;
-  if (nb > static_cast<int>(bsa::kEntColMask) || static_cast<int64_t>(H) * nb > (1 << 30))
+  const int nb = L / block;  // the caller's blocks
+  if (L / bsa::kBlock > static_cast<int>(bsa::kEntColMask) || static_cast<int64_t>(H) * (L / bsa::kBlock) > (1 << 30))
     return BSA_ERR_INVALID_ARG;
   const size_t n_rows = static_cast<size_t>(H) * nb;
   // row_ptr: starts at 0, never decreases; col_idx may be NULL only if it is empty
@@ -448,23 +491,23 @@ int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const i
     lay->H = H;
     lay->L = L;
     lay->block = block;
-    lay->nb = nb;
+    lay->nb = L / bsa::kBlock;
     lay->window = -1;  // not a generated layout
     lay->n_random = -1;
     // rows sorted ascending and deduplicated
-    lay->row_ptr.reserve(n_rows + 1);
-    lay->row_ptr.push_back(0);
-    lay->col_idx.reserve(static_cast<size_t>(nnz_in));
-    std::vector<int32_t> row;
-    // dense[i]: query block i lists every key block in every head
+    std::vector<int32_t> urp, uci, row;
+    urp.reserve(n_rows + 1);
+    urp.push_back(0);
+    uci.reserve(static_cast<size_t>(nnz_in));
+    // dense[i]: block i lists every block in every head
     std::vector<uint8_t> dense(static_cast<size_t>(nb), 1);
     for (size_t x = 0; x < n_rows; ++x) {
       row.assign(col_idx + row_ptr[x], col_idx + row_ptr[x + 1]);
       std::sort(row.begin(), row.end());
       row.erase(std::unique(row.begin(), row.end()), row.end());
       if (static_cast<int>(row.size()) != nb) dense[x % static_cast<size_t>(nb)] = 0;
-      lay->col_idx.insert(lay->col_idx.end(), row.begin(), row.end());
-      lay->row_ptr.push_back(static_cast<int32_t>(lay->col_idx.size()));
+      uci.insert(uci.end(), row.begin(), row.end());
+      urp.push_back(static_cast<int32_t>(uci.size()));
     }
     // The dense query blocks play the part of BigBird's global blocks in the
     // pairing: they pair with each other, so that no sparse row is paired with a
@@ -472,9 +515,7 @@ int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const i
     for (int i = 0; i < nb; ++i)
       if (dense[static_cast<size_t>(i)]) lay->globals.push_back(i);
     lay->n_global = static_cast<int>(lay->globals.size());
-    build_tiles(lay);
-    if (lay->pair_ent.size() > static_cast<size_t>(INT32_MAX) ||
-        lay->ktiles.pair_ent.size() > static_cast<size_t>(INT32_MAX)) {
+    if (!set_rows(lay, std::move(urp), std::move(uci), dense)) {
       delete lay;
       return BSA_ERR_INVALID_ARG;
     }
@@ -492,10 +533,13 @@ int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const i
 int bsa_layout_csr(const bsa_layout* lay, const int32_t** row_ptr, const int32_t** col_idx,
                    int64_t* nnz, int* nb, int* H) {
   if (lay == nullptr) return BSA_ERR_INVALID_ARG;
-  if (row_ptr) *row_ptr = lay->row_ptr.data();
-  if (col_idx) *col_idx = lay->col_idx.data();
-  if (nnz) *nnz = static_cast<int64_t>(lay->col_idx.size());
-  if (nb) *nb = lay->nb;
+  const bool user = lay->block != bsa::kBlock;  // the caller's block units
+  const std::vector<int32_t>& rp = user ? lay->user_row_ptr : lay->row_ptr;
+  const std::vector<int32_t>& ci = user ? lay->user_col_idx : lay->col_idx;
+  if (row_ptr) *row_ptr = rp.data();
+  if (col_idx) *col_idx = ci.data();
+  if (nnz) *nnz = static_cast<int64_t>(ci.size());
+  if (nb) *nb = lay->L / lay->block;
   if (H) *H = lay->H;
   return BSA_OK;
 }
@@ -551,7 +595,7 @@ const char* bsa_strerror(int status) {
   switch (status) {
     case BSA_OK: return "success";
     case BSA_ERR_INVALID_ARG: return "invalid argument";
-    case BSA_ERR_UNSUPPORTED: return "unsupported configuration (block and head dim must be 64, device must be sm_100)";
+    case BSA_ERR_UNSUPPORTED: return "unsupported configuration (block must be a multiple of 64, head dim 64, device sm_100)";
     case BSA_ERR_CUDA: return "CUDA call failed";
     case BSA_ERR_LAYOUT_MISMATCH: return "layout does not match H/L or is not uploaded to the current device";
     case BSA_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";

@@ -80,12 +80,18 @@ constexpr int kEntBitsShift = 24;
 }  // namespace bsa
 
 struct bsa_layout {
+  // block: the caller's block size (a multiple of 64); nb: 64-key blocks, L / 64,
+  // the granularity every table below and every kernel works at
   int H = 0, L = 0, block = 0, nb = 0;
   int window = 0, n_global = 0, n_random = 0;
   uint64_t seed = 0;
-  std::vector<int32_t> globals;     // sorted, distinct
-  std::vector<int32_t> row_ptr;     // H*nb + 1
-  std::vector<int32_t> col_idx;     // nnz
+  std::vector<int32_t> globals;     // sorted, distinct, in the caller's block units
+  std::vector<int32_t> row_ptr;     // H*nb + 1 (64-key blocks)
+  std::vector<int32_t> col_idx;     // nnz (64-key blocks)
+  // the layout in the caller's block units when block > 64 (H*(L/block) + 1 and
+  // its columns); row (h, I) at block 64 m is rows (h, m I .. m I + m - 1) of
+  // the tables above, each listing blocks m J .. m J + m - 1 for J in row (h, I)
+  std::vector<int32_t> user_row_ptr, user_col_idx;
   std::vector<int32_t> pair_q;      // 2 * n_pairs
   int n_pairs = 0;
   std::vector<int32_t> pair_ptr;    // H*n_pairs + 1

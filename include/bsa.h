@@ -46,7 +46,8 @@ extern "C" {
 typedef enum {
   BSA_OK = 0,
   BSA_ERR_INVALID_ARG = -1,     /* null pointer, bad size or range            */
-  BSA_ERR_UNSUPPORTED = -2,     /* block != 64, d != 64, not an sm_100 device  */
+  BSA_ERR_UNSUPPORTED = -2,     /* block not a multiple of 64, d != 64, not an
+                                   sm_100 device                               */
   BSA_ERR_CUDA = -3,            /* a CUDA runtime/driver call failed           */
   BSA_ERR_LAYOUT_MISMATCH = -4, /* layout built for another H/L, or not uploaded
                                    to the current device                       */
@@ -84,9 +85,14 @@ typedef struct bsa_layout bsa_layout;
  *   Rows are sorted ascending and duplicate-free; the layout is shared by all
  *   batch elements.  CSR rows are ordered head-major then query block.
  *
- * block must be 64 (else BSA_ERR_UNSUPPORTED); L > 0 and L % block == 0;
- * H >= 1; window, n_global, n_random >= 0 (else BSA_ERR_INVALID_ARG).
- * On success *out receives a new layout.
+ * block must be a multiple of 64 (else BSA_ERR_UNSUPPORTED); L > 0 and
+ * L % block == 0; H >= 1; window, n_global, n_random >= 0 (else
+ * BSA_ERR_INVALID_ARG).  All of the above is in units of `block` (rows, window,
+ * globals, the random draws' counter i).  The kernels run 64-key blocks: a
+ * layout at block 64 m is expanded exactly, query block I's row becoming the
+ * rows of its m 64-blocks, each listing the m 64-blocks of every key block in it
+ * (the block size the pages leave to tuning, "Transformer计算效率优化：SQA稀疏注意力机制详解",
+ * 5 问题3).  On success *out receives a new layout.
  */
 int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_random,
                      uint64_t seed, const int32_t* globals, bsa_layout** out);
@@ -116,27 +122,32 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
  * ("Transformer计算效率优化：SQA稀疏注意力机制详解", 2.1), the others keeping a
  * local window.
  *
- * block must be 64 (else BSA_ERR_UNSUPPORTED).  BSA_ERR_INVALID_ARG for
- * H < 1, L < 1, L % block != 0, a NULL row_ptr, a bad row_ptr or a column
- * out of range.  The arrays are copied; the caller keeps ownership.
+ * block must be a multiple of 64 (else BSA_ERR_UNSUPPORTED); rows and
+ * columns are in units of `block` and expanded to 64-key blocks as in
+ * bsa_layout_build.  BSA_ERR_INVALID_ARG for H < 1, L < 1, L % block != 0, a
+ * NULL row_ptr, a bad row_ptr or a column out of range.  The arrays are copied;
+ * the caller keeps ownership.
  */
 int bsa_layout_from_csr(int H, int L, int block, const int32_t* row_ptr, const int32_t* col_idx,
                         bsa_layout** out);
 
 /*
- * bsa_layout_csr -- host views of the CSR: row_ptr has H*nb+1 int32 entries,
- * col_idx has nnz int32 entries (key block indices).  Any output pointer may be
- * NULL.  The views stay valid until bsa_layout_free.
+ * bsa_layout_csr -- host views of the CSR in the layout's block units
+ * (nb = L / block): row_ptr has H*nb+1 int32 entries, col_idx has nnz int32
+ * entries (key block indices).  Any output pointer may be NULL.  The views stay
+ * valid until bsa_layout_free.
  */
 int bsa_layout_csr(const bsa_layout* layout, const int32_t** row_ptr,
                    const int32_t** col_idx, int64_t* nnz, int* nb, int* H);
 
-/* bsa_layout_globals -- host view of the sorted global block list. */
+/* bsa_layout_globals -- host view of the sorted global block list, in the
+ * layout's block units. */
 int bsa_layout_globals(const bsa_layout* layout, const int32_t** globals, int* n_global);
 
 /*
  * bsa_layout_tiles -- host views of the 128-row tile decomposition the kernel
- * runs (two query blocks per tile over the union of their rows).
+ * runs (two 64-row query blocks per tile over the union of their rows; block
+ * indices here are always 64-key blocks).
  *   pair_q:   2*n_pairs int32, (first, second) query block; second = -1 when the
  *             tile holds a single block.  Global blocks pair with global blocks.
  *   pair_ptr: H*n_pairs+1 int32 offsets into pair_ent, head-major.

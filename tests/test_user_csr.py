@@ -134,7 +134,8 @@ def test_rejects_bad_csr():
     good_rp = np.array([0, 1, 2, 3, 4], dtype=np.int32)
     good_ci = np.array([0, 1, 2, 3], dtype=np.int32)
     assert _raw_from_csr(1, 64 * nb, 64, good_rp, good_ci) == bsa.BSA_OK
-    assert _raw_from_csr(1, 64 * nb, 128, good_rp, good_ci) == bsa.BSA_ERR_UNSUPPORTED
+    assert _raw_from_csr(1, 64 * nb, 96, good_rp, good_ci) == bsa.BSA_ERR_UNSUPPORTED
+    assert _raw_from_csr(1, 64 * nb, 32, good_rp, good_ci) == bsa.BSA_ERR_UNSUPPORTED
     assert _raw_from_csr(0, 64 * nb, 64, good_rp, good_ci) == bsa.BSA_ERR_INVALID_ARG
     assert _raw_from_csr(1, 64 * nb + 3, 64, good_rp, good_ci) == bsa.BSA_ERR_INVALID_ARG
     assert _raw_from_csr(1, 64 * nb, 64, None, good_ci) == bsa.BSA_ERR_INVALID_ARG
