@@ -24,19 +24,22 @@ from .autograd import block_sparse_attention
 class BigBirdSelfAttention(torch.nn.Module):
     """x [B, L, dim] -> [B, L, dim] with ``num_heads`` heads of 64.
 
-    window, num_global, num_random and seed define the BigBird layout of each
-    sequence length (see bsa_layout_build); it is built and uploaded on first
-    use per (length, device).  ``key_mask`` in forward is uint8 [B, L], 1 = keep.
+    block (a multiple of 64), window, num_global, num_random and seed define the
+    BigBird layout of each sequence length (see bsa_layout_build); it is built
+    and uploaded on first use per (length, device).  ``key_mask`` in forward is
+    uint8 [B, L], 1 = keep.
     """
 
     HEAD_DIM = 64
 
     def __init__(self, dim: int, num_heads: int, window: int = 1, num_global: int = 2, num_random: int = 3,
-                 seed: int = 0, bias: bool = True, out_proj: bool = True):
+                 seed: int = 0, bias: bool = True, out_proj: bool = True, block: int = 64):
         super().__init__()
         if dim != num_heads * self.HEAD_DIM:
             raise ValueError(f"dim must be num_heads * {self.HEAD_DIM}")
-        self.num_heads = num_heads
+        if block < 64 or block % 64:
+            raise ValueError("block must be a multiple of 64")
+        self.num_heads, self.block = num_heads, block
         self.window, self.num_global, self.num_random, self.seed = window, num_global, num_random, seed
         self.qkv = torch.nn.Linear(dim, 3 * dim, bias=bias)
         self.proj = torch.nn.Linear(dim, dim, bias=bias) if out_proj else None
@@ -46,8 +49,8 @@ class BigBirdSelfAttention(torch.nn.Module):
         key = (L, str(device))
         lay = self._layouts.get(key)
         if lay is None:
-            lay = bsa.bsa_layout_build(self.num_heads, L, 64, self.window, self.num_global, self.num_random,
-                                       self.seed)
+            lay = bsa.bsa_layout_build(self.num_heads, L, self.block, self.window, self.num_global,
+                                       self.num_random, self.seed)
             bsa.bsa_layout_upload(lay)
             self._layouts[key] = lay
         return lay

@@ -83,9 +83,11 @@ def test_layer_plumbing_with_fake_library(monkeypatch):
         assert torch.allclose(a.grad, b.grad, rtol=0, atol=1e-8), n
 
 
-def test_layer_rejects_non_64_heads():
+def test_layer_rejects_non_64_heads_and_blocks():
     with pytest.raises(ValueError):
         BigBirdSelfAttention(100, 2)
+    with pytest.raises(ValueError):
+        BigBirdSelfAttention(128, 2, block=96)
 
 
 @pytest.mark.gpu
