@@ -226,7 +226,7 @@ def _workspace(layout: Layout, B: int, device):
     key = (str(device), B)
     ws = layout._workspaces.get(key)
     if ws is None:
-        ws = torch.zeros(bsa_workspace_bytes(layout, B), dtype=torch.uint8, device=device)
+        ws = torch.empty(bsa_workspace_bytes(layout, B), dtype=torch.uint8, device=device)
         layout._workspaces[key] = ws
     return ws
 
@@ -236,8 +236,8 @@ def bsa_forward(q, k, v, layout: Layout, key_mask=None, scale: Optional[float] =
     """O (bf16 [B,H,L,64]) and lse (fp32 [B,H,L]) of the block-sparse attention.
 
     q, k, v: contiguous bf16 CUDA tensors [B, H, L, 64].  key_mask: optional
-    uint8 CUDA tensor [B, L] (1 = keep).  workspace: optional zero-initialised
-    uint8 CUDA tensor of at least bsa_workspace_bytes(layout, B) bytes; when
+    uint8 CUDA tensor [B, L] (1 = keep).  workspace: optional uint8 CUDA tensor
+    of at least bsa_workspace_bytes(layout, B) bytes, any contents; when
     omitted a cached one of the layout is used (not safe for concurrent calls
     on different streams with the same layout).
     """

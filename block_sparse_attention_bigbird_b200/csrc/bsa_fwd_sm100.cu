@@ -8,33 +8,35 @@
 // per-tile list of 64-key blocks ("SQA 稀疏注意力机制详解" 3.1: block-sparse mask,
 // attention only on non-zero blocks).
 //
-// Kernel design: one persistent CTA per SM (448 threads) running two independent
-// pipelines ("slots") side by side, each with its own work items, shared-memory
-// rings, barriers and 256 TMEM columns.  The ex2 unit (16 results per clock per
-// SM) bounds this d = 64 forward; with two slots one softmax warpgroup runs its
-// exponentials while the other is between chunks, so their phases interleave
-// instead of running in lockstep.  Slot s (0 or 1) has:
-//   warps 4s..4s+3  softmax + epilogue: thread (warp w, lane l) owns tile row
-//               r = 32 (w % 4) + l = TMEM lane r, keeps the running max m and sum l
-//               (fp32), writes P (bf16) over the S columns it has read, and raises
-//               m (rescaling l and O) only when a chunk's p would outgrow 2^12.
-//   warp 8+s    TMA producer: Q tile (2 x 64 rows), then K and V of one key block per
-//               chunk of the tile's key-block union into a K ring (released when the
-//               chunk's S is done) and a deeper V ring (released after its PV).
-//   warp 10+2s  tcgen05 S issuer: S = Q K^T (M=128, N=64, K=64) into one of three
-//               TMEM S buffers (warp 10 also allocates and frees TMEM).
-//   warp 11+2s  tcgen05 PV issuer: O += P V (A = P from TMEM, M=128, N=64, K=64).
-//               Two issuing threads per slot keep the tensor pipe fed: each tcgen05
-//               instruction, barrier wait and commit blocks its thread, and d = 64
-//               makes every MMA short.
-// A tile is two query blocks of the same (b, h) over the sorted union of their rows;
-// entries carry per-block membership bits so each half of the tile sees exactly its
-// own row, and a warp whose half does not attend a block skips its exponentials.
-// Long unions (global rows) are cut into chunks run as separate work items; each
-// stores a partial (O, m, l) record, and bsa_merge_kernel, launched after the
-// forward, merges a split tile's records into its output rows.
-// Every wait is bounded (globaltimer); on expiry the CTA records
-// BSA_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+// Kernel design: one persistent CTA per SM (512 threads, four warpgroups) running two
+// independent pipelines ("slots"), each with its own work items, shared-memory rings,
+// barriers and 256 TMEM columns: O (64), S (128) and P (64, bf16 pairs).  A tile is two
+// 64-row query blocks of the same (b, h) over the union of their key-block lists; a
+// chunk is two consecutive union entries (128 keys).
+//   warps 0-3 / 4-7  softmax of slot 0 / 1 (thread r of the slot owns tile row r =
+//               TMEM lane r).  Per chunk: load all of S(g) into registers and hand the S
+//               columns straight back, so S(g + 1) runs during these exponentials; chunk
+//               max on the ALU; p = 2^(s * scale * log2 e - m) on the ex2 unit; P (bf16)
+//               into the P columns once PV(g - 1) has read them.  The running max m is
+//               raised only when a chunk's max exceeds it by more than 2^8 (then l and O
+//               are rescaled), so p <= 2^8.  A finished tile's epilogue runs in the next
+//               tile's first chunk.
+//   warp 8 + s  K producer of slot s: stages the slot's work items; TMA loads of the Q tile
+//               and of K, the chunk's two 64-key blocks per 16 KB stage, 2 stages.
+//   warp 14 + s V producer of slot s: TMA loads of V into 2 stages of 16 KB.
+//   warp 10 + s tcgen05 S issuer: S(g) = Q K_g^T (M=128, N=128, or 64 for a lone entry).
+//   warp 12 + s tcgen05 PV issuer: O (+)= P(g) V_g (A = P from TMEM, 16 keys per MMA).
+// A tcgen05.mma holds its issuing warp for ~120 cycles, and a TMA load's issue waits on
+// its stage; a role per warp keeps these latencies off each other's paths.  Every
+// per-chunk hand-off costs the softmax warps a few hundred cycles of latency, so a chunk
+// spans 128 keys to spread that cost over 128 exponentials per thread.
+// Entries carry per-block membership bits so each half of the tile sees exactly its own
+// row; a warp whose half does not attend a block gives it zero P without exponentials.
+// Long unions (global rows) are cut into chunks run as separate work items; each stores
+// a partial (O, m, l) record, and bsa_merge_kernel, launched after the forward, merges a
+// split tile's records into its output rows.
+// Every wait is bounded (globaltimer); on expiry the CTA records BSA_ERR_DEVICE_TIMEOUT,
+// drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -52,48 +54,57 @@
 namespace bsa {
 
 constexpr int kSlots = 2;
-constexpr int kProducerWarp = 8;  // + slot
-constexpr int kMmaWarp = 10;      // + 2 slot: S issuer; warp 10 allocates and frees TMEM
-constexpr int kPvWarp = 11;       // + 2 slot
-constexpr int kThreads = 448;
-constexpr int kSoftmaxThreads = 128;  // per slot
-constexpr int kItemRing = 4;  // work-item indices a slot's producer may publish ahead
-constexpr int kKStages = 3;  // == kSBufs: K stage g % 3 is free once S(g) is done
-constexpr int kVStages = 4;  // V stage g % 4 is free once PV(g) is done
-constexpr uint32_t kBlkBytes = 64 * 128;     // one 64 x 64 bf16 block
-constexpr uint32_t kQBytes = 2 * kBlkBytes;  // 128-row Q tile
+constexpr int kThreads = 512;
+constexpr int kKProdWarp = 8;  // + slot
+constexpr int kSWarp = 10;     // + slot; warp 10 allocates and frees TMEM
+constexpr int kPvWarp = 12;    // + slot
+constexpr int kVProdWarp = 14;  // + slot
+// Register split: softmax warpgroups 0-1 take kSoftmaxRegs, warpgroups 2-3 (producers
+// and issuers) kOtherRegs; 2 * 128 * (200 + 56) = 65536 = 512 threads x 128.
+constexpr uint32_t kSoftmaxRegs = 200;
+constexpr uint32_t kOtherRegs = 56;
+static_assert(2 * 128 * (kSoftmaxRegs + kOtherRegs) <= 65536, "register split exceeds the launch budget");
+constexpr int kItemRing = 4;  // work items a slot's K producer may publish ahead
+constexpr int kChunkEnt = 2;  // union entries (64-key blocks) per chunk
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
+constexpr uint32_t kBlkBytes = 64 * 128;                 // one 64 x 64 bf16 block
+constexpr uint32_t kQBytes = 2 * kBlkBytes;              // 128-row Q tile
+constexpr uint32_t kStageBytes = kChunkEnt * kBlkBytes;  // one chunk of K (or V)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSlotCols = 256;          // slot s owns columns [256 s, 256 s + 256)
-constexpr uint32_t kSBufs = 3;               // S buffers of 64 columns at +0, +64, +128
-constexpr uint32_t kTmemS = 0;
-constexpr uint32_t kTmemO = 192;             // O at +192
-constexpr float kLazyBound = 4096.0f;  // 2^kLazyLog2, kLazyLog2 = 12: bound on a chunk's sum of p
+constexpr uint32_t kSlotCols = 256;  // slot s owns columns [256 s, 256 s + 256)
+constexpr uint32_t kTmemO = 0;       // O: 64 fp32 columns
+constexpr uint32_t kTmemS = 64;      // S: 128 fp32 columns
+constexpr uint32_t kTmemP = 192;     // P: 128 keys as 64 bf16 pairs
+constexpr float kRescaleLog2 = 8.0f;  // m is raised when a chunk's max exceeds it by more
+constexpr uint32_t kOStageBytes = 32 * 128;  // one warp's 32 O rows, staged for a TMA store
+static_assert(kTmemS + 128 <= kTmemP && kTmemP + 64 <= kSlotCols, "TMEM map");
 
 // shared memory map of one slot (offsets from its 1024-aligned base)
-constexpr uint32_t kSmemQ = 0;
+constexpr uint32_t kSmemQ = 0;  // 2 Q tiles; a finished tile's buffer also stages its O
 constexpr uint32_t kSmemK = kSmemQ + 2 * kQBytes;
-constexpr uint32_t kSmemV = kSmemK + kKStages * kBlkBytes;
-constexpr uint32_t kSmemOStage = kSmemV + kVStages * kBlkBytes;  // 4 x (32 rows x 128 B) O staging
-constexpr uint32_t kOStageBytes = 32 * 128;
-constexpr uint32_t kSmemBar = kSmemOStage + 4 * kOStageBytes;
+constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
+constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
 enum : int {
-  kBarQFull = 0,
-  kBarQEmpty = 2,
-  kBarKFull = 4,                          // [K stage] K of the stage landed (TMA)
-  kBarVFull = kBarKFull + kKStages,       // [V stage] V of the stage landed (TMA)
-  kBarVFree = kBarVFull + kVStages,       // [V stage] MMA commit after the chunk's PV: the V
-                                          // stage is reusable and O holds that chunk
-  kBarSFull = kBarVFree + kVStages,       // [S buffer] MMA commit after S: S readable, and
-                                          // the K stage of the same index reusable
-  kBarPFull = kBarSFull + kSBufs,         // [S buffer] P written, 128 arrivals
-  kBarOFree = kBarPFull + kSBufs,         // 128 arrivals once the epilogue has read O
-  kBarMmaFinal = kBarOFree + 1,           // [2 issuers]
-  kBarItemFull = kBarMmaFinal + 2,             // [item ring] the producer published a work item
-  kBarItemEmpty = kBarItemFull + kItemRing,  // [item ring] 6 arrivals: both issuers and the
-                                             // four softmax warps have read it
+  kBarQFull = 0,                     // [Q stage] the tile's Q landed (TMA)
+  kBarQEmpty = kBarQFull + 2,        // [Q stage] 4 softmax warps: the tile's S MMAs and its
+                                     // O staging are done with the buffer
+  kBarKFull = kBarQEmpty + 2,        // [K stage] K of the chunk landed (TMA)
+  kBarKFree = kBarKFull + kKStages,  // [K stage] MMA commit after the chunk's S
+  kBarVFull = kBarKFree + kKStages,  // [V stage] V of the chunk landed (TMA)
+  kBarVFree = kBarVFull + kVStages,  // [V stage] MMA commit after the chunk's PV: the V stage
+                                     // and the P columns are reusable, O holds chunk g
+  kBarSFull = kBarVFree + kVStages,  // MMA commit after S: the S columns are readable
+  kBarSFree = kBarSFull + 1,         // 4 softmax warps have loaded S
+  kBarPFull = kBarSFree + 1,         // 4 softmax warps have stored P
+  kBarMmaFinal = kBarPFull + 1,      // [2 issuers]
+  kBarItemFull = kBarMmaFinal + 2,   // [item ring] the K producer published a work item
+  kBarItemEmpty = kBarItemFull + kItemRing,  // [item ring] 7 arrivals: V producer, both
+                                             // issuers, the four softmax warps
   kNumBars = kBarItemEmpty + kItemRing
 };
-constexpr uint32_t kItemReaders = 6;
+constexpr uint32_t kItemReaders = 7;
+constexpr uint32_t kWarpArrivals = 4;  // barriers the four softmax warps arrive on once each
 
 // One published work item in shared memory: its index, its fields, its query-block
 // pair and, per union entry, the entry and the key-padding bits of its key block.
@@ -112,20 +123,20 @@ struct ItemStage {
 static_assert(sizeof(ItemStage) % 16 == 0, "stage alignment");
 constexpr uint32_t kSmemItems = (kSmemBar + 8 * kNumBars + 15) & ~15u;  // ItemStage[kItemRing]
 constexpr uint32_t kSlotBytes = (kSmemItems + sizeof(ItemStage) * kItemRing + 1023) & ~1023u;
-constexpr uint32_t kSmemMisc = kSlots * kSlotBytes;          // u32 TMEM base, int abort flag
+constexpr uint32_t kSmemMisc = kSlots * kSlotBytes;  // u32 TMEM base, int abort flag
 constexpr uint32_t kSmemUsed = kSmemMisc + 16;
 constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // slack for 1024-byte alignment
 static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+static_assert(kQBytes == 4 * kOStageBytes, "a Q buffer stages the four warps' O rows");
 
 // Where one slot's roles find their resources.  Work items are handed out
-// dynamically: the slot's producer takes the next index from a global counter and
+// dynamically: the slot's K producer takes the next index from a global counter and
 // publishes it to the slot's other roles through a small ring in shared memory.
 struct Slot {
   uint32_t sQ, sK, sV, bars;
-  uint8_t* ostage;   // O staging of softmax warp w at ostage + (w % 4) * kOStageBytes
-  uint32_t sO;       // its shared-memory address
-  ItemStage* items;  // the item ring
-  uint32_t tmem;  // TMEM address of the slot's column 0
+  uint8_t* q_generic;  // generic pointer to the Q buffers (O staging)
+  ItemStage* items;    // the item ring
+  uint32_t tmem;       // TMEM address of the slot's column 0
 };
 
 struct FwdParams {
@@ -138,7 +149,7 @@ struct FwdParams {
   const uint32_t* pair_ent;
   const unsigned long long* keybits;  // [B, nb] or null
   float* partials;
-  int* sched;    // [0] next work item, [1] slots finished; zero between calls
+  int* sched;  // [0] next work item, [1] slots finished; cleared before each launch
   int B, H, L, nb, items_per_batch, n_split, n_records;
   int split_items;  // the first split_items items of a batch element are split-tile chunks
   float scale_log2;
@@ -148,49 +159,62 @@ struct FwdParams {
 constexpr int kItemNone = -1;   // no work left
 constexpr int kItemAbort = -2;  // a wait gave up
 
+__device__ __forceinline__ uint32_t bar_at(uint32_t bars, int i) { return bars + 8u * static_cast<uint32_t>(i); }
+
 // The slot's k-th work item for an issuer (one thread): its index and entry count.
 // The stage is released at once.
 __device__ __forceinline__ int take_item_one(const Slot& sl, uint32_t k, int* count, volatile int* abort_flag,
                                              uint64_t timeout_ns) {
   const uint32_t i = k % kItemRing;
-  if (!wait_one(sl.bars + 8u * (kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
+  if (!wait_one<2>(bar_at(sl.bars, kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
     return kItemAbort;
   const ItemStage& st = sl.items[i];
   const int t = st.t;
   *count = st.w.count;
-  ptx::mbar_arrive(sl.bars + 8u * (kBarItemEmpty + i));
+  ptx::mbar_arrive(bar_at(sl.bars, kBarItemEmpty + i));
   return t;
 }
 
-// The slot's k-th work item for a softmax warp, which keeps reading its stage until
-// the item's epilogue and then releases it (release_item_warp).
+// The slot's k-th work item for a warp that keeps reading its stage (the V producer
+// until its last load, a softmax warp until the item's epilogue); released with
+// release_item_warp.
+template <int kRegion>
 __device__ __forceinline__ int take_item_warp(const Slot& sl, uint32_t k, volatile int* abort_flag,
                                               uint64_t timeout_ns) {
   const uint32_t i = k % kItemRing;
-  if (!wait_warp(sl.bars + 8u * (kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
+  if (!wait_warp<kRegion>(bar_at(sl.bars, kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
     return kItemAbort;
   return sl.items[i].t;
 }
 
 __device__ __forceinline__ void release_item_warp(const Slot& sl, uint32_t k, int lane) {
   __syncwarp();
-  if (lane == 0) ptx::mbar_arrive(sl.bars + 8u * (kBarItemEmpty + k % kItemRing));
+  if (lane == 0) ptx::mbar_arrive(bar_at(sl.bars, kBarItemEmpty + k % kItemRing));
 }
 
-// TMA producer, one warp.  Per work item the warp stages the item, its union
-// entries and their key-padding bits in the slot's item ring; then lane 0 issues
-// the loads: the Q tile, and for each chunk g (one key block) its K into K stage
-// g % 3 (once S(g - 3) is done) and its V into V stage g % 5 (once PV(g - 5) is
-// done).
-__device__ __forceinline__ void producer_role(const FwdParams& p, const Slot& sl, int lane,
-                                              volatile int* abort_flag) {
-  const uint32_t sQ = sl.sQ, sK = sl.sK, sV = sl.sV, bars = sl.bars;
-  static_assert(kKStages == static_cast<int>(kSBufs), "K stages are released by the S-full commits");
-  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+// Lets every copy a producer thread issued land before the CTA exits (after an abort):
+// the last issue into ring slot s of n issues had index s + R * floor((n - 1 - s) / R).
+__device__ __forceinline__ void drain_ring(uint32_t bars, int first_bar, uint32_t n, uint32_t ring,
+                                           volatile int* abort_flag, uint64_t timeout_ns) {
+  for (uint32_t s = 0; s < ring; ++s) {
+    if (n > s) {
+      const uint32_t last = s + ring * ((n - 1u - s) / ring);
+      wait_force<2>(bar_at(bars, first_bar + static_cast<int>(s)), (last / ring) & 1u, abort_flag, timeout_ns);
+    }
+  }
+}
+
+// K producer, one warp.  Per work item the warp stages the item, its union entries and
+// their key-padding bits in the slot's item ring; then lane 0 issues the loads: the Q
+// tile into Q buffer (tile % 2) once the tile two back has released it, and for each
+// chunk g its K blocks into K stage g % 2 once S(g - 2) is done.
+__device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, int lane, volatile int* abort_flag) {
+  const uint32_t sQ = sl.sQ, sK = sl.sK, bars = sl.bars;
+  auto bar = [&](int i) { return bar_at(bars, i); };
   const uint64_t pol_q = ptx::policy_evict_first();
   const uint64_t pol_kv = ptx::policy_evict_last();
   const int total = p.B * p.items_per_batch;
-  uint32_t nq = 0, nk = 0, nv = 0;  // Q tiles, K blocks, V blocks issued (lane 0)
+  uint32_t nq = 0, nk = 0;  // Q tiles and K blocks issued (lane 0)
   bool alive = true;
   int t_next = lane == 0 ? atomicAdd(p.sched, 1) : 0;
   for (uint32_t k = 0;; ++k) {
@@ -199,8 +223,8 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const Slot& sl
     const uint32_t ii = k % kItemRing;
     bool ok = true;
     if (lane == 0)
-      ok = wait_one(bar(kBarItemEmpty + static_cast<int>(ii)), ((k / kItemRing) & 1u) ^ 1u, abort_flag,
-                    p.timeout_ns);
+      ok = wait_one<2>(bar(kBarItemEmpty + static_cast<int>(ii)), ((k / kItemRing) & 1u) ^ 1u, abort_flag,
+                          p.timeout_ns);
     if (!__shfl_sync(0xffffffffu, ok, 0)) {
       alive = false;
       break;
@@ -245,7 +269,7 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const Slot& sl
       const int row0 = (st.b * p.H + w.h) * p.L;
       const int qa = st.qa, qb = st.qb;
       const uint32_t qs = nq & 1u;
-      if (!wait_one(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+      if (!wait_one<2>(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
         alive = false;
       } else {
         ptx::mbar_arrive_expect_tx(bar(kBarQFull + qs), kQBytes);
@@ -253,24 +277,18 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const Slot& sl
         ptx::tma_load_2d(sQ + qs * kQBytes + kBlkBytes, &p.tm_q, bar(kBarQFull + qs), 0,
                          row0 + (qb >= 0 ? qb : qa) * 64, pol_q);
         ++nq;
-        for (int e = 0; e < w.count; ++e) {
-          const int j = static_cast<int>(st.ent[e] & kEntColMask);
+        for (int e0 = 0; e0 < w.count; e0 += kChunkEnt) {
+          const int ne = min(kChunkEnt, w.count - e0);
           const uint32_t ks = nk % kKStages;
-          if (!wait_one(bar(kBarSFull + ks), ((nk / kKStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+          if (!wait_one<2>(bar(kBarKFree + ks), ((nk / kKStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
             alive = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(bar(kBarKFull + ks), kBlkBytes);
-          ptx::tma_load_2d(sK + ks * kBlkBytes, &p.tm_k, bar(kBarKFull + ks), 0, row0 + j * 64, pol_kv);
+          ptx::mbar_arrive_expect_tx(bar(kBarKFull + ks), kBlkBytes * ne);
+          for (int x = 0; x < ne; ++x)
+            ptx::tma_load_2d(sK + ks * kStageBytes + x * kBlkBytes, &p.tm_k, bar(kBarKFull + ks), 0,
+                             row0 + static_cast<int>(st.ent[e0 + x] & kEntColMask) * 64, pol_kv);
           ++nk;
-          const uint32_t vs = nv % kVStages;
-          if (!wait_one(bar(kBarVFree + vs), ((nv / kVStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
-            alive = false;
-            break;
-          }
-          ptx::mbar_arrive_expect_tx(bar(kBarVFull + vs), kBlkBytes);
-          ptx::tma_load_2d(sV + vs * kBlkBytes, &p.tm_v, bar(kBarVFull + vs), 0, row0 + j * 64, pol_kv);
-          ++nv;
         }
       }
     }
@@ -281,37 +299,64 @@ __device__ __forceinline__ void producer_role(const FwdParams& p, const Slot& sl
   }
   if (lane != 0) return;
   if (alive) {
-    // Every slot's producer counts itself out once it has drawn its last index; the
-    // last one resets both counters for the next call.
+    // Every slot's K producer counts itself out once it has drawn its last index; the
+    // last one resets both counters, so the workspace is left as the call found it.
     __threadfence();
     if (atomicAdd(p.sched + 1, 1) == kSlots * static_cast<int>(gridDim.x) - 1) {
       p.sched[0] = 0;
       p.sched[1] = 0;
     }
   } else {
-    // Aborted: let every copy this thread issued land before the CTA exits.  The
-    // last issue into ring slot s had index s + R * floor((n - 1 - s) / R).
-    auto drain = [&](int first_bar, uint32_t n, uint32_t ring) {
-      for (uint32_t s = 0; s < ring; ++s) {
-        if (n > s) {
-          const uint32_t last = s + ring * ((n - 1u - s) / ring);
-          wait_force(bar(first_bar + static_cast<int>(s)), (last / ring) & 1u, abort_flag, p.timeout_ns);
-        }
-      }
-    };
-    drain(kBarQFull, nq, 2u);
-    drain(kBarKFull, nk, static_cast<uint32_t>(kKStages));
-    drain(kBarVFull, nv, static_cast<uint32_t>(kVStages));
+    drain_ring(bars, kBarQFull, nq, 2u, abort_flag, p.timeout_ns);
+    drain_ring(bars, kBarKFull, nk, static_cast<uint32_t>(kKStages), abort_flag, p.timeout_ns);
   }
 }
 
-// tcgen05 S issuer, one thread.  S(g) = Q K_g^T into S buffer g % 3 once K(g) has
-// landed and PV(g - 3), the previous reader of that buffer, is done.  Its commit
-// also releases K stage g % 3 to the producer.
+// V producer, one warp: follows the item ring and loads V of chunk g into V stage
+// g % 2 once PV(g - 2) is done, releasing each item after its last load.
+__device__ __forceinline__ void v_producer(const FwdParams& p, const Slot& sl, int lane, volatile int* abort_flag) {
+  const uint32_t sV = sl.sV, bars = sl.bars;
+  auto bar = [&](int i) { return bar_at(bars, i); };
+  const uint64_t pol_kv = ptx::policy_evict_last();
+  uint32_t nv = 0;
+  bool alive = true;
+  for (uint32_t k = 0; alive; ++k) {
+    const int t = take_item_warp<2>(sl, k, abort_flag, p.timeout_ns);
+    if (t < 0) {
+      if (t == kItemAbort) alive = false;
+      break;
+    }
+    const ItemStage& st = sl.items[k % kItemRing];
+    if (lane == 0) {
+      const int row0 = (st.b * p.H + st.w.h) * p.L;
+      for (int e0 = 0; e0 < st.w.count; e0 += kChunkEnt) {
+        const int ne = min(kChunkEnt, st.w.count - e0);
+        const uint32_t vs = nv % kVStages;
+        if (!wait_one<2>(bar(kBarVFree + vs), ((nv / kVStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+          alive = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(bar(kBarVFull + vs), kBlkBytes * ne);
+        for (int x = 0; x < ne; ++x)
+          ptx::tma_load_2d(sV + vs * kStageBytes + x * kBlkBytes, &p.tm_v, bar(kBarVFull + vs), 0,
+                           row0 + static_cast<int>(st.ent[e0 + x] & kEntColMask) * 64, pol_kv);
+        ++nv;
+      }
+    }
+    alive = __shfl_sync(0xffffffffu, alive, 0);
+    release_item_warp(sl, k, lane);
+  }
+  if (lane == 0 && !alive) drain_ring(bars, kBarVFull, nv, static_cast<uint32_t>(kVStages), abort_flag, p.timeout_ns);
+}
+
+// tcgen05 S issuer, one thread.  S(g) = Q K_g^T (N = 64 per key block of the chunk) into
+// the S columns once K(g) has landed and the softmax has loaded S(g - 1).  Its commits
+// signal S full and release K stage g % 2.
 __device__ __forceinline__ void s_issuer(const FwdParams& p, const Slot& sl, volatile int* abort_flag) {
   const uint32_t sQ = sl.sQ, sK = sl.sK, bars = sl.bars, tmem = sl.tmem;
-  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
-  constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 64, false);
+  auto bar = [&](int i) { return bar_at(bars, i); };
+  constexpr uint32_t kIdescS2 = ptx::idesc_bf16_f32(128, 128, false);
+  constexpr uint32_t kIdescS1 = ptx::idesc_bf16_f32(128, 64, false);
   // descriptor start-address fields count 16-byte units
   const uint64_t dq0 = ptx::smem_desc_sw128(sQ, 16);
   const uint64_t dk0 = ptx::smem_desc_sw128(sK, 16);
@@ -321,113 +366,94 @@ __device__ __forceinline__ void s_issuer(const FwdParams& p, const Slot& sl, vol
     int count = 0;
     if (take_item_one(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
     const uint32_t qs = nq & 1u;
-    if (!wait_one(bar(kBarQFull + qs), (nq >> 1) & 1u, abort_flag, p.timeout_ns)) break;
+    if (!wait_one<2>(bar(kBarQFull + qs), (nq >> 1) & 1u, abort_flag, p.timeout_ns)) break;
     const uint64_t dq = dq0 + qs * (kQBytes >> 4);
-    for (int n = 0; n < count; ++n, ++g) {
+    for (int e0 = 0; e0 < count; e0 += kChunkEnt, ++g) {
       const uint32_t ks = g % kKStages;
-      if (!wait_one(bar(kBarKFull + ks), (g / kKStages) & 1u, abort_flag, p.timeout_ns)) {
+      if (!wait_one<2>(bar(kBarKFull + ks), (g / kKStages) & 1u, abort_flag, p.timeout_ns) ||
+          (g > 0 && !wait_one<2>(bar(kBarSFree), (g - 1u) & 1u, abort_flag, p.timeout_ns))) {
         alive = false;
         break;
       }
-      if (g >= kSBufs) {
-        const uint32_t gp = g - kSBufs;
-        if (!wait_one(bar(kBarVFree + gp % kVStages), (gp / kVStages) & 1u, abort_flag, p.timeout_ns)) {
-          alive = false;
-          break;
-        }
-      }
       ptx::tc_fence_after();
-      const uint64_t dk = dk0 + ks * (kBlkBytes >> 4);
-      const uint32_t d = tmem + kTmemS + (g % kSBufs) * 64u;
-      ptx::mma_ss(d, dq, dk, kIdescS, 0u);  // head dim 64 = 4 x 16: +32 bytes per step
-      ptx::mma_ss(d, dq + 2, dk + 2, kIdescS, 1u);
-      ptx::mma_ss(d, dq + 4, dk + 4, kIdescS, 1u);
-      ptx::mma_ss(d, dq + 6, dk + 6, kIdescS, 1u);
-      ptx::mma_commit(bar(kBarSFull + g % kSBufs));
-      if (n == count - 1) ptx::mma_commit(bar(kBarQEmpty + qs));
+      const uint64_t dk = dk0 + ks * (kStageBytes >> 4);
+      const uint32_t d = tmem + kTmemS;
+      const uint32_t idesc = count - e0 >= 2 ? kIdescS2 : kIdescS1;
+      ptx::mma_ss(d, dq, dk, idesc, 0u);  // head dim 64 = 4 x 16: +32 bytes per step
+      ptx::mma_ss(d, dq + 2, dk + 2, idesc, 1u);
+      ptx::mma_ss(d, dq + 4, dk + 4, idesc, 1u);
+      ptx::mma_ss(d, dq + 6, dk + 6, idesc, 1u);
+      ptx::mma_commit(bar(kBarSFull));
+      ptx::mma_commit(bar(kBarKFree + static_cast<int>(ks)));
     }
   }
   // Every MMA this thread issued must finish before TMEM is released.
   ptx::mma_commit(bar(kBarMmaFinal));
-  wait_force(bar(kBarMmaFinal), 0, abort_flag, p.timeout_ns);
+  wait_force<2>(bar(kBarMmaFinal), 0, abort_flag, p.timeout_ns);
 }
 
 // tcgen05 PV issuer, one thread.  Chunk g: once V(g) has landed and the softmax has
-// written P(g), O (+)= P V, then one commit that frees V stage g % 5, tells the S
-// issuer S buffer g % 3 is free, and tells the softmax warps that O holds chunk g.
-// A tile's first PV waits until the previous tile's epilogue has read O.
+// written P(g), O (+)= P(g) V_g, 16 keys per MMA (the first MMA of a tile overwrites
+// O), then one commit that frees V stage g % 2 and the P columns and tells the softmax
+// warps that O holds chunk g.
 __device__ __forceinline__ void pv_issuer(const FwdParams& p, const Slot& sl, volatile int* abort_flag) {
   const uint32_t sV = sl.sV, bars = sl.bars, tmem = sl.tmem;
-  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  auto bar = [&](int i) { return bar_at(bars, i); };
   constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 64, true);
   const uint64_t dv0 = ptx::smem_desc_sw128(sV, 0);
+  const uint32_t d = tmem + kTmemO;
   uint32_t g = 0;
   bool alive = true;
   for (uint32_t nq = 0; alive; ++nq) {
     int count = 0;
     if (take_item_one(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
-    for (int n = 0; n < count; ++n, ++g) {
-      if (n == 0 && !wait_one(bar(kBarOFree), (nq & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
-        alive = false;
-        break;
-      }
-      const uint32_t vs = g % kVStages, sb = g % kSBufs;
-      if (!wait_one(bar(kBarVFull + vs), (g / kVStages) & 1u, abort_flag, p.timeout_ns) ||
-          !wait_one(bar(kBarPFull + sb), (g / kSBufs) & 1u, abort_flag, p.timeout_ns)) {
+    for (int e0 = 0; e0 < count; e0 += kChunkEnt, ++g) {
+      const uint32_t vs = g % kVStages;
+      if (!wait_one<2>(bar(kBarVFull + vs), (g / kVStages) & 1u, abort_flag, p.timeout_ns) ||
+          !wait_one<2>(bar(kBarPFull), g & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
       ptx::tc_fence_after();
-      const uint32_t acc0 = n == 0 ? 0u : 1u;
-      const uint64_t dv = dv0 + vs * (kBlkBytes >> 4);
-      const uint32_t d = tmem + kTmemO;
-      const uint32_t a = tmem + kTmemS + sb * 64u;
-      ptx::mma_ts(d, a, dv, kIdescPV, acc0);  // 16 keys per MMA
+      const uint64_t dv = dv0 + vs * (kStageBytes >> 4);
+      const uint32_t a = tmem + kTmemP;
+      ptx::mma_ts(d, a, dv, kIdescPV, e0 == 0 ? 0u : 1u);  // 16 keys per MMA
       ptx::mma_ts(d, a + 8u, dv + (2048u >> 4), kIdescPV, 1u);
       ptx::mma_ts(d, a + 16u, dv + (4096u >> 4), kIdescPV, 1u);
       ptx::mma_ts(d, a + 24u, dv + (6144u >> 4), kIdescPV, 1u);
-      ptx::mma_commit(bar(kBarVFree + vs));
+      if (count - e0 >= 2) {
+        ptx::mma_ts(d, a + 32u, dv + (8192u >> 4), kIdescPV, 1u);
+        ptx::mma_ts(d, a + 40u, dv + (10240u >> 4), kIdescPV, 1u);
+        ptx::mma_ts(d, a + 48u, dv + (12288u >> 4), kIdescPV, 1u);
+        ptx::mma_ts(d, a + 56u, dv + (14336u >> 4), kIdescPV, 1u);
+      }
+      ptx::mma_commit(bar(kBarVFree + static_cast<int>(vs)));
     }
   }
   ptx::mma_commit(bar(kBarMmaFinal + 1));
-  wait_force(bar(kBarMmaFinal + 1), 0, abort_flag, p.timeout_ns);
+  wait_force<2>(bar(kBarMmaFinal + 1), 0, abort_flag, p.timeout_ns);
 }
 
-__device__ __forceinline__ void mask_cols(float (&s)[64], unsigned long long mk) {
-  if (mk == ~0ull) return;
-#pragma unroll
-  for (int c = 0; c < 64; ++c)
-    if (!((mk >> c) & 1ull)) s[c] = -INFINITY;
-}
-
-// What the epilogue of a finished tile needs; it runs one chunk later (after the
-// first chunk of the next tile) so the wait for the tile's last PV is hidden.
+// What the epilogue of a finished tile needs; it runs in the first chunk of the next
+// tile, after that chunk's wait for the tile's last PV.
 struct TileDone {
-  uint32_t k;       // the item's position in the slot's item sequence (its stage: k % ring)
-  uint32_t g_last;  // global index of the tile's last chunk
-  float m, l;       // the row's running max (log2 units) and sum
+  uint32_t k;  // the item's position in the slot's item sequence (its stage: k % ring)
+  float m, l;  // the row's running max (log2 units) and sum
 };
 
-// Epilogue of a finished tile: normalise O and store it with lse (or, for a chunk
-// of a split tile, its partial record).  Kept out of line: it runs once per tile
-// and would otherwise crowd the chunk loop's registers.
-__device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& td, const ItemStage& st,
-                                           const Slot& sl, uint32_t bars,
-                                           uint32_t obase, int warp, int lane, volatile int* abort_flag) {
-  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+// Epilogue of a finished tile (its last PV is done): normalise O and store it with
+// lse, or, for a chunk of a split tile, its partial record.  O rows go through the
+// tile's own Q buffer (its S MMAs are complete) and one TMA store per warp.  Out of
+// line: it runs once per tile and would otherwise crowd the chunk loop's code and
+// registers (only the softmax warps call it, so it is compiled to their budget).
+__device__ __noinline__ void tile_epilogue(const FwdParams& p, const TileDone& td, const ItemStage& st,
+                                              const Slot& sl, uint32_t obase, int warp, int lane) {
   const int r = (warp & 3) * 32 + lane;
   const int half = r >> 6;
   const int tb = st.b;
   const WorkItem& tw = st.w;
   const int tqa = st.qa, tqb = st.qb;
   const int tbh = tb * p.H + tw.h;
-  // PV of the tile's last chunk.  Unambiguous phase: S(g_last) was seen, and it was
-  // issued after PV(g_last - 3) was done; PV(g_last + kVStages) needs P this warp
-  // has not produced.
-  if (!wait_warp(bar(kBarVFree + static_cast<int>(td.g_last % kVStages)), (td.g_last / kVStages) & 1u,
-                 abort_flag, p.timeout_ns))
-    return false;
-  ptx::tc_fence_after();
   float o[64];
   {
     uint32_t raw[2][32];
@@ -439,21 +465,18 @@ __device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& t
 #pragma unroll
     for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(raw[c >> 5][c & 31]);
   }
-  ptx::tc_fence_before();
-  ptx::mbar_arrive(bar(kBarOFree));  // O may now be overwritten by the next tile
   const float m = td.m, l = td.l;
   const bool row_active = half == 0 || tqb >= 0;
   const int qblk = half ? tqb : tqa;
   const size_t row = static_cast<size_t>(tbh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
   if (tw.split < 0) {
     if (row_active) {  // warp-uniform: a warp's 32 rows lie in one half
-      // O rows through this warp's staging buffer (128-byte swizzle: 16-byte
-      // chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)), then one TMA store of
-      // the warp's 32 x 64 tile.
+      // O rows through this warp's quarter of the tile's Q buffer (128-byte swizzle:
+      // 16-byte chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)), then one TMA store
+      // of the warp's 32 x 64 tile.
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint8_t* stg = sl.ostage + (warp & 3) * kOStageBytes;
-      if (lane == 0) ptx::bulk_wait_read_all();  // the previous tile's store has read it
-      __syncwarp();
+      const uint32_t qs = td.k & 1u;
+      uint8_t* stg = sl.q_generic + qs * kQBytes + (warp & 3) * kOStageBytes;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         uint4 u;
@@ -466,13 +489,13 @@ __device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& t
       ptx::fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        ptx::tma_store_2d(&p.tm_o, sl.sO + (warp & 3) * kOStageBytes, 0,
+        ptx::tma_store_2d(&p.tm_o, sl.sQ + qs * kQBytes + (warp & 3) * kOStageBytes, 0,
                           static_cast<int>(row - static_cast<size_t>(r & 31)));
         ptx::bulk_commit_group();
       }
       p.lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
-    return true;
+    return;
   }
   // ---- split chunk: its partial record (unnormalised O, m, l)
   float* rec = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec) * kRecFloats;
@@ -482,13 +505,75 @@ __device__ __noinline__ bool tile_epilogue(const FwdParams& p, const TileDone& t
     orow[v4] = make_float4(o[v4 * 4 + 0], o[v4 * 4 + 1], o[v4 * 4 + 2], o[v4 * 4 + 3]);
   rec[kTileRows * 64 + r] = l > 0.f ? m : -INFINITY;
   rec[kTileRows * 64 + kTileRows + r] = l;
-  return true;
+}
+
+// Releases the Q buffer of the tile whose epilogue ran last: its O store (if any)
+// has finished reading the staged rows.
+__device__ __forceinline__ void release_q(const Slot& sl, uint32_t k, int lane) {
+  if (lane == 0) ptx::bulk_wait_read_all();
+  __syncwarp();
+  if (lane == 0) ptx::mbar_arrive(bar_at(sl.bars, kBarQEmpty + static_cast<int>(k & 1u)));
+}
+
+// Masks the scores of padded keys (keys 0-31 in a, 32-63 in b).
+__device__ __forceinline__ void mask_group(uint32_t (&a)[32], uint32_t (&b)[32], unsigned long long mk) {
+  if (mk == ~0ull) return;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    if (!((mk >> c) & 1ull)) a[c] = __float_as_uint(-INFINITY);
+    if (!((mk >> (c + 32)) & 1ull)) b[c] = __float_as_uint(-INFINITY);
+  }
+}
+
+__device__ __forceinline__ float group_max(const uint32_t (&a)[32], const uint32_t (&b)[32]) {
+  auto f = [](uint32_t x) { return __uint_as_float(x); };
+  // four independent chains of three-input maxima
+  float mx[4] = {fmaxf(f(a[0]), f(a[1])), fmaxf(f(a[2]), f(a[3])), fmaxf(f(b[0]), f(b[1])),
+                 fmaxf(f(b[2]), f(b[3]))};
+#pragma unroll
+  for (int c = 4; c < 32; c += 4) {
+    mx[0] = ptx::fmax3(mx[0], f(a[c]), f(a[c + 1]));
+    mx[1] = ptx::fmax3(mx[1], f(a[c + 2]), f(a[c + 3]));
+    mx[2] = ptx::fmax3(mx[2], f(b[c]), f(b[c + 1]));
+    mx[3] = ptx::fmax3(mx[3], f(b[c + 2]), f(b[c + 3]));
+  }
+  return fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+}
+
+// p = 2^(s * scale_log2 - m) for the 64 scores of one group (keys 0-31 in a, 32-63 in
+// b), packed to bf16 pairs in key order; returns the fp32 sum of p.  The scaling and
+// the sums run on packed fp32 pairs (two lanes per instruction).
+__device__ __forceinline__ float group_exp(const uint32_t (&a)[32], const uint32_t (&b)[32], uint64_t sc2,
+                                           uint64_t nm2, uint32_t (&pk)[32]) {
+  uint64_t acc0 = 0ull, acc1 = 0ull;
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const uint32_t* src = c < 16 ? a : b;
+    const int cc = (c & 15) * 2;
+    float x0, x1;
+    ptx::unpack2(ptx::ffma2(ptx::pack2(__uint_as_float(src[cc]), __uint_as_float(src[cc + 1])), sc2, nm2), x0, x1);
+    const float p0 = ptx::ex2_approx(x0), p1 = ptx::ex2_approx(x1);
+    if (c & 1)
+      acc1 = ptx::fadd2(acc1, ptx::pack2(p0, p1));
+    else
+      acc0 = ptx::fadd2(acc0, ptx::pack2(p0, p1));
+    pk[c] = pack_bf16x2(p0, p1);
+  }
+  float s0, s1;
+  ptx::unpack2(ptx::fadd2(acc0, acc1), s0, s1);
+  return s0 + s1;
+}
+
+// The membership-and-padding mask of union entry e for this half of the tile: 0 when
+// the half does not attend the key block, else the block's kept-key bits.
+__device__ __forceinline__ unsigned long long entry_mask(const ItemStage& st, int e, int half) {
+  return ((st.ent[e] >> (kEntBitsShift + half)) & 1u) ? st.kb[e] : 0ull;
 }
 
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl, int warp, int lane,
                                              volatile int* abort_flag) {
   const uint32_t bars = sl.bars, tmem = sl.tmem;
-  auto bar = [&](int i) { return bars + 8u * static_cast<uint32_t>(i); };
+  auto bar = [&](int i) { return bar_at(bars, i); };
   const int r = (warp & 3) * 32 + lane;  // tile row == TMEM lane (warp w reaches lanes 32 (w % 4)..)
   const int half = r >> 6;               // warp-uniform: a warp's 32 rows lie in one half
   const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -496,106 +581,104 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
   const float sl2 = p.scale_log2;
   uint32_t g = 0;
   bool alive = true;
+  // waits for PV(x): its commit freed V stage x % 2
+  auto wait_pv = [&](uint32_t x) {
+    return wait_warp<1>(bar(kBarVFree + static_cast<int>(x % kVStages)), (x / kVStages) & 1u, abort_flag,
+                           p.timeout_ns);
+  };
 
   TileDone pend{};
-  bool have_pend = false;
+  bool have_pend = false;  // a finished tile waits for its epilogue
+  bool q_pending = false;  // the tile of the last epilogue still holds its Q buffer
+  uint32_t q_k = 0;
   for (uint32_t k = 0; alive; ++k) {
-    const int t = take_item_warp(sl, k, abort_flag, p.timeout_ns);
+    const int t = take_item_warp<1>(sl, k, abort_flag, p.timeout_ns);
     if (t < 0) {
       if (t == kItemAbort) alive = false;
       break;
     }
-    // the tile's union entries and their key-padding bits, staged by the producer
+    // the tile's union entries and their key-padding bits, staged by the K producer
     const ItemStage& st = sl.items[k % kItemRing];
     const int count = st.w.count;
     float m_run = -INFINITY, l_run = 0.f;
-    for (int n = 0; n < count; ++n, ++g) {
-      const uint32_t e = st.ent[n];
-      const unsigned long long kb = st.kb[n];
-      const unsigned long long mk = ((e >> (kEntBitsShift + half)) & 1u) ? kb : 0ull;
-      const uint32_t sb = g % kSBufs;
-      if (!wait_warp(bar(kBarSFull + static_cast<int>(sb)), (g / kSBufs) & 1u, abort_flag, p.timeout_ns)) {
+    // masks of the chunk's two entries, read one chunk ahead
+    unsigned long long mk0 = entry_mask(st, 0, half);
+    unsigned long long mk1 = count >= 2 ? entry_mask(st, 1, half) : 0ull;
+    for (int e0 = 0; e0 < count; e0 += kChunkEnt, ++g) {
+      if (q_pending && e0 > 0) {  // one chunk after the epilogue: its O store has had time
+        q_pending = false;
+        release_q(sl, q_k, lane);
+      }
+      const bool two = count - e0 >= 2;
+      if (!wait_warp<1>(bar(kBarSFull), g & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
       ptx::tc_fence_after();
-      const uint32_t sbase = tmem + lane_addr + kTmemS + sb * 64u;
-      // p = 2^(s * scale * log2 e - m) with the row's running max m as it stands (a
-      // lazy max): m is raised only on the row's first attended chunk, or when the
-      // chunk's sum of p would exceed 2^kLazyLog2 -- then the chunk is redone with
-      // its own max folded into m, and l and O are rescaled.  So every p stays below
-      // 2^kLazyLog2, which bf16 P and fp32 O and l hold without loss of relative
-      // precision, and the common chunk reads S once and takes no max.
+      // all of S(g) into registers; the S columns go straight back to the S issuer
+      const uint32_t sbase = tmem + lane_addr + kTmemS;
+      // (loaded whatever the membership: a load under a condition makes the compiler keep
+      // both versions of the registers alive)
+      uint32_t a0[32], b0[32], a1[32], b1[32];
+      ptx::tmem_ld32(sbase, a0);
+      ptx::tmem_ld32(sbase + 32u, b0);
+      ptx::tmem_ld32(sbase + 64u, a1);
+      ptx::tmem_ld32(sbase + 96u, b1);
+      ptx::tmem_wait_ld();
+      ptx::reg_fence(a0);
+      ptx::reg_fence(b0);
+      ptx::reg_fence(a1);
+      ptx::reg_fence(b1);
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(kBarSFree));
+      // the next chunk's masks, while this one computes
+      const unsigned long long nmk0 = e0 + 2 < count ? entry_mask(st, e0 + 2, half) : 0ull;
+      const unsigned long long nmk1 = e0 + 3 < count ? entry_mask(st, e0 + 3, half) : 0ull;
+      // keys dropped by the padding mask inside an attended block (rare)
+      if (((mk0 + 1ull) > 1ull) || ((mk1 + 1ull) > 1ull)) {  // some mask neither 0 nor all ones
+        if (mk0 != 0ull) mask_group(a0, b0, mk0);
+        if (mk1 != 0ull) mask_group(a1, b1, mk1);
+      }
+      // chunk max over the keys this row attends (mk != 0 keeps at least one key); the
+      // running max is raised only past it by more than 2^kRescaleLog2
+      const float gm0 = group_max(a0, b0), gm1 = group_max(a1, b1);
+      const float cm = fmaxf(mk0 != 0ull ? gm0 : -INFINITY, mk1 != 0ull ? gm1 : -INFINITY);
+      const float cm2 = cm * sl2;  // scale > 0: the max of the scaled scores
+      const float m_new = cm2 > m_run + kRescaleLog2 ? cm2 : m_run;
+      const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
+      uint32_t pk0[32], pk1[32];
       float psum = 0.f;
-      float m_new = m_run;
-      uint32_t pk[32];
-      if (mk != 0ull) {
-        bool need_max = __any_sync(0xffffffffu, m_run == -INFINITY);
-        const uint64_t sc2 = ptx::pack2(sl2, sl2);
-        for (;;) {
-          uint32_t raw[2][32];
-          ptx::tmem_ld32(sbase + 0, raw[0]);
-          ptx::tmem_ld32(sbase + 32, raw[1]);
-          ptx::tmem_wait_ld();
-          ptx::reg_fence(raw[0]);
-          ptx::reg_fence(raw[1]);
-          float s[64];
-#pragma unroll
-          for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(raw[c >> 5][c & 31]);
-          mask_cols(s, mk);
-          if (need_max) {  // warp-uniform
-            float mx4[4] = {s[0], s[1], s[2], s[3]};
-#pragma unroll
-            for (int c = 4; c < 64; c += 2) mx4[(c >> 1) & 3] = ptx::fmax3(mx4[(c >> 1) & 3], s[c], s[c + 1]);
-            const float mx = fmaxf(ptx::fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
-            // mk != 0 keeps at least one key, so mx is finite (scale > 0)
-            m_new = fmaxf(m_run, mx * sl2);
-          }
-          const uint64_t nm2 = ptx::pack2(-m_new, -m_new);
-          uint64_t acc0 = 0ull, acc1 = 0ull;  // packed partial row sums
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float x0, x1;
-            ptx::unpack2(ptx::ffma2(ptx::pack2(s[2 * c], s[2 * c + 1]), sc2, nm2), x0, x1);
-            const float p0 = ptx::ex2_approx(x0), p1 = ptx::ex2_approx(x1);
-            if (c & 1)
-              acc1 = ptx::fadd2(acc1, ptx::pack2(p0, p1));
-            else
-              acc0 = ptx::fadd2(acc0, ptx::pack2(p0, p1));
-            pk[c] = pack_bf16x2(p0, p1);
-          }
-          float a0, a1;
-          ptx::unpack2(ptx::fadd2(acc0, acc1), a0, a1);
-          psum = a0 + a1;
-          // !(<=) also catches an infinite or NaN sum
-          if (need_max || !__any_sync(0xffffffffu, !(psum <= kLazyBound))) break;
-          need_max = true;
-        }
-        // P (bf16, two keys per column) over S columns already read.  The buffer's
-        // previous reader, PV of chunk g - 3, completed before S(g) was issued.
-        ptx::tmem_st32(sbase, pk);
+      if (mk0 != 0ull) {
+        psum += group_exp(a0, b0, sc2, nm2, pk0);
       } else {
-        // this half of the tile does not attend the block (or all of its keys are
-        // padding): its P rows are zero
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
-        ptx::tmem_st32(sbase, pk);
+        for (int c = 0; c < 32; ++c) pk0[c] = 0u;
+      }
+      if (mk1 != 0ull) {
+        psum += group_exp(a1, b1, sc2, nm2, pk1);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk1[c] = 0u;
       }
       const bool grew = m_new != m_run;
       const float alpha = grew ? ptx::ex2_approx(m_run - m_new) : 1.f;  // 2^-inf = 0
-      const bool had_mass = l_run > 0.f;
-      l_run = l_run * alpha + psum;
-      if (n > 0 && __any_sync(0xffffffffu, grew && had_mass)) {
-        // O must hold PV of chunk g - 1 before it is rescaled: wait for its V-free
-        // phase.  Unambiguous: S(g) was issued after PV(g - 3) was done, and
-        // PV(g - 1 + kVStages) needs this warp's P first.
-        const uint32_t gp = g - 1u;
-        if (!wait_warp(bar(kBarVFree + static_cast<int>(gp % kVStages)), (gp / kVStages) & 1u, abort_flag,
-                       p.timeout_ns)) {
-          alive = false;
-          break;
-        }
-        ptx::tc_fence_after();
+      const bool rescale = grew && l_run > 0.f;  // O holds this tile's earlier chunks
+      // PV(g - 1) done: the P columns are free, and O holds the previous chunk (the
+      // previous tile's last, at e0 == 0) for the epilogue or a rescale
+      if (g > 0 && !wait_pv(g - 1)) {
+        alive = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      if (e0 == 0 && have_pend) {  // the previous tile's epilogue
+        have_pend = false;
+        tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, obase, warp, lane);
+        release_item_warp(sl, pend.k, lane);
+        q_pending = true;
+        q_k = pend.k;
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
         for (int hlf = 0; hlf < 2; ++hlf) {
           uint32_t o[32];
@@ -607,26 +690,32 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
           ptx::tmem_st32(obase + 32u * hlf, o);
         }
       }
+      const uint32_t pbase = tmem + lane_addr + kTmemP;
+      ptx::tmem_st32(pbase, pk0);
+      if (two) ptx::tmem_st32(pbase + 32u, pk1);
+      l_run = l_run * alpha + psum;
       m_run = m_new;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(bar(kBarPFull + static_cast<int>(sb)));
-      if (n == 0 && have_pend) {  // the previous tile's epilogue, one chunk late
-        have_pend = false;
-        if (!tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, bars, obase, warp, lane, abort_flag)) {
-          alive = false;
-          break;
-        }
-        release_item_warp(sl, pend.k, lane);
-      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(kBarPFull));
+      mk0 = nmk0;
+      mk1 = nmk1;
     }
     if (!alive) break;
-    pend = TileDone{k, g - 1u, m_run, l_run};
+    if (q_pending) {  // a one-chunk tile: release before the next item's loads need the buffer
+      q_pending = false;
+      release_q(sl, q_k, lane);
+    }
+    pend = TileDone{k, m_run, l_run};
     have_pend = true;
   }
-  if (alive && have_pend &&
-      tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, bars, obase, warp, lane, abort_flag))
+  if (alive && have_pend && wait_pv(g - 1)) {
+    // the last tile: its last PV is done
+    ptx::tc_fence_after();
+    tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, obase, warp, lane);
     release_item_warp(sl, pend.k, lane);
+  }
   if (lane == 0) ptx::bulk_wait_all();  // O stores complete before the CTA exits
 }
 
@@ -643,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
       const uint32_t bars = base + s * kSlotBytes + kSmemBar;
       for (int i = 0; i < kNumBars; ++i) {
         uint32_t count = 1;
-        if ((i >= kBarPFull && i < kBarPFull + static_cast<int>(kSBufs)) || i == kBarOFree) count = kSoftmaxThreads;
+        if ((i >= kBarQEmpty && i < kBarQEmpty + 2) || i == kBarSFree || i == kBarPFull) count = kWarpArrivals;
         if (i >= kBarItemEmpty && i < kBarItemEmpty + kItemRing) count = kItemReaders;
         ptx::mbar_init(bars + 8u * i, count);
       }
@@ -651,13 +740,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
     misc[1] = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == kKProdWarp && lane == 0) {
     ptx::prefetch_tensormap(&p.tm_q);
     ptx::prefetch_tensormap(&p.tm_k);
     ptx::prefetch_tensormap(&p.tm_v);
     ptx::prefetch_tensormap(&p.tm_o);
   }
-  if (warp == kMmaWarp) {
+  if (warp == kSWarp) {
     ptx::tmem_alloc(ptx::smem_addr(const_cast<uint32_t*>(&misc[0])), kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -666,34 +755,37 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   ptx::tc_fence_after();
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
-  const int slot = warp < 8 ? (warp >> 2) : warp < kMmaWarp ? warp - kProducerWarp : (warp - kMmaWarp) >> 1;
+  const int slot = warp < 8 ? (warp >> 2) : (warp & 1);
   Slot sl;
   sl.sQ = base + slot * kSlotBytes + kSmemQ;
   sl.sK = base + slot * kSlotBytes + kSmemK;
   sl.sV = base + slot * kSlotBytes + kSmemV;
   sl.bars = base + slot * kSlotBytes + kSmemBar;
+  sl.q_generic = smem + slot * kSlotBytes + kSmemQ;
   sl.items = reinterpret_cast<ItemStage*>(smem + slot * kSlotBytes + kSmemItems);
-  sl.ostage = smem + slot * kSlotBytes + kSmemOStage;
-  sl.sO = base + slot * kSlotBytes + kSmemOStage;
   sl.tmem = misc[0] + static_cast<uint32_t>(slot) * kSlotCols;
 
   if (warp < 8) {
+    ptx::setmaxnreg_inc<kSoftmaxRegs>();
     softmax_role(p, sl, warp, lane, abort_flag);
-  } else if (warp < kMmaWarp) {
-    producer_role(p, sl, lane, abort_flag);
-    __syncwarp();
-  } else if (warp == kMmaWarp + 2 * slot) {
-    if (lane == 0) s_issuer(p, sl, abort_flag);
-    __syncwarp();
-  } else if (warp == kPvWarp + 2 * slot) {
-    if (lane == 0) pv_issuer(p, sl, abort_flag);
+  } else {
+    ptx::setmaxnreg_dec<kOtherRegs>();
+    if (warp < kSWarp) {
+      k_producer(p, sl, lane, abort_flag);
+    } else if (warp < kPvWarp) {
+      if (lane == 0) s_issuer(p, sl, abort_flag);
+    } else if (warp < kVProdWarp) {
+      if (lane == 0) pv_issuer(p, sl, abort_flag);
+    } else {
+      v_producer(p, sl, lane, abort_flag);
+    }
     __syncwarp();
   }
 
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == kMmaWarp) ptx::tmem_dealloc(misc[0], kTmemCols);
+  if (warp == kSWarp) ptx::tmem_dealloc(misc[0], kTmemCols);
 }
 
 // Merge of split tiles: one warp per (batch element, split tile, tile row).  The
@@ -866,6 +958,103 @@ int device_setup(int dev, DeviceInfo* out) {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// A forward call whose arguments have been checked: its workspace plan and device.
+struct ForwardCall {
+  WorkspacePlan plan;
+  int dev = -1;
+  DeviceInfo info;
+};
+
+// The checks a forward entry point makes before it enqueues anything, so that a
+// call that fails leaves the GPU untouched: first the arguments (no CUDA call;
+// fills in the workspace plan), then -- after the entry point has checked its
+// scratch against the plan -- the device.
+int validate_forward_args(const void* q, const void* k, const void* v, int B, int H, int L, int d,
+                          const bsa_layout* lay, const void* out, const float* lse, float scale, ForwardCall* c) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || lay == nullptr ||
+      B < 1 || H < 1 || L < 1)
+    return BSA_ERR_INVALID_ARG;
+  if (d != kHeadDim) return BSA_ERR_UNSUPPORTED;
+  if (H != lay->H || L != lay->L) return BSA_ERR_LAYOUT_MISMATCH;
+  if (static_cast<int64_t>(B) * H * L > INT32_MAX - 64) return BSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
+    return BSA_ERR_INVALID_ARG;
+  if (!(scale == scale) || std::isinf(scale)) return BSA_ERR_INVALID_ARG;
+  c->plan = plan_workspace(*lay, B);
+  return BSA_OK;
+}
+
+int validate_forward_device(const bsa_layout* lay, ForwardCall* c) {
+  if (lay->device < 0) return BSA_ERR_LAYOUT_MISMATCH;
+  if (cudaGetDevice(&c->dev) != cudaSuccess) return BSA_ERR_CUDA;
+  if (c->dev != lay->device) return BSA_ERR_LAYOUT_MISMATCH;
+  return device_setup(c->dev, &c->info);
+}
+
+// Enqueues a checked forward call on workspace ws (at least c.plan.total bytes):
+// clears the schedule counters, then the key bits (with a mask), the forward and
+// the split-row merge.
+int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const void* v, int B, int H, int L, int d,
+                    const bsa_layout* lay, const uint8_t* key_mask, float scale, void* out, float* lse,
+                    uint8_t* ws, cudaStream_t s) {
+  const WorkspacePlan& plan = c.plan;
+  FwdParams prm{};
+  const uint64_t rows = static_cast<uint64_t>(B) * H * L;
+  if (!make_map(&prm.tm_q, q, rows, 64) || !make_map(&prm.tm_k, k, rows, 64) ||
+      !make_map(&prm.tm_v, v, rows, 64) || !make_map(&prm.tm_o, out, rows, 32))
+    return BSA_ERR_CUDA;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.items = lay->d_items;
+  prm.pair_q = lay->d_pair_q;
+  prm.pair_ent = lay->d_pair_ent;
+  prm.keybits = key_mask ? reinterpret_cast<const unsigned long long*>(ws + plan.keybits_off) : nullptr;
+  prm.partials = reinterpret_cast<float*>(ws + plan.partials_off);
+  prm.sched = reinterpret_cast<int*>(ws + plan.sched_off);
+  prm.B = B;
+  prm.H = H;
+  prm.L = L;
+  prm.nb = lay->nb;
+  prm.items_per_batch = static_cast<int>(lay->items.size());
+  prm.n_split = lay->n_split;
+  prm.n_records = lay->n_records;
+  prm.split_items = static_cast<int>(std::count_if(lay->items.begin(), lay->items.end(),
+                                                   [](const WorkItem& it) { return it.split >= 0; }));
+  const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(d));
+  prm.scale_log2 = sc * kLog2e;
+  prm.timeout_ns = kDefaultTimeoutNs;
+
+  // the schedule counters start at zero whatever an earlier call (or a device
+  // error) left in the workspace
+  if (cudaMemsetAsync(ws + plan.sched_off, 0, plan.sched_bytes, s) != cudaSuccess) return BSA_ERR_CUDA;
+  if (key_mask != nullptr &&
+      launch_keybits(key_mask, reinterpret_cast<unsigned long long*>(ws + plan.keybits_off), B, L, lay->nb, s) !=
+          cudaSuccess)
+    return BSA_ERR_CUDA;
+  const int64_t total = static_cast<int64_t>(B) * prm.items_per_batch;
+  // two slots per CTA; items are drawn dynamically
+  const int grid = static_cast<int>(std::min<int64_t>((total + kSlots - 1) / kSlots, c.info.sms));
+  if (grid < 1) return BSA_OK;
+  bsa_fwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  if (lay->n_split > 0) {
+    MergeParams mp{};
+    mp.partials = prm.partials;
+    mp.splits = lay->d_splits;
+    mp.out = prm.out;
+    mp.lse = lse;
+    mp.B = B;
+    mp.H = H;
+    mp.L = L;
+    mp.n_split = lay->n_split;
+    mp.n_records = lay->n_records;
+    const int64_t tasks = static_cast<int64_t>(B) * lay->n_split * kTileRows;
+    bsa_merge_kernel<<<static_cast<int>((tasks + 3) / 4), 128, 0, s>>>(mp);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  return BSA_OK;
+}
+
 }  // namespace
 
 void free_device(bsa_layout* lay) {
@@ -957,80 +1146,14 @@ int bsa_layout_upload(bsa_layout* lay, void* stream) {
 int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L, int d,
                 const bsa_layout* lay, const uint8_t* key_mask, float scale, void* out, float* lse,
                 void* workspace, size_t workspace_bytes, void* stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr ||
-      lay == nullptr || B < 1 || H < 1 || L < 1)
-    return BSA_ERR_INVALID_ARG;
-  if (d != kHeadDim) return BSA_ERR_UNSUPPORTED;
-  if (H != lay->H || L != lay->L) return BSA_ERR_LAYOUT_MISMATCH;
-  if (static_cast<int64_t>(B) * H * L > INT32_MAX - 64) return BSA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
-    return BSA_ERR_INVALID_ARG;
-  if (!(scale == scale) || std::isinf(scale)) return BSA_ERR_INVALID_ARG;
-  const WorkspacePlan plan = plan_workspace(*lay, B);
-  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < plan.total)
-    return BSA_ERR_WORKSPACE;
-  if (lay->device < 0) return BSA_ERR_LAYOUT_MISMATCH;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
-  if (dev != lay->device) return BSA_ERR_LAYOUT_MISMATCH;
-  DeviceInfo info;
-  const int st = device_setup(dev, &info);
+  ForwardCall c;
+  int st = validate_forward_args(q, k, v, B, H, L, d, lay, out, lse, scale, &c);
   if (st != BSA_OK) return st;
-
-  FwdParams prm{};
-  const uint64_t rows = static_cast<uint64_t>(B) * H * L;
-  if (!make_map(&prm.tm_q, q, rows, 64) || !make_map(&prm.tm_k, k, rows, 64) ||
-      !make_map(&prm.tm_v, v, rows, 64) || !make_map(&prm.tm_o, out, rows, 32))
-    return BSA_ERR_CUDA;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  prm.out = static_cast<__nv_bfloat16*>(out);
-  prm.lse = lse;
-  prm.items = lay->d_items;
-  prm.pair_q = lay->d_pair_q;
-  prm.pair_ent = lay->d_pair_ent;
-  prm.keybits = key_mask ? reinterpret_cast<const unsigned long long*>(ws + plan.keybits_off) : nullptr;
-  prm.partials = reinterpret_cast<float*>(ws + plan.partials_off);
-  prm.sched = reinterpret_cast<int*>(ws + plan.sched_off);
-  prm.B = B;
-  prm.H = H;
-  prm.L = L;
-  prm.nb = lay->nb;
-  prm.items_per_batch = static_cast<int>(lay->items.size());
-  prm.n_split = lay->n_split;
-  prm.n_records = lay->n_records;
-  prm.split_items = static_cast<int>(std::count_if(lay->items.begin(), lay->items.end(),
-                                                   [](const WorkItem& it) { return it.split >= 0; }));
-  const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(d));
-  prm.scale_log2 = sc * kLog2e;
-  prm.timeout_ns = kDefaultTimeoutNs;
-
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (key_mask != nullptr &&
-      launch_keybits(key_mask, reinterpret_cast<unsigned long long*>(ws + plan.keybits_off), B, L, lay->nb, s) !=
-          cudaSuccess)
-    return BSA_ERR_CUDA;
-  const int64_t total = static_cast<int64_t>(B) * prm.items_per_batch;
-  // two slots per CTA; items are drawn dynamically
-  const int grid = static_cast<int>(std::min<int64_t>((total + kSlots - 1) / kSlots, info.sms));
-  if (grid < 1) return BSA_OK;
-  bsa_fwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(prm);
-  if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
-  if (lay->n_split > 0) {
-    MergeParams mp{};
-    mp.partials = prm.partials;
-    mp.splits = lay->d_splits;
-    mp.out = prm.out;
-    mp.lse = lse;
-    mp.B = B;
-    mp.H = H;
-    mp.L = L;
-    mp.n_split = lay->n_split;
-    mp.n_records = lay->n_records;
-    const int64_t tasks = static_cast<int64_t>(B) * lay->n_split * kTileRows;
-    bsa_merge_kernel<<<static_cast<int>((tasks + 3) / 4), 128, 0, s>>>(mp);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
-  }
-  return BSA_OK;
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < c.plan.total) return BSA_ERR_WORKSPACE;
+  st = validate_forward_device(lay, &c);
+  if (st != BSA_OK) return st;
+  return enqueue_forward(c, q, k, v, B, H, L, d, lay, key_mask, scale, out, lse,
+                         static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 int bsa_sync_status(void* stream) {
@@ -1066,45 +1189,32 @@ int bsa_debug_wait_timeout(uint64_t timeout_ns, void* stream) {
 static __device__ __align__(256) unsigned char g_bsa_static_ws[BSA_STATIC_WORKSPACE_BYTES];
 
 namespace {
+// Per device, the array's device address once a lookup has succeeded (a failed
+// lookup is retried on the next call).  Not refreshed after cudaDeviceReset.
 void* g_static_ws_addr[kMaxDevices];
-cudaError_t g_static_ws_err[kMaxDevices];
-std::once_flag g_static_ws_once[kMaxDevices];
+std::mutex g_static_ws_mu;
 }  // namespace
 
 extern "C" int bsa_forward_static_ws(const void* q, const void* k, const void* v, int B, int H, int L,
                                      int d, const bsa_layout* lay, const uint8_t* key_mask, float scale,
                                      void* out, float* lse, void* stream) {
-  // The checks bsa_forward makes before touching the GPU, repeated so that a bad
-  // call enqueues nothing (not even the ticket clear below).
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr ||
-      lay == nullptr || B < 1 || H < 1 || L < 1)
-    return BSA_ERR_INVALID_ARG;
-  if (d != kHeadDim) return BSA_ERR_UNSUPPORTED;
-  if (H != lay->H || L != lay->L) return BSA_ERR_LAYOUT_MISMATCH;
-  if (static_cast<int64_t>(B) * H * L > INT32_MAX - 64) return BSA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
-    return BSA_ERR_INVALID_ARG;
-  if (!(scale == scale) || std::isinf(scale)) return BSA_ERR_INVALID_ARG;
-  const WorkspacePlan plan = plan_workspace(*lay, B);
-  if (plan.total > BSA_STATIC_WORKSPACE_BYTES) return BSA_ERR_STATIC_WORKSPACE;
-  if (lay->device < 0) return BSA_ERR_LAYOUT_MISMATCH;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
-  if (dev != lay->device) return BSA_ERR_LAYOUT_MISMATCH;
-  if (dev < 0 || dev >= kMaxDevices) return BSA_ERR_UNSUPPORTED;
-  DeviceInfo info;
-  const int st = device_setup(dev, &info);
+  ForwardCall c;
+  int st = validate_forward_args(q, k, v, B, H, L, d, lay, out, lse, scale, &c);
   if (st != BSA_OK) return st;
-  // once per device, with that device current: the array's address on it
-  std::call_once(g_static_ws_once[dev], [dev] {
-    g_static_ws_err[dev] = cudaGetSymbolAddress(&g_static_ws_addr[dev], g_bsa_static_ws);
-  });
-  if (g_static_ws_err[dev] != cudaSuccess || g_static_ws_addr[dev] == nullptr) return BSA_ERR_CUDA;
-  uint8_t* ws = static_cast<uint8_t*>(g_static_ws_addr[dev]);
-  // the schedule counters must start at zero; the other regions are written before read
-  if (cudaMemsetAsync(ws + plan.sched_off, 0, plan.sched_bytes, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
-    return BSA_ERR_CUDA;
-  return bsa_forward(q, k, v, B, H, L, d, lay, key_mask, scale, out, lse, ws, BSA_STATIC_WORKSPACE_BYTES,
-                     stream);
+  if (c.plan.total > BSA_STATIC_WORKSPACE_BYTES) return BSA_ERR_STATIC_WORKSPACE;
+  st = validate_forward_device(lay, &c);
+  if (st != BSA_OK) return st;
+  void* addr = nullptr;
+  {
+    // with this device current: the array's address on it
+    std::lock_guard<std::mutex> lk(g_static_ws_mu);
+    if (g_static_ws_addr[c.dev] == nullptr) {
+      void* found = nullptr;
+      if (cudaGetSymbolAddress(&found, g_bsa_static_ws) != cudaSuccess || found == nullptr) return BSA_ERR_CUDA;
+      g_static_ws_addr[c.dev] = found;
+    }
+    addr = g_static_ws_addr[c.dev];
+  }
+  return enqueue_forward(c, q, k, v, B, H, L, d, lay, key_mask, scale, out, lse, static_cast<uint8_t*>(addr),
+                         static_cast<cudaStream_t>(stream));
 }

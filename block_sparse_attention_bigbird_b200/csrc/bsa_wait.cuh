@@ -26,8 +26,8 @@ constexpr uint32_t kWaitSleepNs = 20000;  // upper bound on one sleep inside a b
 static __device__ int g_bsa_status;
 
 // ------------------------------------------------------------ bounded waits
-static __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                       uint64_t timeout_ns, bool honor_abort) {
+__device__ __forceinline__ bool wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t timeout_ns, bool honor_abort) {
   const uint64_t t0 = ptx::globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     // sleeping in the barrier instead of spinning leaves issue slots to the
@@ -44,18 +44,29 @@ static __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, vol
   }
 }
 
+// The slow path, out of line.  kRegion tells apart the copies called from warps with
+// different register budgets (setmaxnreg): one function may be called only from code
+// compiled to one budget, so each such region gets its own instantiation.
+template <int kRegion>
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       uint64_t timeout_ns, bool honor_abort) {
+  return wait_spin(bar, parity, abort_flag, timeout_ns, honor_abort);
+}
+
 // Whole-warp wait; the result is warp-uniform.
+template <int kRegion = 0>
 __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint64_t timeout_ns) {
   bool ok = ptx::mbar_try_wait(bar, parity);
   if (__all_sync(0xffffffffu, ok)) return true;
-  ok = wait_slow(bar, parity, abort_flag, timeout_ns, true);
+  ok = wait_slow<kRegion>(bar, parity, abort_flag, timeout_ns, true);
   return __all_sync(0xffffffffu, ok);
 }
 
+template <int kRegion = 0>
 __device__ __forceinline__ void wait_force(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            uint64_t timeout_ns) {
-  if (!ptx::mbar_try_wait(bar, parity)) wait_slow(bar, parity, abort_flag, timeout_ns, false);
+  if (!ptx::mbar_try_wait(bar, parity)) wait_slow<kRegion>(bar, parity, abort_flag, timeout_ns, false);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -65,10 +76,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // ------------------------------------------------------------ roles
 // Single-thread wait (the TMA and MMA roles run on one elected lane).
+template <int kRegion = 0>
 __device__ __forceinline__ bool wait_one(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                          uint64_t timeout_ns) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, abort_flag, timeout_ns, true);
+  return wait_slow<kRegion>(bar, parity, abort_flag, timeout_ns, true);
 }
 
 }  // namespace bsa

@@ -230,6 +230,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// ----------------------------------------------------------------- register split
+// Per-warpgroup register budget (every warp of the warpgroup executes it).  The
+// budgets of all warpgroups must add up to no more than the block's launch budget.
+template <uint32_t kRegs>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // ----------------------------------------------------------------- misc
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

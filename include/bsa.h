@@ -198,10 +198,12 @@ void bsa_layout_free(bsa_layout* layout);
  * bsa_workspace_bytes -- device scratch bytes bsa_forward needs for batch size
  * B: the counters of the dynamic work schedule, the per-key-block padding bits
  * and the partial results of split rows (global rows whose key-block list is cut
- * into chunks that run as separate work items).  The workspace must be
- * ZERO-FILLED before its first use; every call that completes without a device
- * error leaves the counters zero again, so it can be reused without clearing.
- * After a call that ended in a device error, clear it again.
+ * into chunks that run as separate work items).  It needs no clearing: every
+ * call first zeroes the 256 bytes of schedule counters it uses (one
+ * cudaMemsetAsync on the call's stream) and writes every other byte before
+ * reading it, so a workspace in any state -- fresh, reused, or left by a call
+ * that ended in a device error -- can be passed.  Concurrent calls need
+ * separate workspaces.
  */
 int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
 
@@ -217,9 +219,10 @@ int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
  *             scores over the attended keys; -inf (with O = 0) for a row whose
  *             attended set is empty.
  *   workspace device, at least bsa_workspace_bytes(layout, B) bytes, 256-byte
- *             aligned, zero-filled before first use (see above).
- * Enqueues up to three kernels on `stream`: the key-padding bits (with a key
- * mask), the forward, and the merge of split rows (when the layout has any).
+ *             aligned, any contents (see above).
+ * Enqueues on `stream` a 256-byte memset of the schedule counters and up to
+ * three kernels: the key-padding bits (with a key mask), the forward, and the
+ * merge of split rows (when the layout has any).
  * Returns after enqueueing (no synchronisation, no allocation).  A device-side
  * timeout is reported later by bsa_sync_status.
  */
@@ -242,8 +245,10 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int L
  *   - Returns BSA_ERR_STATIC_WORKSPACE, before anything is enqueued, when
  *     bsa_workspace_bytes(layout, B) exceeds BSA_STATIC_WORKSPACE_BYTES.
  *   - The first call on a device looks up the buffer's device address for that
- *     device (cudaGetSymbolAddress, no allocation); make that first call before
- *     any stream capture.
+ *     device (cudaGetSymbolAddress, no allocation) and keeps it once the lookup
+ *     succeeds (a failed lookup is retried by the next call); make that first
+ *     call before any stream capture.  The kept address is not refreshed after
+ *     cudaDeviceReset: do not reset a device between calls.
  *   - Every call clears the buffer's schedule counters with cudaMemsetAsync on
  *     `stream`, then enqueues the forward.  All calls on a device share the one
  *     buffer, which keeps the last call's contents: calls whose execution

@@ -160,17 +160,23 @@ def test_constant_v_gives_constant_output_everywhere(bsa):
     assert torch.isfinite(lse).all().item()
 
 
-def test_deterministic_and_workspace_left_clean(bsa):
+def test_deterministic_and_any_workspace_contents(bsa):
+    """Two calls give bit-identical results, and a workspace full of garbage (as a
+    call that ended in a device error could leave it) gives the same result as a
+    zeroed one: each call clears the schedule counters it uses."""
     w = workloads.custom(2, 2, 64 * 64, 1, 2, 3, seed=1)
     q, k, v = [t.cuda() for t in workloads.make_qkv(w)]
     lay = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
     bsa.bsa_layout_upload(lay)
-    ws = torch.zeros(bsa.bsa_workspace_bytes(lay, w.B), dtype=torch.uint8, device="cuda")
+    n = bsa.bsa_workspace_bytes(lay, w.B)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
     o1, l1 = bsa.bsa_forward(q, k, v, lay, workspace=ws)
     o2, l2 = bsa.bsa_forward(q, k, v, lay, workspace=ws)
+    dirty = torch.full((n,), 0x5A, dtype=torch.uint8, device="cuda")
+    o3, l3 = bsa.bsa_forward(q, k, v, lay, workspace=dirty)
     assert bsa.bsa_sync_status() == 0
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
-    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0   # schedule counters back at zero
+    assert torch.equal(o1, o3) and torch.equal(l1, l3)
 
 
 def test_bounded_wait_reports_timeout_and_context_survives(bsa):
