@@ -7,6 +7,8 @@
   layout (a library routine).
 - Closed forms: the columns of dV sum to the sum of dO over non-empty rows;
   constant keys give dQ = 0; excluded keys get dK = dV = 0; dO = 0 gives zeros.
+- The magnitude sums that set the GPU tolerances, against per-token, per-key
+  scalar loops with math.exp (to 1e-12 relative).
 """
 
 import math
@@ -161,3 +163,52 @@ def test_rows_api_matches_full():
             assert np.abs(rv - dv[b, h, kt]).max() < 1e-12
             for a, m in ((sq, mq[b, h, qt]), (sk, mk[b, h, kt]), (sv, mv[b, h, kt])):
                 assert np.abs(a - m).max() < 1e-12
+
+
+def _magnitudes_by_scalar_loops(q, k, v, do, lay, km, scale):
+    """The magnitude sums of the docstring, written out term by term: for each
+    (b, h, query token t) the attended key set is listed from the layout's block
+    row and the key mask, P comes from math.exp, and every sum is a Python loop.
+    Nothing here is masked-dense and nothing is shared with the oracle's numpy form."""
+    B, H, L, d = q.shape
+    block = lay["block"]
+    mq, mk, mv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            for t in range(L):
+                blocks = [int(j) for j in OL.row(lay, h, t // block)]
+                keys = [p for j in blocks for p in range(j * block, (j + 1) * block)
+                        if km is None or int(km[b][p]) != 0]
+                if not keys:
+                    continue
+                s = {p: scale * sum(q[b, h, t, c] * k[b, h, p, c] for c in range(d)) for p in keys}
+                mx = max(s.values())
+                den = sum(math.exp(s[p] - mx) for p in keys)
+                P = {p: math.exp(s[p] - mx) / den for p in keys}
+                o = [sum(P[p] * v[b, h, p, c] for p in keys) for c in range(d)]
+                dabs = sum(abs(do[b, h, t, c]) * abs(o[c]) for c in range(d))
+                for p in keys:
+                    dp = sum(do[b, h, t, c] * v[b, h, p, c] for c in range(d))
+                    w = P[p] * (abs(dp) + dabs)
+                    for c in range(d):
+                        mq[b, h, t, c] += scale * w * abs(k[b, h, p, c])
+                        mk[b, h, p, c] += scale * w * abs(q[b, h, t, c])
+                        mv[b, h, p, c] += P[p] * abs(do[b, h, t, c])
+    return mq, mk, mv
+
+
+def test_magnitudes_match_scalar_loops():
+    # Pins the with_magnitude sums (their Dabs, |dP| and |K| / |Q| / |dO| factors)
+    # against an explicit per-token, per-key evaluation, with a padded key tail and
+    # a non-default scale so that a dropped factor or a transposed operand shows.
+    B, H, L, d = 1, 2, 64 * 3, 3
+    lay = OL.build_layout(H, L, 64, 0, 1, 1, 11)
+    q, k, v, do = (_rand((B, H, L, d), s) for s in (51, 52, 53, 54))
+    km = np.ones((B, L), dtype=np.uint8)
+    km[0, -20:] = 0
+    _, _, _, (mq, mk, mv) = OB.attention_backward(q, k, v, do, lay, key_mask=km, scale=0.7,
+                                                  with_magnitude=True)
+    rq, rk, rv = _magnitudes_by_scalar_loops(q, k, v, do, lay, km, 0.7)
+    for got, ref in ((mq, rq), (mk, rk), (mv, rv)):
+        assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+    assert np.all(mk[0, :, -20:] == 0) and np.all(mv[0, :, -20:] == 0)
