@@ -64,11 +64,12 @@ def masked_softmax_av(s: np.ndarray, allowed: np.ndarray, v: np.ndarray):
     return o, lse
 
 
-def attention(q, k, v, layout: dict, key_mask=None, scale=None, query_blocks=None):
+def attention(q, k, v, layout: dict, key_mask=None, scale=None, query_blocks=None, pairs=None):
     """O [B,H,L,d] and lse [B,H,L] in fp64 for the block layout (masked-dense).
 
     ``query_blocks`` optionally restricts the computation to those query blocks
-    (the other rows of the result stay zero); the arithmetic is unchanged.
+    and ``pairs`` to those (batch element, head) pairs (the other rows of the
+    result stay zero); the arithmetic is unchanged.
     """
     q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
     B, H, L, d = q.shape
@@ -79,16 +80,15 @@ def attention(q, k, v, layout: dict, key_mask=None, scale=None, query_blocks=Non
     assert layout["H"] == H and layout["L"] == L
     out = np.zeros((B, H, L, d))
     lse = np.zeros((B, H, L))
-    for b in range(B):
-        for h in range(H):
-            kt = k[b, h].T
-            for i in (range(nb) if query_blocks is None else query_blocks):
-                allowed = token_mask_row(layout, h, i, L)
-                if km is not None:
-                    allowed = allowed & km[b]
-                rows = slice(i * block, (i + 1) * block)
-                s = (q[b, h, rows] @ kt) * scale
-                out[b, h, rows], lse[b, h, rows] = masked_softmax_av(s, allowed, v[b, h])
+    for b, h in ([(b, h) for b in range(B) for h in range(H)] if pairs is None else pairs):
+        kt = k[b, h].T
+        for i in (range(nb) if query_blocks is None else query_blocks):
+            allowed = token_mask_row(layout, h, i, L)
+            if km is not None:
+                allowed = allowed & km[b]
+            rows = slice(i * block, (i + 1) * block)
+            s = (q[b, h, rows] @ kt) * scale
+            out[b, h, rows], lse[b, h, rows] = masked_softmax_av(s, allowed, v[b, h])
     return out, lse
 
 

@@ -6,9 +6,15 @@ tests/test_bwd_protocol.py).  A role is a list of operations on named mbarriers:
   ("arrive", bar)    one arrival by the role itself
   ("async", bar)     one arrival that happens later, in any order with the other
                      pending ones (a TMA load's completion or an MMA commit)
+  ("async", bar, f)  the same, calling f() when the operation lands (before the
+                     arrival): the moment an asynchronous copy or MMA has finished
+                     reading and writing its buffers
+  ("do", f)          calls f() when the role reaches it: a read or a write of a
+                     buffer, whose assertions check that the buffer holds what the
+                     role expects
 The replay asserts that each wait is met by exactly the phase it targets (a
-parity wait cannot tell phase t from phase t + 2) and that no schedule
-deadlocks.
+parity wait cannot tell phase t from phase t + 2), that every "do" and landing
+check holds, and that no schedule deadlocks.
 """
 
 import random
@@ -58,11 +64,16 @@ def replay(bars, roles, seed):
             return
         c = rnd.choice(choices)
         if c == "async":
-            bars[inflight.pop(rnd.randrange(len(inflight)))].arrive()
+            landed = inflight.pop(rnd.randrange(len(inflight)))
+            if len(landed) > 1:
+                landed[1]()
+            bars[landed[0]].arrive()
             continue
         op = roles[c][pc[c]]
         pc[c] += 1
         if op[0] == "arrive":
             bars[op[1]].arrive()
         elif op[0] == "async":
-            inflight.append(op[1])
+            inflight.append(op[1:])
+        elif op[0] == "do":
+            op[1]()

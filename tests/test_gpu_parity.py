@@ -145,6 +145,39 @@ def test_parity_full_size_sampled(bsa, name):
     assert np.isfinite(lse).all()
 
 
+FULL_HEADS = [
+    # name, (b, h) pairs checked on every row, which query blocks ("all" or the
+    # global blocks plus the blocks of the padded key tail and the 4 blocks before it)
+    ("c3", [(0, 0), (3, 11)], "all"),
+    ("c4", [(0, 9)], "all"),
+    ("c5", [(0, 7)], "globals_and_tail"),
+]
+
+
+@pytest.mark.parametrize("name,pairs,which", FULL_HEADS, ids=[f[0] for f in FULL_HEADS])
+def test_parity_full_heads(bsa, name, pairs, which):
+    """Every row of whole heads at the benchmark shapes, as launched by the
+    benchmark: all 256 query blocks of the first and last (b, h) of the L=16384
+    shape; all 128 blocks of one head of the 13-global shape (13 global query
+    blocks split across chunks and merged); and in the L=131072 shape with the
+    padded key tail, the global query blocks plus every query block of the
+    padded tail and the 4 before it (whose windows reach the padding)."""
+    w = workloads.get(name)
+    km = workloads.make_key_mask(w)
+    (q, k, v), _, ref_lay, o, lse = _run(bsa, w, key_mask=km)
+    if which == "all":
+        blocks = list(range(w.nb))
+    else:
+        tail0 = (w.L - w.key_pad_tail) // w.block - 4
+        blocks = sorted(set(int(g) for g in ref_lay["globals"]) | set(range(tail0, w.nb)))
+    if name == "c4":
+        assert len(ref_lay["globals"]) == 13
+    o_ref, lse_ref = OA.attention(q, k, v, ref_lay, key_mask=km, query_blocks=blocks, pairs=pairs)
+    rows = np.concatenate([np.arange(i * w.block, (i + 1) * w.block) for i in blocks])
+    for b, h in pairs:
+        _check(o[b, h, rows], lse[b, h, rows], o_ref[b, h, rows], lse_ref[b, h, rows])
+
+
 def test_constant_v_gives_constant_output_everywhere(bsa):
     # A property that holds at any size: softmax rows sum to 1, so v == c gives
     # O == c up to the bf16 rounding of P (l is summed from the unrounded fp32 p).

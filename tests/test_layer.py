@@ -113,3 +113,46 @@ def test_layer_equals_its_steps_spelled_out():
     assert bsa.bsa_sync_status() == 0
     for t in (x.grad, mod.qkv.weight.grad, mod.qkv.bias.grad, mod.proj.weight.grad):
         assert torch.isfinite(t.float()).all() and t.float().abs().sum() > 0
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+def test_layer_on_gpu_matches_fp64_dense_layer():
+    """The bf16 layer on the GPU (cuBLAS projections, the library's attention and
+    gradients) against the same layer evaluated in fp64 on the CPU from the same
+    bf16 weights and inputs: dense masked softmax over the oracle's layout, with
+    torch autograd for the gradients.  The bf16 rounding of q, k, v, O and y costs
+    about 0.4 % of the output's scale here; the bounds leave a 5x margin, while a
+    wrong head split, q/k/v order or gradient routing is off by O(1)."""
+    B, H, L = 2, 4, 64 * 24
+    dev = torch.device("cuda")
+    torch.manual_seed(1)
+    mod = BigBirdSelfAttention(H * 64, H, window=1, num_global=2, num_random=2, seed=3).to(dev, torch.bfloat16)
+    ref = BigBirdSelfAttention(H * 64, H).double()
+    ref.load_state_dict({n: t.detach().cpu().double() for n, t in mod.state_dict().items()})
+    x = torch.randn(B, L, H * 64).to(torch.bfloat16)
+    km = torch.ones(B, L, dtype=torch.uint8)
+    km[1, -40:] = 0
+    xg = x.to(dev).requires_grad_(True)
+    y = mod(xg, key_mask=km.to(dev))
+    (y.float().square().sum() * 0.5).backward()
+    assert bsa.bsa_sync_status() == 0
+    lay = OL.build_layout(H, L, 64, 1, 2, 2, 3)
+    xr = x.double().requires_grad_(True)
+    y_ref = _dense_reference(ref, xr, lay, km.numpy())
+    scale = y_ref.abs().max().item()
+    err = (y.detach().cpu().double() - y_ref).abs().max().item()
+    assert err <= 2e-2 * scale, (err, scale)
+    # the loss gradient dy = y of each side's own output, so the checks below
+    # also carry the forward's rounding
+    y_ref.backward(y_ref.detach())
+    for got, want, name in ((xg.grad, xr.grad, "x"),
+                            (mod.qkv.weight.grad, ref.qkv.weight.grad, "qkv.weight"),
+                            (mod.qkv.bias.grad, ref.qkv.bias.grad, "qkv.bias"),
+                            (mod.proj.weight.grad, ref.proj.weight.grad, "proj.weight"),
+                            (mod.proj.bias.grad, ref.proj.bias.grad, "proj.bias")):
+        g = got.detach().cpu().double()
+        assert torch.isfinite(g).all(), name
+        m = want.abs().max().item()
+        e = (g - want).abs().max().item()
+        assert e <= 5e-2 * m, (name, e, m)

@@ -172,3 +172,48 @@ def test_head_shard_rows_and_two_gloo_ranks_reproduce_single_process():
     assert [s[:2] for s in shards] == [(0, 3), (3, 5)]
     assert np.array_equal(np.concatenate([s[2] for s in shards], axis=1), o_ref)
     assert np.array_equal(np.concatenate([s[3] for s in shards], axis=1), lse_ref)
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_sharded_layouts_on_the_gpu_reproduce_the_full_run(world):
+    """The work each rank of a head-sharded job does, run shard after shard on one
+    GPU: every rank builds its layout from its heads' CSR rows
+    (sharding.head_rows -> bsa_layout_from_csr) and runs the forward and the
+    backward on its heads' slices.  Put back together, the shards equal the
+    single-layout run bit for bit (a head's tiles, entries and schedule do not
+    depend on the other heads) and the fp64 oracle within the parity tolerances."""
+    from block_sparse_attention_bigbird_b200 import bsa
+    from test_backward import _check_grads
+    from test_gpu_parity import _check
+    # global query rows long enough to be split into chunks, and a padded key tail
+    w = workloads.custom(2, 5, 64 * 64, 1, 2, 3, seed=9, key_pad_tail=30)
+    qc, kc, vc = workloads.make_qkv(w)
+    doc = workloads.make_grad(w, seed=100)
+    kmc = workloads.make_key_mask(w)
+    dev = torch.device("cuda")
+    q, k, v, do, km = (t.to(dev) for t in (qc, kc, vc, doc, kmc))
+    full = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(full)
+    o_full, lse_full = bsa.bsa_forward(q, k, v, full, key_mask=km)
+    g_full = bsa.bsa_backward(q, k, v, o_full, do, lse_full, full, key_mask=km)
+    rp, ci = bsa.bsa_layout_csr(full)
+    outs = []
+    for rank in range(world):
+        h0, h1 = sharding.head_shard(w.H, rank, world)
+        srp, sci = sharding.head_rows(rp, ci, w.nb, h0, h1)
+        mine = bsa.bsa_layout_from_csr(h1 - h0, w.L, srp, sci)
+        bsa.bsa_layout_upload(mine)
+        qs, ks, vs, dos = (t[:, h0:h1].contiguous() for t in (q, k, v, do))
+        o, lse = bsa.bsa_forward(qs, ks, vs, mine, key_mask=km)
+        outs.append((o, lse) + tuple(bsa.bsa_backward(qs, ks, vs, o, dos, lse, mine, key_mask=km)))
+    assert bsa.bsa_sync_status() == 0
+    got = [torch.cat([s[i] for s in outs], dim=1) for i in range(5)]
+    for a, b in zip(got, (o_full, lse_full) + tuple(g_full)):
+        assert torch.equal(a, b)
+    ref = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    o_ref, lse_ref = OA.attention(qc, kc, vc, ref, key_mask=kmc)
+    _check(got[0].float().cpu().numpy(), got[1].cpu().numpy(), o_ref, lse_ref)
+    dq, dk, dv, mags = OB.attention_backward(qc, kc, vc, doc, ref, key_mask=kmc, with_magnitude=True)
+    _check_grads([t.float().cpu().numpy() for t in got[2:]], (dq, dk, dv), mags)
