@@ -151,7 +151,6 @@ struct FwdParams {
   float* partials;
   int* sched;  // [0] next work item, [1] slots finished; cleared before each launch
   int B, H, L, nb, items_per_batch, n_split, n_records;
-  int split_items;  // the first split_items items of a batch element are split-tile chunks
   float scale_log2;
   unsigned long long timeout_ns;
 };
@@ -232,19 +231,11 @@ __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, i
     // stage the item for the slot's other roles
     ItemStage& st = sl.items[ii];
     if (t >= 0) {
-      // t enumerates (batch element, item): first the split-tile chunks of every
-      // batch element (the longest items, kept away from the end of the run), then
-      // the other tiles batch element by batch element (its K/V stay in L2)
-      const int ns = p.split_items;
-      int b, i;
-      if (t < p.B * ns) {
-        i = t / p.B;
-        b = t - i * p.B;
-      } else {
-        const int nn = p.items_per_batch - ns, u = t - p.B * ns;
-        b = u / nn;
-        i = ns + (u - b * nn);
-      }
+      // t enumerates (batch element, item), batch element by batch element so that
+      // its K/V stay in L2 while its items run; within one, the split-tile chunks
+      // (the longest items, which read every key block of their head) come first
+      const int b = t / p.items_per_batch;
+      const int i = t - b * p.items_per_batch;
       const WorkItem w = p.items[i];
       for (int e = lane; e < w.count; e += 32) {
         const uint32_t en = p.pair_ent[w.start + e];
@@ -1018,8 +1009,6 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
   prm.items_per_batch = static_cast<int>(lay->items.size());
   prm.n_split = lay->n_split;
   prm.n_records = lay->n_records;
-  prm.split_items = static_cast<int>(std::count_if(lay->items.begin(), lay->items.end(),
-                                                   [](const WorkItem& it) { return it.split >= 0; }));
   const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(d));
   prm.scale_log2 = sc * kLog2e;
   prm.timeout_ns = kDefaultTimeoutNs;

@@ -286,10 +286,10 @@ void build_tiles(bsa_layout* lay, const std::vector<uint8_t>& dense) {
   make_tiles(H, nb, lay->row_ptr, lay->col_idx, dense, &lay->pair_q, &lay->n_pairs, &lay->pair_ptr,
              &lay->pair_ent);
   const int P = lay->n_pairs;
-  // Work items of one batch element: first the chunks of split tiles (the forward
-  // hands these out first, for the whole batch: they are the longest items), then
-  // the other tiles, head-major so that items running at the same time share the
-  // head's K/V in L2.
+  // Work items of one batch element: first the chunks of split tiles (the longest
+  // items, kept away from the end of the element's run), then the other tiles,
+  // head-major so that items running at the same time share the head's K/V in L2.
+  // The forward hands out every item of one batch element before the next one's.
   lay->items.clear();
   lay->splits.clear();
   lay->n_split = 0;
