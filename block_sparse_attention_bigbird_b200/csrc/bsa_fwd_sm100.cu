@@ -77,6 +77,7 @@ constexpr uint32_t kTmemO = 0;       // O: 64 fp32 columns
 constexpr uint32_t kTmemS = 64;      // S: 128 fp32 columns
 constexpr uint32_t kTmemP = 192;     // P: 128 keys as 64 bf16 pairs
 constexpr float kRescaleLog2 = 8.0f;  // m is raised when a chunk's max exceeds it by more
+constexpr float kRescaleBound = 256.0f;  // 2^kRescaleLog2
 constexpr uint32_t kOStageBytes = 32 * 128;  // one warp's 32 O rows, staged for a TMA store
 static_assert(kTmemS + 128 <= kTmemP && kTmemP + 64 <= kSlotCols, "TMEM map");
 
@@ -606,52 +607,70 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         break;
       }
       ptx::tc_fence_after();
-      // all of S(g) into registers; the S columns go straight back to the S issuer
+      // All of S(g) into registers (loaded whatever the membership: a load under a
+      // condition makes the compiler keep both versions of the registers alive).
+      //
+      // The running max m follows one rule: it is raised to the chunk max cm when cm
+      // exceeds it by more than kRescaleLog2, so every p = 2^(s - m) stays at or below
+      // 2^kRescaleLog2.  The chunk max itself is needed only on a row's first attended
+      // chunk (m = -inf) or when some p could pass that bound; so a chunk first takes its
+      // exponentials with m as it stands, and only when some row's sum of p exceeds
+      // 2^kRescaleLog2 (the one case where a single p may) is S loaded again, its max
+      // taken and the chunk redone.  m, p and l come out as with the max taken every
+      // time (up to a score within rounding of the bound).  A warp's rows share
+      // membership and key bits, so the branches are warp-uniform.  The S columns go
+      // back to the S issuer once the chunk stands.
       const uint32_t sbase = tmem + lane_addr + kTmemS;
-      // (loaded whatever the membership: a load under a condition makes the compiler keep
-      // both versions of the registers alive)
-      uint32_t a0[32], b0[32], a1[32], b1[32];
-      ptx::tmem_ld32(sbase, a0);
-      ptx::tmem_ld32(sbase + 32u, b0);
-      ptx::tmem_ld32(sbase + 64u, a1);
-      ptx::tmem_ld32(sbase + 96u, b1);
-      ptx::tmem_wait_ld();
-      ptx::reg_fence(a0);
-      ptx::reg_fence(b0);
-      ptx::reg_fence(a1);
-      ptx::reg_fence(b1);
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(kBarSFree));
       // the next chunk's masks, while this one computes
       const unsigned long long nmk0 = e0 + 2 < count ? entry_mask(st, e0 + 2, half) : 0ull;
       const unsigned long long nmk1 = e0 + 3 < count ? entry_mask(st, e0 + 3, half) : 0ull;
-      // keys dropped by the padding mask inside an attended block (rare)
-      if (((mk0 + 1ull) > 1ull) || ((mk1 + 1ull) > 1ull)) {  // some mask neither 0 nor all ones
-        if (mk0 != 0ull) mask_group(a0, b0, mk0);
-        if (mk1 != 0ull) mask_group(a1, b1, mk1);
-      }
-      // chunk max over the keys this row attends (mk != 0 keeps at least one key); the
-      // running max is raised only past it by more than 2^kRescaleLog2
-      const float gm0 = group_max(a0, b0), gm1 = group_max(a1, b1);
-      const float cm = fmaxf(mk0 != 0ull ? gm0 : -INFINITY, mk1 != 0ull ? gm1 : -INFINITY);
-      const float cm2 = cm * sl2;  // scale > 0: the max of the scaled scores
-      const float m_new = cm2 > m_run + kRescaleLog2 ? cm2 : m_run;
-      const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
+      float m_new = m_run;
+      bool take_max = __any_sync(0xffffffffu, m_run == -INFINITY);
       uint32_t pk0[32], pk1[32];
-      float psum = 0.f;
-      if (mk0 != 0ull) {
-        psum += group_exp(a0, b0, sc2, nm2, pk0);
-      } else {
+      float psum;
+      for (;;) {
+        uint32_t a0[32], b0[32], a1[32], b1[32];
+        ptx::tmem_ld32(sbase, a0);
+        ptx::tmem_ld32(sbase + 32u, b0);
+        ptx::tmem_ld32(sbase + 64u, a1);
+        ptx::tmem_ld32(sbase + 96u, b1);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence(a0);
+        ptx::reg_fence(b0);
+        ptx::reg_fence(a1);
+        ptx::reg_fence(b1);
+        // keys dropped by the padding mask inside an attended block (rare)
+        if (((mk0 + 1ull) > 1ull) || ((mk1 + 1ull) > 1ull)) {  // some mask neither 0 nor all ones
+          if (mk0 != 0ull) mask_group(a0, b0, mk0);
+          if (mk1 != 0ull) mask_group(a1, b1, mk1);
+        }
+        if (take_max) {  // the chunk max over the keys this row attends (mk != 0 keeps one)
+          const float gm0 = group_max(a0, b0), gm1 = group_max(a1, b1);
+          const float cm = fmaxf(mk0 != 0ull ? gm0 : -INFINITY, mk1 != 0ull ? gm1 : -INFINITY);
+          const float cm2 = cm * sl2;  // scale > 0: the max of the scaled scores
+          m_new = cm2 > m_run + kRescaleLog2 ? cm2 : m_run;
+        }
+        const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
+        psum = 0.f;
+        if (mk0 != 0ull) {
+          psum += group_exp(a0, b0, sc2, nm2, pk0);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk0[c] = 0u;
-      }
-      if (mk1 != 0ull) {
-        psum += group_exp(a1, b1, sc2, nm2, pk1);
-      } else {
+          for (int c = 0; c < 32; ++c) pk0[c] = 0u;
+        }
+        if (mk1 != 0ull) {
+          psum += group_exp(a1, b1, sc2, nm2, pk1);
+        } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk1[c] = 0u;
+          for (int c = 0; c < 32; ++c) pk1[c] = 0u;
+        }
+        // every p <= psum: a sum within the bound keeps m (a NaN sum takes the max path)
+        if (take_max || !__any_sync(0xffffffffu, !(psum <= kRescaleBound))) break;
+        take_max = true;
       }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar(kBarSFree));
       const bool grew = m_new != m_run;
       const float alpha = grew ? ptx::ex2_approx(m_run - m_new) : 1.f;  // 2^-inf = 0
       const bool rescale = grew && l_run > 0.f;  // O holds this tile's earlier chunks
