@@ -112,6 +112,7 @@ constexpr uint32_t kWarpArrivals = 4;  // barriers the four softmax warps arrive
 constexpr int kMaxItemEntries = 64;
 static_assert(kSplitThreshold <= kMaxItemEntries && kSplitChunk <= kMaxItemEntries,
               "an item's entries must fit its stage");
+static_assert(kMaxItemEntries <= 64, "a softmax warp keeps an item's entry bits in two 32-lane ballots");
 struct ItemStage {
   int t;  // work item index, or kItemNone
   int qa, qb;
@@ -485,7 +486,7 @@ __device__ __noinline__ void tile_epilogue(const FwdParams& p, const TileDone& t
                           static_cast<int>(row - static_cast<size_t>(r & 31)));
         ptx::bulk_commit_group();
       }
-      p.lse[row] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+      p.lse[row] = l > 0.f ? (m + ptx::lg2_approx(l)) * kLn2 : -INFINITY;
     }
     return;
   }
@@ -594,8 +595,18 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
     const int count = st.w.count;
     float m_run = -INFINITY, l_run = 0.f;
     // masks of the chunk's two entries, read one chunk ahead
-    unsigned long long mk0 = entry_mask(st, 0, half);
-    unsigned long long mk1 = count >= 2 ? entry_mask(st, 1, half) : 0ull;
+    // Per union entry, one bit each: this half attends the entry's key block and not all
+    // of its keys are padded (att), and some of them are (part).  Lane x looks at entries
+    // x and x + 32 (an item has at most 64), and the warp's ballots hold the bits.
+    uint64_t att_bits, part_bits;
+    {
+      const unsigned long long k0 = lane < count ? entry_mask(st, lane, half) : 0ull;
+      const unsigned long long k1 = lane + 32 < count ? entry_mask(st, lane + 32, half) : 0ull;
+      att_bits = static_cast<uint64_t>(__ballot_sync(0xffffffffu, k0 != 0ull)) |
+                 (static_cast<uint64_t>(__ballot_sync(0xffffffffu, k1 != 0ull)) << 32);
+      part_bits = static_cast<uint64_t>(__ballot_sync(0xffffffffu, k0 + 1ull > 1ull)) |
+                  (static_cast<uint64_t>(__ballot_sync(0xffffffffu, k1 + 1ull > 1ull)) << 32);
+    }
     for (int e0 = 0; e0 < count; e0 += kChunkEnt, ++g) {
       if (q_pending && e0 > 0) {  // one chunk after the epilogue: its O store has had time
         q_pending = false;
@@ -622,8 +633,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       // back to the S issuer once the chunk stands.
       const uint32_t sbase = tmem + lane_addr + kTmemS;
       // the next chunk's masks, while this one computes
-      const unsigned long long nmk0 = e0 + 2 < count ? entry_mask(st, e0 + 2, half) : 0ull;
-      const unsigned long long nmk1 = e0 + 3 < count ? entry_mask(st, e0 + 3, half) : 0ull;
+      const bool att0 = (att_bits >> e0) & 1ull, att1 = (att_bits >> (e0 + 1)) & 1ull;
+      const bool part = ((part_bits >> e0) & 3ull) != 0ull;
       float m_new = m_run;
       bool take_max = __any_sync(0xffffffffu, m_run == -INFINITY);
       uint32_t pk0[32], pk1[32];
@@ -640,25 +651,25 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         ptx::reg_fence(a1);
         ptx::reg_fence(b1);
         // keys dropped by the padding mask inside an attended block (rare)
-        if (((mk0 + 1ull) > 1ull) || ((mk1 + 1ull) > 1ull)) {  // some mask neither 0 nor all ones
-          if (mk0 != 0ull) mask_group(a0, b0, mk0);
-          if (mk1 != 0ull) mask_group(a1, b1, mk1);
+        if (part) {  // an attended key block with some padded keys (rare)
+          if (att0) mask_group(a0, b0, entry_mask(st, e0, half));
+          if (att1) mask_group(a1, b1, entry_mask(st, e0 + 1, half));
         }
         if (take_max) {  // the chunk max over the keys this row attends (mk != 0 keeps one)
           const float gm0 = group_max(a0, b0), gm1 = group_max(a1, b1);
-          const float cm = fmaxf(mk0 != 0ull ? gm0 : -INFINITY, mk1 != 0ull ? gm1 : -INFINITY);
+          const float cm = fmaxf(att0 ? gm0 : -INFINITY, att1 ? gm1 : -INFINITY);
           const float cm2 = cm * sl2;  // scale > 0: the max of the scaled scores
           m_new = cm2 > m_run + kRescaleLog2 ? cm2 : m_run;
         }
         const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
         psum = 0.f;
-        if (mk0 != 0ull) {
+        if (att0) {
           psum += group_exp(a0, b0, sc2, nm2, pk0);
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) pk0[c] = 0u;
         }
-        if (mk1 != 0ull) {
+        if (att1) {
           psum += group_exp(a1, b1, sc2, nm2, pk1);
         } else {
 #pragma unroll
@@ -709,8 +720,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(bar(kBarPFull));
-      mk0 = nmk0;
-      mk1 = nmk1;
     }
     if (!alive) break;
     if (q_pending) {  // a one-chunk tile: release before the next item's loads need the buffer
