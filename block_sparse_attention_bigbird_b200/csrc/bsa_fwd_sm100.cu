@@ -96,8 +96,8 @@ enum : int {
   kBarVFree = kBarVFull + kVStages,  // [V stage] MMA commit after the chunk's PV: the V stage
                                      // and the P columns are reusable, O holds chunk g
   kBarSFull = kBarVFree + kVStages,  // MMA commit after S: the S columns are readable
-  kBarSFree = kBarSFull + 1,         // 4 softmax warps have loaded S
-  kBarPFull = kBarSFree + 1,         // 4 softmax warps have stored P
+  kBarSFree = kBarSFull + 1,         // the 128 softmax threads are done with S
+  kBarPFull = kBarSFree + 1,         // the 128 softmax threads have stored P
   kBarMmaFinal = kBarPFull + 1,      // [2 issuers]
   kBarItemFull = kBarMmaFinal + 2,   // [item ring] the K producer published a work item
   kBarItemEmpty = kBarItemFull + kItemRing,  // [item ring] 7 arrivals: V producer, both
@@ -105,7 +105,8 @@ enum : int {
   kNumBars = kBarItemEmpty + kItemRing
 };
 constexpr uint32_t kItemReaders = 7;
-constexpr uint32_t kWarpArrivals = 4;  // barriers the four softmax warps arrive on once each
+constexpr uint32_t kWarpArrivals = 4;     // Q release: one arrival per softmax warp
+constexpr uint32_t kThreadArrivals = 128;  // S free, P full: every softmax thread arrives
 
 // One published work item in shared memory: its index, its fields, its query-block
 // pair and, per union entry, the entry and the key-padding bits of its key block.
@@ -518,6 +519,36 @@ __device__ __forceinline__ void mask_group(uint32_t (&a)[32], uint32_t (&b)[32],
   }
 }
 
+// Rare paths, out of line so that the chunk loop's code stays small (softmax warps only).
+// Scores of padded keys of one 64-key group of this warp's rows set to -inf in TMEM.
+__device__ __noinline__ void mask_scores(uint32_t taddr, unsigned long long mk) {
+  uint32_t a[32], b[32];
+  ptx::tmem_ld32(taddr, a);
+  ptx::tmem_ld32(taddr + 32u, b);
+  ptx::tmem_wait_ld();
+  ptx::reg_fence(a);
+  ptx::reg_fence(b);
+  mask_group(a, b, mk);
+  ptx::tmem_st32(taddr, a);
+  ptx::tmem_st32(taddr + 32u, b);
+  ptx::tmem_wait_st();
+}
+
+// O (64 columns of this warp's rows) scaled by alpha in TMEM; the caller's next
+// tcgen05.wait::st covers the stores.
+__device__ __noinline__ void rescale_o(uint32_t obase, float alpha) {
+#pragma unroll
+  for (int hlf = 0; hlf < 2; ++hlf) {
+    uint32_t o[32];
+    ptx::tmem_ld32(obase + 32u * hlf, o);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence(o);
+#pragma unroll
+    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+    ptx::tmem_st32(obase + 32u * hlf, o);
+  }
+}
+
 __device__ __forceinline__ float group_max(const uint32_t (&a)[32], const uint32_t (&b)[32]) {
   auto f = [](uint32_t x) { return __uint_as_float(x); };
   // four independent chains of three-input maxima
@@ -594,7 +625,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
     const ItemStage& st = sl.items[k % kItemRing];
     const int count = st.w.count;
     float m_run = -INFINITY, l_run = 0.f;
-    // masks of the chunk's two entries, read one chunk ahead
     // Per union entry, one bit each: this half attends the entry's key block and not all
     // of its keys are padded (att), and some of them are (part).  Lane x looks at entries
     // x and x + 32 (an item has at most 64), and the warp's ballots hold the bits.
@@ -632,9 +662,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       // membership and key bits, so the branches are warp-uniform.  The S columns go
       // back to the S issuer once the chunk stands.
       const uint32_t sbase = tmem + lane_addr + kTmemS;
-      // the next chunk's masks, while this one computes
       const bool att0 = (att_bits >> e0) & 1ull, att1 = (att_bits >> (e0 + 1)) & 1ull;
       const bool part = ((part_bits >> e0) & 3ull) != 0ull;
+      if (part) {  // an attended key block with some padded keys (rare): -inf in TMEM
+        if (att0) mask_scores(sbase, entry_mask(st, e0, half));
+        if (att1) mask_scores(sbase + 64u, entry_mask(st, e0 + 1, half));
+      }
       float m_new = m_run;
       bool take_max = __any_sync(0xffffffffu, m_run == -INFINITY);
       uint32_t pk0[32], pk1[32];
@@ -650,11 +683,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         ptx::reg_fence(b0);
         ptx::reg_fence(a1);
         ptx::reg_fence(b1);
-        // keys dropped by the padding mask inside an attended block (rare)
-        if (part) {  // an attended key block with some padded keys (rare)
-          if (att0) mask_group(a0, b0, entry_mask(st, e0, half));
-          if (att1) mask_group(a1, b1, entry_mask(st, e0 + 1, half));
-        }
         if (take_max) {  // the chunk max over the keys this row attends (mk != 0 keeps one)
           const float gm0 = group_max(a0, b0), gm1 = group_max(a1, b1);
           const float cm = fmaxf(att0 ? gm0 : -INFINITY, att1 ? gm1 : -INFINITY);
@@ -680,8 +708,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         take_max = true;
       }
       ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(kBarSFree));
+      ptx::mbar_arrive(bar(kBarSFree));  // every thread
       const bool grew = m_new != m_run;
       const float alpha = grew ? ptx::ex2_approx(m_run - m_new) : 1.f;  // 2^-inf = 0
       const bool rescale = grew && l_run > 0.f;  // O holds this tile's earlier chunks
@@ -699,18 +726,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         q_pending = true;
         q_k = pend.k;
       }
-      if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-          uint32_t o[32];
-          ptx::tmem_ld32(obase + 32u * hlf, o);
-          ptx::tmem_wait_ld();
-          ptx::reg_fence(o);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          ptx::tmem_st32(obase + 32u * hlf, o);
-        }
-      }
+      if (__any_sync(0xffffffffu, rescale)) rescale_o(obase, alpha);
       const uint32_t pbase = tmem + lane_addr + kTmemP;
       ptx::tmem_st32(pbase, pk0);
       if (two) ptx::tmem_st32(pbase + 32u, pk1);
@@ -718,8 +734,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       m_run = m_new;
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar(kBarPFull));
+      ptx::mbar_arrive(bar(kBarPFull));  // every thread
     }
     if (!alive) break;
     if (q_pending) {  // a one-chunk tile: release before the next item's loads need the buffer
@@ -751,7 +766,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
       const uint32_t bars = base + s * kSlotBytes + kSmemBar;
       for (int i = 0; i < kNumBars; ++i) {
         uint32_t count = 1;
-        if ((i >= kBarQEmpty && i < kBarQEmpty + 2) || i == kBarSFree || i == kBarPFull) count = kWarpArrivals;
+        if (i >= kBarQEmpty && i < kBarQEmpty + 2) count = kWarpArrivals;
+        if (i == kBarSFree || i == kBarPFull) count = kThreadArrivals;
         if (i >= kBarItemEmpty && i < kBarItemEmpty + kItemRing) count = kItemReaders;
         ptx::mbar_init(bars + 8u * i, count);
       }

@@ -9,6 +9,10 @@ one set of P columns (PFull, released with the V stage by the PV commit), and O,
 whose epilogue runs in the first chunk of the next tile and stages its rows in
 the finished tile's Q buffer.
 
+SFree and PFull take one arrival from every softmax thread; a warp's 32 arrivals
+follow its own TMEM accesses in program order, so the model counts one arrival
+per warp.
+
 The test replays the roles' sequences under random interleavings, for random
 work lists, with every asynchronous copy and MMA landing at a random later
 moment, and asserts
