@@ -154,6 +154,8 @@ struct FwdParams {
   float* partials;
   int* sched;  // [0] next work item, [1] slots finished; cleared before each launch
   int B, H, L, nb, items_per_batch, n_split, n_records;
+  int split_items;  // the first split_items items of a batch element are split-tile chunks
+  int split_lead;   // split chunks are handed out this many batch elements early
   float scale_log2;
   unsigned long long timeout_ns;
 };
@@ -206,6 +208,30 @@ __device__ __forceinline__ void drain_ring(uint32_t bars, int first_bar, uint32_
   }
 }
 
+// The order in which work items are handed out: t -> (batch element, item).  A batch
+// element's items are its ns split-tile chunks (the longest items: each reads every key
+// block of its head), then its nn other tiles.  Elements follow one another, so that one
+// element's K/V stay in L2 while its items run, except that the split chunks of element
+// b are handed out d elements early, at the start of element b - d's items (elements
+// 0..d's at the very start), so that no long item starts near the end of the run.  The
+// host picks d from the item lengths; d = 0 is the plain element-after-element order.
+__host__ __device__ __forceinline__ int2 item_of(int t, int B, int ns, int nn, int d) {
+  const int per = ns + nn;
+  if (d == 0 || ns == 0) return make_int2(t / per, t - (t / per) * per);
+  if (t < (d + 1) * ns) return make_int2(t / ns, t - (t / ns) * ns);  // chunks of elements 0..d
+  t -= (d + 1) * ns;
+  if (t < nn) return make_int2(0, ns + t);  // element 0's other tiles
+  t -= nn;
+  const int full = B - 1 - d;  // elements 1..B-1-d: chunks of element j + d, tiles of j
+  if (t < full * per) {
+    const int j = 1 + t / per, u = t - (j - 1) * per;
+    return u < ns ? make_int2(j + d, u) : make_int2(j, u);
+  }
+  t -= full * per;  // elements B-d..B-1: tiles only
+  const int j = B - d + t / nn;
+  return make_int2(j, ns + (t - (j - (B - d)) * nn));
+}
+
 // K producer, one warp.  Per work item the warp stages the item, its union entries and
 // their key-padding bits in the slot's item ring; then lane 0 issues the loads: the Q
 // tile into Q buffer (tile % 2) once the tile two back has released it, and for each
@@ -234,11 +260,8 @@ __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, i
     // stage the item for the slot's other roles
     ItemStage& st = sl.items[ii];
     if (t >= 0) {
-      // t enumerates (batch element, item), batch element by batch element so that
-      // its K/V stay in L2 while its items run; within one, the split-tile chunks
-      // (the longest items, which read every key block of their head) come first
-      const int b = t / p.items_per_batch;
-      const int i = t - b * p.items_per_batch;
+      const int2 bi = item_of(t, p.B, p.split_items, p.items_per_batch - p.split_items, p.split_lead);
+      const int b = bi.x, i = bi.y;
       const WorkItem w = p.items[i];
       for (int e = lane; e < w.count; e += 32) {
         const uint32_t en = p.pair_ent[w.start + e];
@@ -1051,6 +1074,8 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
   prm.L = L;
   prm.nb = lay->nb;
   prm.items_per_batch = static_cast<int>(lay->items.size());
+  prm.split_items = static_cast<int>(std::count_if(lay->items.begin(), lay->items.end(),
+                                                   [](const WorkItem& it) { return it.split >= 0; }));
   prm.n_split = lay->n_split;
   prm.n_records = lay->n_records;
   const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(d));
@@ -1068,6 +1093,20 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
   // two slots per CTA; items are drawn dynamically
   const int grid = static_cast<int>(std::min<int64_t>((total + kSlots - 1) / kSlots, c.info.sms));
   if (grid < 1) return BSA_OK;
+  // How many batch elements early the split chunks go out: the last element's must
+  // start while each slot still has at least one such chunk's length of work ahead.
+  prm.split_lead = 0;
+  if (prm.split_items > 0 && B > 1) {
+    int64_t work = 0;  // chunks of one batch element
+    int longest = 0;
+    for (const WorkItem& it : lay->items) {
+      const int ch = (it.count + kChunkEnt - 1) / kChunkEnt;
+      work += ch;
+      if (it.split >= 0) longest = std::max(longest, ch);
+    }
+    const int64_t slots = static_cast<int64_t>(kSlots) * grid;
+    while (prm.split_lead < B - 1 && (prm.split_lead + 1) * work < longest * slots) ++prm.split_lead;
+  }
   bsa_fwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   if (lay->n_split > 0) {
