@@ -491,16 +491,20 @@ __device__ __noinline__ void tile_epilogue(const FwdParams& p, const TileDone& t
       // O rows through this warp's quarter of the tile's Q buffer (128-byte swizzle:
       // 16-byte chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)), then one TMA store
       // of the warp's 32 x 64 tile.
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? ptx::rcp_approx(l) : 0.f;
+      const uint64_t inv2 = ptx::pack2(inv, inv);
       const uint32_t qs = td.k & 1u;
       uint8_t* stg = sl.q_generic + qs * kQBytes + (warp & 3) * kOStageBytes;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        uint4 u;
-        u.x = pack_bf16x2(o[8 * j + 0] * inv, o[8 * j + 1] * inv);
-        u.y = pack_bf16x2(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-        u.z = pack_bf16x2(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-        u.w = pack_bf16x2(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
+        uint32_t w4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float y0, y1;
+          ptx::unpack2(ptx::fmul2(ptx::pack2(o[8 * j + 2 * q], o[8 * j + 2 * q + 1]), inv2), y0, y1);
+          w4[q] = pack_bf16x2(y0, y1);
+        }
+        const uint4 u = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) = u;
       }
       ptx::fence_proxy_async_smem();
@@ -572,6 +576,16 @@ __device__ __noinline__ void rescale_o(uint32_t obase, float alpha) {
   }
 }
 
+// Zeros 32 TMEM columns of this warp's rows (the P of a group this half does not
+// attend): eight four-column stores from one zero register, instead of 32 registers
+// set to zero for one wide store.
+__device__ __forceinline__ void tmem_zero32(uint32_t taddr) {
+  const uint32_t z = 0u;
+#pragma unroll
+  for (int i = 0; i < 32; i += 4)
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %1, %1, %1};" ::"r"(taddr + i), "r"(z) : "memory");
+}
+
 __device__ __forceinline__ float group_max(const uint32_t (&a)[32], const uint32_t (&b)[32]) {
   auto f = [](uint32_t x) { return __uint_as_float(x); };
   // four independent chains of three-input maxima
@@ -590,8 +604,8 @@ __device__ __forceinline__ float group_max(const uint32_t (&a)[32], const uint32
 // p = 2^(s * scale_log2 - m) for the 64 scores of one group (keys 0-31 in a, 32-63 in
 // b), packed to bf16 pairs in key order; returns the fp32 sum of p.  The scaling and
 // the sums run on packed fp32 pairs (two lanes per instruction).
-__device__ __forceinline__ float group_exp(const uint32_t (&a)[32], const uint32_t (&b)[32], uint64_t sc2,
-                                           uint64_t nm2, uint32_t (&pk)[32]) {
+__device__ __forceinline__ float group_exp(uint32_t (&a)[32], const uint32_t (&b)[32], uint64_t sc2,
+                                           uint64_t nm2) {
   uint64_t acc0 = 0ull, acc1 = 0ull;
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
@@ -604,7 +618,7 @@ __device__ __forceinline__ float group_exp(const uint32_t (&a)[32], const uint32
       acc1 = ptx::fadd2(acc1, ptx::pack2(p0, p1));
     else
       acc0 = ptx::fadd2(acc0, ptx::pack2(p0, p1));
-    pk[c] = pack_bf16x2(p0, p1);
+    a[c] = pack_bf16x2(p0, p1);  // in place: a[c] was read at step c / 2
   }
   float s0, s1;
   ptx::unpack2(ptx::fadd2(acc0, acc1), s0, s1);
@@ -693,10 +707,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       }
       float m_new = m_run;
       bool take_max = __any_sync(0xffffffffu, m_run == -INFINITY);
-      uint32_t pk0[32], pk1[32];
+      // P is written over the scores it came from (a0 and a1 hold P after the
+      // exponentials), so that the TMEM stores read the registers the loads wrote
+      uint32_t a0[32], b0[32], a1[32], b1[32];
       float psum;
       for (;;) {
-        uint32_t a0[32], b0[32], a1[32], b1[32];
         ptx::tmem_ld32(sbase, a0);
         ptx::tmem_ld32(sbase + 32u, b0);
         ptx::tmem_ld32(sbase + 64u, a1);
@@ -715,16 +730,10 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
         psum = 0.f;
         if (att0) {
-          psum += group_exp(a0, b0, sc2, nm2, pk0);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pk0[c] = 0u;
+          psum += group_exp(a0, b0, sc2, nm2);
         }
         if (att1) {
-          psum += group_exp(a1, b1, sc2, nm2, pk1);
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pk1[c] = 0u;
+          psum += group_exp(a1, b1, sc2, nm2);
         }
         // every p <= psum: a sum within the bound keeps m (a NaN sum takes the max path)
         if (take_max || !__any_sync(0xffffffffu, !(psum <= kRescaleBound))) break;
@@ -751,8 +760,10 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       }
       if (__any_sync(0xffffffffu, rescale)) rescale_o(obase, alpha);
       const uint32_t pbase = tmem + lane_addr + kTmemP;
-      ptx::tmem_st32(pbase, pk0);
-      if (two) ptx::tmem_st32(pbase + 32u, pk1);
+      if (att0) ptx::tmem_st32(pbase, a0); else tmem_zero32(pbase);
+      if (two) {
+        if (att1) ptx::tmem_st32(pbase + 32u, a1); else tmem_zero32(pbase + 32u);
+      }
       l_run = l_run * alpha + psum;
       m_run = m_new;
       ptx::tmem_wait_st();
