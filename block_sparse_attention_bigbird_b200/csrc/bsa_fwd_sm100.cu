@@ -263,13 +263,47 @@ __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, i
       const int2 bi = item_of(t, p.B, p.split_items, p.items_per_batch - p.split_items, p.split_lead);
       const int b = bi.x, i = bi.y;
       const WorkItem w = p.items[i];
-      for (int e = lane; e < w.count; e += 32) {
-        const uint32_t en = p.pair_ent[w.start + e];
-        st.ent[e] = en;
-        st.kb[e] = p.keybits != nullptr ? p.keybits[static_cast<size_t>(b) * p.nb + (en & kEntColMask)] : ~0ull;
+      int kept = w.count;
+      if (p.keybits == nullptr) {
+        for (int e = lane; e < w.count; e += 32) {
+          st.ent[e] = p.pair_ent[w.start + e];
+          st.kb[e] = ~0ull;
+        }
+      } else {
+        // Entries whose 64 keys are all padded are dropped here, so that no load or MMA
+        // is issued for them.  Lane x looks at entries x and x + 32 (at most 64); the
+        // kept ones are packed in order.  If none is kept, entry 0 stays with no
+        // membership bits: its P is zero and the tile's rows are still written.
+        const bool h0 = lane < w.count, h1 = lane + 32 < w.count;
+        const uint32_t en0 = h0 ? p.pair_ent[w.start + lane] : 0u;
+        const uint32_t en1 = h1 ? p.pair_ent[w.start + lane + 32] : 0u;
+        const unsigned long long* kbb = p.keybits + static_cast<size_t>(b) * p.nb;
+        const unsigned long long kb0 = h0 ? kbb[en0 & kEntColMask] : 0ull;
+        const unsigned long long kb1 = h1 ? kbb[en1 & kEntColMask] : 0ull;
+        const uint32_t keep0 = __ballot_sync(0xffffffffu, kb0 != 0ull);
+        const uint32_t keep1 = __ballot_sync(0xffffffffu, kb1 != 0ull);
+        const uint32_t below = (1u << lane) - 1u;
+        const int n0 = __popc(keep0);
+        kept = n0 + __popc(keep1);
+        if (kb0 != 0ull) {
+          st.ent[__popc(keep0 & below)] = en0;
+          st.kb[__popc(keep0 & below)] = kb0;
+        }
+        if (kb1 != 0ull) {
+          st.ent[n0 + __popc(keep1 & below)] = en1;
+          st.kb[n0 + __popc(keep1 & below)] = kb1;
+        }
+        if (kept == 0) {
+          if (lane == 0) {
+            st.ent[0] = en0 & kEntColMask;
+            st.kb[0] = 0ull;
+          }
+          kept = 1;
+        }
       }
       if (lane == 0) {
         st.w = w;
+        st.w.count = kept;
         st.b = b;
         st.qa = p.pair_q[2 * w.pair];
         st.qb = p.pair_q[2 * w.pair + 1];
