@@ -123,6 +123,21 @@ def _nnz_eff(w, row_ptr, col_idx) -> int:
     return w.B * per_batch
 
 
+def _mma_useful_frac(w, lay, nnz_eff) -> float:
+    """Useful non-zero blocks / 64x64 block-equivalents the forward's MMAs compute.
+
+    Each union entry of a 128-row tile costs an M=128 S MMA and PV MMA over one 64-key
+    block: two 64x64 block-equivalents, of which a one-half entry (attended by one of
+    the tile's two query blocks) uses one.  Entries of fully padded key blocks are
+    dropped by the kernel and not counted."""
+    from block_sparse_attention_bigbird_b200 import bsa
+    _, pair_ptr, pair_ent = bsa.bsa_layout_tiles(lay)
+    cols = pair_ent & 0xFFFFFF
+    dead = _dead_from(w)
+    issued_per_batch = int(len(cols) if dead is None else np.count_nonzero(cols < dead))
+    return nnz_eff / (2.0 * w.B * issued_per_batch)
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons in a background thread."""
 
@@ -489,6 +504,7 @@ def run_ours(args, w, world, rank, local):
                      "kernel": "bsa_fwd_kernel (+ bsa_merge_kernel when the layout has split rows)",
                      "peak_source": f"{peak_src} bf16 burst",
                      "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+                     "mma_useful_frac": _mma_useful_frac(w, lay, nnz_eff),
                      "ex2": _ex2_ceiling(nnz_eff, kernel_ms, dev, peaks)},
         "e2e": {"value": job_flop / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
