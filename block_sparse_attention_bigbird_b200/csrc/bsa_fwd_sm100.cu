@@ -156,6 +156,7 @@ struct FwdParams {
   int B, H, L, nb, items_per_batch, n_split, n_records;
   int split_items;  // the first split_items items of a batch element are split-tile chunks
   int split_lead;   // split chunks are handed out this many batch elements early
+  const int32_t* item_order;  // null, or the items of one batch element head by head
   float scale_log2;
   unsigned long long timeout_ns;
 };
@@ -261,7 +262,7 @@ __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, i
     ItemStage& st = sl.items[ii];
     if (t >= 0) {
       const int2 bi = item_of(t, p.B, p.split_items, p.items_per_batch - p.split_items, p.split_lead);
-      const int b = bi.x, i = bi.y;
+      const int b = bi.x, i = p.item_order != nullptr ? p.item_order[bi.y] : bi.y;
       const WorkItem w = p.items[i];
       int kept = w.count;
       if (p.keybits == nullptr) {
@@ -1141,7 +1142,8 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
   // How many batch elements early the split chunks go out: the last element's must
   // start while each slot still has at least one such chunk's length of work ahead.
   prm.split_lead = 0;
-  if (prm.split_items > 0 && B > 1) {
+  prm.item_order = nullptr;
+  if (prm.split_items > 0) {
     int64_t work = 0;  // chunks of one batch element
     int longest = 0;
     for (const WorkItem& it : lay->items) {
@@ -1151,6 +1153,10 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
     }
     const int64_t slots = static_cast<int64_t>(kSlots) * grid;
     while (prm.split_lead < B - 1 && (prm.split_lead + 1) * work < longest * slots) ++prm.split_lead;
+    // One head's items are enough work to hand out its split chunks just before its
+    // other tiles (the last head's chunks still start early enough): head by head.
+    if (prm.split_lead == 0 && work >= static_cast<int64_t>(longest) * slots * H)
+      prm.item_order = lay->d_head_order;
   }
   bsa_fwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
@@ -1182,6 +1188,7 @@ void free_device(bsa_layout* lay) {
     cudaFree(lay->d_pair_q);
     cudaFree(lay->d_pair_ent);
     cudaFree(lay->d_items);
+    cudaFree(lay->d_head_order);
     cudaFree(lay->d_splits);
     cudaFree(lay->d_kpair_q);
     cudaFree(lay->d_kpair_ent);
@@ -1194,6 +1201,7 @@ void free_device(bsa_layout* lay) {
   lay->d_pair_q = nullptr;
   lay->d_pair_ent = nullptr;
   lay->d_items = nullptr;
+  lay->d_head_order = nullptr;
   lay->d_splits = nullptr;
   lay->d_kpair_q = nullptr;
   lay->d_kpair_ent = nullptr;
@@ -1226,6 +1234,8 @@ int bsa_layout_upload(bsa_layout* lay, void* stream) {
       {reinterpret_cast<void**>(&lay->d_pair_q), lay->pair_q.data(), lay->pair_q.size() * sizeof(int32_t)},
       {reinterpret_cast<void**>(&lay->d_pair_ent), lay->pair_ent.data(), lay->pair_ent.size() * sizeof(uint32_t)},
       {reinterpret_cast<void**>(&lay->d_items), lay->items.data(), lay->items.size() * sizeof(WorkItem)},
+      {reinterpret_cast<void**>(&lay->d_head_order), lay->head_order.data(),
+       lay->head_order.size() * sizeof(int32_t)},
       {reinterpret_cast<void**>(&lay->d_splits), lay->splits.data(), lay->splits.size() * sizeof(SplitTile)},
       {reinterpret_cast<void**>(&lay->d_kpair_q), lay->ktiles.pair_q.data(),
        lay->ktiles.pair_q.size() * sizeof(int32_t)},

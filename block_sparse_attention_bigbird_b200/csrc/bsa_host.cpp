@@ -318,6 +318,12 @@ void build_tiles(bsa_layout* lay, const std::vector<uint8_t>& dense) {
       }
     }
   }
+  lay->head_order.clear();
+  for (int h = 0; h < H; ++h)
+    for (const bool split_pass : {true, false})
+      for (size_t x = 0; x < lay->items.size(); ++x)
+        if (lay->items[x].h == h && (lay->items[x].split >= 0) == split_pass)
+          lay->head_order.push_back(static_cast<int32_t>(x));
   // Backward.  dQ runs over the same query tiles.  dK and dV run over key tiles:
   // the transposed CSR (row (h, j) = the query blocks whose row holds key block j,
   // ascending) cut into tiles the same way, the key blocks every query block

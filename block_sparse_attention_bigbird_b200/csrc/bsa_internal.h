@@ -97,6 +97,10 @@ struct bsa_layout {
   std::vector<int32_t> pair_ptr;    // H*n_pairs + 1
   std::vector<uint32_t> pair_ent;   // union entries
   std::vector<bsa::WorkItem> items; // schedule for ONE batch element (head-major)
+  // the same items head by head, each head's split chunks first: item indices, for the
+  // forward's order when one head's work is long enough to hand out its split chunks
+  // just before its other tiles (its K/V then stay in L2)
+  std::vector<int32_t> head_order;
   std::vector<bsa::SplitTile> splits;  // the split tiles of one batch element
   int n_split = 0;                  // split tiles per batch element
   int n_records = 0;                // partial records per batch element
@@ -109,6 +113,7 @@ struct bsa_layout {
   int32_t* d_pair_q = nullptr;
   uint32_t* d_pair_ent = nullptr;
   bsa::WorkItem* d_items = nullptr;
+  int32_t* d_head_order = nullptr;
   bsa::SplitTile* d_splits = nullptr;
   int32_t* d_kpair_q = nullptr;
   uint32_t* d_kpair_ent = nullptr;
