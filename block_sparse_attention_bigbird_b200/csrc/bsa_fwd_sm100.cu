@@ -14,13 +14,14 @@
 // 64-row query blocks of the same (b, h) over the union of their key-block lists; a
 // chunk is two consecutive union entries (128 keys).
 //   warps 0-3 / 4-7  softmax of slot 0 / 1 (thread r of the slot owns tile row r =
-//               TMEM lane r).  Per chunk: load all of S(g) into registers and hand the S
-//               columns straight back, so S(g + 1) runs during these exponentials; chunk
-//               max on the ALU; p = 2^(s * scale * log2 e - m) on the ex2 unit; P (bf16)
-//               into the P columns once PV(g - 1) has read them.  The running max m is
-//               raised only when a chunk's max exceeds it by more than 2^8 (then l and O
-//               are rescaled), so p <= 2^8.  A finished tile's epilogue runs in the next
-//               tile's first chunk.
+//               TMEM lane r).  Per chunk: load all of S(g) into registers; p = 2^(s *
+//               scale * log2 e - m) on the ex2 unit with the running max m as it stands;
+//               hand the S columns back; P (bf16) into the P columns once PV(g - 1) has
+//               read them.  m is raised only when a chunk's max exceeds it by more than
+//               2^8 (then l and O are rescaled), so p <= 2^8; the chunk max is taken only
+//               on a row's first chunk or when a row's sum of p passes 2^8 (the chunk is
+//               then redone from S loaded again).  A finished tile's epilogue runs in the
+//               next tile's first chunk.
 //   warp 8 + s  K producer of slot s: stages the slot's work items; TMA loads of the Q tile
 //               and of K, the chunk's two 64-key blocks per 16 KB stage, 2 stages.
 //   warp 14 + s V producer of slot s: TMA loads of V into 2 stages of 16 KB.
@@ -31,7 +32,9 @@
 // per-chunk hand-off costs the softmax warps a few hundred cycles of latency, so a chunk
 // spans 128 keys to spread that cost over 128 exponentials per thread.
 // Entries carry per-block membership bits so each half of the tile sees exactly its own
-// row; a warp whose half does not attend a block gives it zero P without exponentials.
+// row (a softmax warp keeps an item's bits as two ballots); a warp whose half does not
+// attend a block gives it zero P without exponentials, and entries whose 64 keys are all
+// padded are dropped when the item is staged.
 // Long unions (global rows) are cut into chunks run as separate work items; each stores
 // a partial (O, m, l) record, and bsa_merge_kernel, launched after the forward, merges a
 // split tile's records into its output rows.
