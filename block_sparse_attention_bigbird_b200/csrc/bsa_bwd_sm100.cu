@@ -54,6 +54,7 @@
 namespace bsa {
 namespace {
 
+static_assert(kSplitThreshold <= 64 && kSplitChunk <= 64, "a backward item has at most 64 entries");
 constexpr int kComputeWarps = 8;
 constexpr int kComputeThreads = 32 * kComputeWarps;
 constexpr int kProducerWarp = 8;
@@ -397,8 +398,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
         lse2 = p.lse2[grow];
         drow = p.dsum[grow];
       }
+      // the item's union entries, lane x holding entries x and x + 32 (an item has at
+      // most 64), handed round by shuffles instead of a global load per entry
+      const uint32_t ent_lo = lane < t.w.count ? p.pair_ent[t.w.start + lane] : 0u;
+      const uint32_t ent_hi = lane + 32 < t.w.count ? p.pair_ent[t.w.start + lane + 32] : 0u;
       for (int n = 0; n < t.w.count; ++n, ++g) {
-        const uint32_t e = p.pair_ent[t.w.start + n];
+        const uint32_t e = __shfl_sync(0xffffffffu, n < 32 ? ent_lo : ent_hi, n & 31);
         const uint32_t ss = g & 1u, es = g % kEStages;
         if (!wait_warp(bar(kBarScoreFull + static_cast<int>(ss)), (g >> 1) & 1u, abort_flag, p.timeout_ns)) {
           ok = false;
