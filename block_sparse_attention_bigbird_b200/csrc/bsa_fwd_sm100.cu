@@ -912,6 +912,10 @@ struct MergeParams {
 };
 
 __global__ void __launch_bounds__(128) bsa_merge_kernel(const __grid_constant__ MergeParams p) {
+  // launched as the forward's programmatic dependent: its launch overlaps the
+  // forward's end, and this wait returns once the forward has finished and its
+  // records are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kGroup = 8;
   const int lane = threadIdx.x & 31;
   const int task = blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -1175,8 +1179,17 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
     mp.n_split = lay->n_split;
     mp.n_records = lay->n_records;
     const int64_t tasks = static_cast<int64_t>(B) * lay->n_split * kTileRows;
-    bsa_merge_kernel<<<static_cast<int>((tasks + 3) / 4), 128, 0, s>>>(mp);
-    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((tasks + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, bsa_merge_kernel, mp) != cudaSuccess) return BSA_ERR_CUDA;
   }
   return BSA_OK;
 }
