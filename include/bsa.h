@@ -222,7 +222,10 @@ int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
  *             aligned, any contents (see above).
  * Enqueues on `stream` a 256-byte memset of the schedule counters and up to
  * three kernels: the key-padding bits (with a key mask), the forward, and the
- * merge of split rows (when the layout has any).
+ * merge of split rows (when the layout has any; it is launched as a
+ * programmatic dependent of the forward, so its launch overlaps the forward's
+ * end).  Key blocks whose 64 keys are all dropped by the key mask cost no
+ * loads or MMAs.
  * Returns after enqueueing (no synchronisation, no allocation).  A device-side
  * timeout is reported later by bsa_sync_status.
  */
