@@ -67,9 +67,8 @@ constexpr uint32_t kOpBytes = 2 * kBlkBytes;  // a 128-row tile operand
 constexpr uint32_t kVecBytes = 64 * 4;
 constexpr uint32_t kTmemCols = 512;
 // TMEM: score stage s at 128 s (S or S^T at +0, dP or dP^T at +64); accumulator
-// stage a at 256 + kAccCols a (dQ; or dV at +0 and dK at +64)
+// stage a after the score stages, kAccCols apart (dQ; or dV at +0 and dK at +64)
 constexpr uint32_t kTmemScore = 0;
-constexpr uint32_t kTmemAcc = 256;
 
 // shared memory (offsets from the 1024-aligned base)
 constexpr uint32_t kSmemTile = 0;                                // [2 stages][operand A | operand B]
@@ -81,10 +80,10 @@ enum : int {
   kBarTileEmpty = 2,                     // [2] the tile's last score MMAs are done
   kBarEntFull = 4,                       // [4] the entry's blocks (and vectors) landed
   kBarEntEmpty = kBarEntFull + kEStages,      // [4] the entry's accumulating MMAs are done
-  kBarScoreFull = kBarEntEmpty + kEStages,    // [2] S and dP of the entry are in TMEM
-  kBarScoreFree = kBarScoreFull + 2,          // [2] the entry's accumulating MMAs read its dS
-  kBarDsFull = kBarScoreFree + 2,             // [2] 256 arrivals: dS (and P^T) written
-  kBarAccFull = kBarDsFull + 2,               // [2] the tile's last accumulating MMAs are done
+  kBarScoreFull = kBarEntEmpty + kEStages,    // [3] S and dP of the entry are in TMEM
+  kBarScoreFree = kBarScoreFull + 3,          // [3] the entry's accumulating MMAs read its dS
+  kBarDsFull = kBarScoreFree + 3,             // [3] 256 arrivals: dS (and P^T) written
+  kBarAccFull = kBarDsFull + 3,               // [2] the tile's last accumulating MMAs are done (dK/dV uses one)
   kBarAccEmpty = kBarAccFull + 2,             // [2] 256 arrivals: the epilogue read the accumulators
   kBarFinal = kBarAccEmpty + 2,               // [2] the issuers' last commits
   kNumBars = kBarFinal + 2
@@ -191,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
-      const bool many = (i >= kBarDsFull && i < kBarDsFull + 2) || (i >= kBarAccEmpty && i < kBarAccEmpty + 2);
+      const bool many = (i >= kBarDsFull && i < kBarDsFull + 3) || (i >= kBarAccEmpty && i < kBarAccEmpty + 2);
       ptx::mbar_init(bar(i), many ? static_cast<uint32_t>(kComputeThreads) : 1u);
     }
     misc[1] = 0;
@@ -208,6 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
   const int total = p.B * p.n_items;
   constexpr uint32_t kAccCols = kDkv ? 128u : 64u;
+  // three score stages; accumulators: two stages of 64 columns (dQ), one of 128 (dK/dV)
+  constexpr uint32_t kSStages = 3u;
+  constexpr uint32_t kAccStages = kDkv ? 1u : 2u;
+  constexpr uint32_t kAccBase = 384u;
+  static_assert(128u * kSStages <= kAccBase && kAccBase + kAccStages * kAccCols <= kTmemCols, "TMEM map");
   auto tile_op = [&](uint32_t ts, int op) { return base + kSmemTile + ts * 2 * kOpBytes + op * kOpBytes; };
   auto ent_op = [&](uint32_t es, int op) { return base + kSmemEnt + es * 2 * kBlkBytes + op * kBlkBytes; };
 
@@ -284,9 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
           break;
         }
         for (int n = 0; n < r.w.count; ++n, ++g) {
-          const uint32_t es = g % kEStages, ss = g & 1u;
+          const uint32_t es = g % kEStages, ss = g % kSStages;
           if (!wait_one(bar(kBarEntFull + static_cast<int>(es)), (g / kEStages) & 1u, abort_flag, p.timeout_ns) ||
-              !wait_one(bar(kBarScoreFree + static_cast<int>(ss)), ((g >> 1) & 1u) ^ 1u, abort_flag,
+              !wait_one(bar(kBarScoreFree + static_cast<int>(ss)), ((g / kSStages) & 1u) ^ 1u, abort_flag,
                         p.timeout_ns)) {
             ok = false;
             break;
@@ -312,15 +316,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
       bool ok = true, issued = false;
       for (int it = blockIdx.x; it < total && ok; it += gridDim.x, ++k) {
         const ItemRef r = item_at(p, it);
-        const uint32_t as = k & 1u;
-        if (!wait_one(bar(kBarAccEmpty + static_cast<int>(as)), ((k >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+        const uint32_t as = k % kAccStages;
+        if (!wait_one(bar(kBarAccEmpty + static_cast<int>(as)), ((k / kAccStages) & 1u) ^ 1u, abort_flag,
+                      p.timeout_ns)) {
           ok = false;
           break;
         }
-        const uint32_t acc = tmem + kTmemAcc + kAccCols * as;
+        const uint32_t acc = tmem + kAccBase + kAccCols * as;
         for (int n = 0; n < r.w.count; ++n, ++g) {
-          const uint32_t es = g % kEStages, ss = g & 1u;
-          if (!wait_one(bar(kBarDsFull + static_cast<int>(ss)), (g >> 1) & 1u, abort_flag, p.timeout_ns)) {
+          const uint32_t es = g % kEStages, ss = g % kSStages;
+          if (!wait_one(bar(kBarDsFull + static_cast<int>(ss)), (g / kSStages) & 1u, abort_flag, p.timeout_ns)) {
             ok = false;
             break;
           }
@@ -358,13 +363,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
     uint32_t pend_k = 0;
     ItemRef pend{};
     auto epilogue = [&](uint32_t kt, const ItemRef& t) -> bool {
-      const uint32_t as = kt & 1u;
-      if (!wait_warp(bar(kBarAccFull + static_cast<int>(as)), (kt >> 1) & 1u, abort_flag, p.timeout_ns)) return false;
+      const uint32_t as = kt % kAccStages;
+      if (!wait_warp(bar(kBarAccFull + static_cast<int>(as)), (kt / kAccStages) & 1u, abort_flag, p.timeout_ns))
+        return false;
       ptx::tc_fence_after();
       const bool active = half == 0 || t.tb >= 0;
       const size_t grow =
           static_cast<size_t>(t.row0) + static_cast<size_t>(half ? t.tb : t.ta) * 64 + static_cast<size_t>(r & 63);
-      const uint32_t acc = tmem + lane_addr + kTmemAcc + kAccCols * as + 32u * ch;
+      const uint32_t acc = tmem + lane_addr + kAccBase + kAccCols * as + 32u * ch;
       float* rec = nullptr;
       if (t.w.rec >= 0)
         rec = p.records + (static_cast<size_t>(t.b) * p.n_records + t.w.rec) * (kDkv ? kBwdDkvRecFloats : kBwdDqRecFloats) +
@@ -404,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
       const uint32_t ent_hi = lane + 32 < t.w.count ? p.pair_ent[t.w.start + lane + 32] : 0u;
       for (int n = 0; n < t.w.count; ++n, ++g) {
         const uint32_t e = __shfl_sync(0xffffffffu, n < 32 ? ent_lo : ent_hi, n & 31);
-        const uint32_t ss = g & 1u, es = g % kEStages;
-        if (!wait_warp(bar(kBarScoreFull + static_cast<int>(ss)), (g >> 1) & 1u, abort_flag, p.timeout_ns)) {
+        const uint32_t ss = g % kSStages, es = g % kEStages;
+        if (!wait_warp(bar(kBarScoreFull + static_cast<int>(ss)), (g / kSStages) & 1u, abort_flag, p.timeout_ns)) {
           ok = false;
           break;
         }
