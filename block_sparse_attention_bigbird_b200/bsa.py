@@ -66,6 +66,12 @@ _SIGNATURES = {
                                     ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                     ctypes.c_size_t, ctypes.c_void_p]),
+    "bsa_qkv_projection": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p, ctypes.c_void_p]),
+    "bsa_out_projection": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                          ctypes.c_void_p]),
     "bsa_sync_status": (ctypes.c_int, [ctypes.c_void_p]),
     "bsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "bsa_debug_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p]),
@@ -335,6 +341,68 @@ def bsa_backward(q, k, v, out, dout, lse, layout: Layout, key_mask=None, scale: 
                             ctypes.c_void_p(_stream_ptr(stream)))
     _check(code, "bsa_backward")
     return dq, dk, dv
+
+
+def _check_bf16(name, t, dim):
+    import torch
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != dim:
+        raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor of {dim} dimensions")
+
+
+def bsa_qkv_projection(x, weight, bias=None, num_heads: Optional[int] = None, q=None, k=None, v=None,
+                       stream=None):
+    """q, k, v = the heads of x W^T + bias, each bf16 [B, H, L, 64].
+
+    x: bf16 [B, L, C] with C = 64 H; weight: bf16 [3C, C] (rows: the q features,
+    then k, then v; within each, head h's 64 features at 64 h); bias: bf16 [3C]
+    or None.  The library's tcgen05 GEMM writes the three outputs in the head
+    layout directly.
+    """
+    import torch
+    _check_bf16("x", x, 3)
+    _check_bf16("weight", weight, 2)
+    B, L, C = x.shape
+    H = num_heads if num_heads is not None else C // 64
+    if C != 64 * H or tuple(weight.shape) != (3 * C, C):
+        raise ValueError("x must be [B, L, 64 H] and weight [3 C, C]")
+    if bias is not None:
+        _check_bf16("bias", bias, 1)
+        if bias.numel() != 3 * C:
+            raise ValueError("bias must have 3 C elements")
+    outs = []
+    for t in (q, k, v):
+        outs.append(torch.empty((B, H, L, 64), dtype=torch.bfloat16, device=x.device) if t is None else t)
+    code = lib.bsa_qkv_projection(x.data_ptr(), weight.data_ptr(), bias.data_ptr() if bias is not None else None,
+                                  B, L, H, outs[0].data_ptr(), outs[1].data_ptr(), outs[2].data_ptr(),
+                                  ctypes.c_void_p(_stream_ptr(stream)))
+    _check(code, "bsa_qkv_projection")
+    return tuple(outs)
+
+
+def bsa_out_projection(o, weight, bias=None, y=None, stream=None):
+    """y = merge_heads(o) W^T + bias, bf16 [B, L, N].
+
+    o: bf16 [B, H, L, 64] (the attention output); weight: bf16 [N, 64 H] with N
+    a multiple of 64; bias: bf16 [N] or None.  The heads are merged by the
+    GEMM's own tile loads.
+    """
+    import torch
+    _check_bf16("o", o, 4)
+    _check_bf16("weight", weight, 2)
+    B, H, L, d = o.shape
+    N = weight.shape[0]
+    if d != 64 or weight.shape[1] != 64 * H:
+        raise ValueError("o must be [B, H, L, 64] and weight [N, 64 H]")
+    if bias is not None:
+        _check_bf16("bias", bias, 1)
+        if bias.numel() != N:
+            raise ValueError("bias must have N elements")
+    if y is None:
+        y = torch.empty((B, L, N), dtype=torch.bfloat16, device=o.device)
+    code = lib.bsa_out_projection(o.data_ptr(), weight.data_ptr(), bias.data_ptr() if bias is not None else None,
+                                  B, H, L, N, y.data_ptr(), ctypes.c_void_p(_stream_ptr(stream)))
+    _check(code, "bsa_out_projection")
+    return y
 
 
 def bsa_sync_status(stream=None) -> int:

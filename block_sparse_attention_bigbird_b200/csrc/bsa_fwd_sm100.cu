@@ -1308,7 +1308,8 @@ int bsa_sync_status(void* stream) {
     if (cudaMemcpyToSymbol(g_bsa_status, &zero, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
   }
   const int st_bwd = bwd_take_status();  // the backward kernels' status word
-  return st != 0 ? st : st_bwd;
+  const int st_proj = proj_take_status();  // the projection kernels' status word
+  return st != 0 ? st : (st_bwd != 0 ? st_bwd : st_proj);
 }
 
 int bsa_debug_wait_timeout(uint64_t timeout_ns, void* stream) {

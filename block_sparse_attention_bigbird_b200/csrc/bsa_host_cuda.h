@@ -22,4 +22,7 @@ cudaError_t launch_keybits(const uint8_t* key_mask, unsigned long long* bits, in
 // 0, a negative bsa_status a kernel recorded, or BSA_ERR_CUDA if the read failed.
 int bwd_take_status();
 
+// The same for the projection kernels (bsa_proj_sm100.cu).
+int proj_take_status();
+
 }  // namespace bsa

@@ -305,6 +305,43 @@ int bsa_backward(const void* q, const void* k, const void* v, const void* out, c
                  size_t workspace_bytes, void* stream);
 
 /*
+ * bsa_qkv_projection -- the layer's QKV projection, written in the attention's
+ * head layout ("BigBird 稀疏注意力机制解析", 代码实现: self.qkv =
+ * nn.Linear(dim, dim * 3), then split into heads).  With C = 64 H:
+ *   x     device, bf16 [B, L, C] row-major;
+ *   w     device, bf16 [3 C, C] row-major (a linear layer's [out, in] weight):
+ *         rows 0..C-1 make q, C..2C-1 k, 2C..3C-1 v; within each, rows
+ *         64 h..64 h+63 are head h's 64 features;
+ *   bias  device, bf16 [3 C], or NULL for none;
+ *   q, k, v  device, bf16 [B, H, L, 64], written:
+ *         q[b, h, l, j] = bf16_rne(sum_c x[b, l, c] w[64 h + j, c] + bias[64 h + j])
+ *         (k and v with rows C + 64 h + j and 2 C + 64 h + j), fp32 accumulation.
+ * All pointers 16-byte aligned; the caller owns every buffer.  B, L, H >= 1
+ * (else BSA_ERR_INVALID_ARG).  Enqueues one kernel on `stream` (tcgen05 GEMM,
+ * 128 x 256 tiles, the head split done by its stores); no allocation, no
+ * synchronisation; a device-side timeout is reported by bsa_sync_status.
+ * BSA_ERR_UNSUPPORTED on a device that is not sm_100.
+ */
+int bsa_qkv_projection(const void* x, const void* w, const void* bias, int B, int L, int H, void* q,
+                       void* k, void* v, void* stream);
+
+/*
+ * bsa_out_projection -- the layer's output projection over the merged heads
+ * ("BERT 稀疏注意力机制入门指南", PyTorch 实现: self.proj = nn.Linear(dim,
+ * dim) after the heads are concatenated):
+ *   o     device, bf16 [B, H, L, 64] (the attention output);
+ *   w     device, bf16 [N, 64 H] row-major (a linear layer's [out, in] weight);
+ *   bias  device, bf16 [N], or NULL;
+ *   y     device, bf16 [B, L, N], written:
+ *         y[b, l, n] = bf16_rne(sum_{h, j} o[b, h, l, j] w[n, 64 h + j] + bias[n]).
+ * N a positive multiple of 64 (else BSA_ERR_INVALID_ARG); pointers 16-byte
+ * aligned; B, L, H >= 1.  Enqueues one kernel (the heads are merged by the
+ * GEMM's own tile loads); no allocation, no synchronisation.
+ */
+int bsa_out_projection(const void* o, const void* w, const void* bias, int B, int H, int L, int N, void* y,
+                       void* stream);
+
+/*
  * bsa_sync_status -- synchronises `stream`, then returns and clears the
  * device-side status word of the current device: BSA_OK, or
  * BSA_ERR_DEVICE_TIMEOUT if a kernel's bounded wait gave up (its outputs are
