@@ -291,9 +291,13 @@ def run_reference(args, w, world, rank):
     nb = w.nb
     n_blocks = max(1, min(nb, int(os.environ.get("BSA_REF_BLOCKS", "8"))))
     backward = args.pass_ == "backward"
+    layer = args.pass_ == "layer"
     if backward:
         do = workloads.make_grad(w, seed=100)
         sample_fn = lambda h: _oracle_bwd_sample(w, lay, q, k, v, do, km, h, n_blocks)  # noqa: E731
+    elif layer:
+        lp = _layer_params(w, seed=0)
+        sample_fn = lambda h: _oracle_layer_sample(w, lay, *lp, km, h, n_blocks)  # noqa: E731
     else:
         sample_fn = lambda h: _oracle_sample(w, lay, q, k, v, km, h, n_blocks)  # noqa: E731
     for s in range(args.warmup):
@@ -305,9 +309,14 @@ def run_reference(args, w, world, rank):
         tot_f += fl
     val = tot_f / tot_t / 1e12
     cores = _oracle_cores()
-    sample = (f"per step: {'gradients from ' if backward else ''}query blocks 0..{n_blocks - 1} of batch 0, "
-              f"head step%H ({n_blocks * 64} of {w.L} query rows), fp64 masked-dense")
-    line = {"impl": "reference", "metric": METRIC_BWD if backward else METRIC, "value": val, "unit": UNIT,
+    if layer:
+        sample = (f"per step: head step%H of batch 0: q for query blocks 0..{n_blocks - 1}, k and v for every "
+                  f"row, attention on those blocks, the head's share of the output projection (fp64)")
+    else:
+        sample = (f"per step: {'gradients from ' if backward else ''}query blocks 0..{n_blocks - 1} of batch 0, "
+                  f"head step%H ({n_blocks * 64} of {w.L} query rows), fp64 masked-dense")
+    metric = METRIC_BWD if backward else (METRIC_LAYER if layer else METRIC)
+    line = {"impl": "reference", "metric": metric, "value": val, "unit": UNIT,
             "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -670,6 +679,199 @@ def run_backward(args, w, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+METRIC_LAYER = "BigBird layer forward TFLOP/s (dense projections + attention on non-zero blocks)"
+
+
+def _layer_params(w, seed):
+    """x [B, L, C] and the two projections' bf16 weights and biases (C = 64 H), seeded."""
+    g = torch.Generator().manual_seed(seed)
+    C = w.H * w.d
+    x = torch.randn(w.B, w.L, C, generator=g).to(torch.bfloat16)
+    wq = (torch.randn(3 * C, C, generator=g) * C ** -0.5).to(torch.bfloat16)
+    bq = (torch.randn(3 * C, generator=g) * 0.1).to(torch.bfloat16)
+    wo = (torch.randn(C, C, generator=g) * C ** -0.5).to(torch.bfloat16)
+    bo = (torch.randn(C, generator=g) * 0.1).to(torch.bfloat16)
+    return x, wq, bq, wo, bo
+
+
+def _oracle_layer_sample(w, lay, x, wq, bq, wo, bo, km, h, n_blocks):
+    """The layer's work for head h of batch 0 on query blocks [0, n_blocks): the oracle's
+    q, k, v of that head (k, v for every key row), its attention on those query blocks
+    and the head's share of the output projection; returns (seconds, flop)."""
+    from oracle import attention as OA
+    from oracle import projection as OP
+    C = w.H * w.d
+    rows = n_blocks * 64
+    view = _head_view(lay, h)
+    rp, ci = view["row_ptr"], view["col_idx"]
+    nnz = int(rp[n_blocks])
+    dead = _dead_from(w)
+    if dead is not None:
+        nnz -= int(np.count_nonzero(ci[:rp[n_blocks]] >= dead))
+    kmask = None if km is None else km[0:1]
+    t0 = time.perf_counter()
+    sl = [slice(i * C + h * 64, i * C + h * 64 + 64) for i in range(3)]
+    xq = x[0].double().numpy()
+    qh = np.zeros((w.L, 64))
+    qh[:rows] = OP.linear(xq[:rows], wq[sl[0]], bq[sl[0]])
+    kh = OP.linear(xq, wq[sl[1]], bq[sl[1]])
+    vh = OP.linear(xq, wq[sl[2]], bq[sl[2]])
+    o, _ = OA.attention(qh[None, None], kh[None, None], vh[None, None], view, key_mask=kmask,
+                        query_blocks=range(n_blocks))
+    OP.linear(o[0, 0, :rows], wo[:, h * 64:(h + 1) * 64])
+    dt = time.perf_counter() - t0
+    flop = 2 * 64 * C * (rows + 2 * w.L) + nnz * FLOP_PER_BLOCK + 2 * rows * 64 * C
+    return dt, flop
+
+
+def run_layer(args, w, world, rank, local):
+    """The fused BigBird layer forward: bsa_qkv_projection, bsa_forward, bsa_out_projection."""
+    from block_sparse_attention_bigbird_b200 import bsa
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    if w.d != 64:
+        raise SystemExit("the layer pass needs d = 64")
+    C = w.H * w.d
+    x, wq, bq, wo, bo = _layer_params(w, seed=rank)
+    km = workloads.make_key_mask(w)
+    lay = bsa.bsa_layout_build(w.H, w.L, w.block, w.window, w.n_global, w.n_random, w.seed)
+    bsa.bsa_layout_upload(lay)
+    row_ptr, col_idx = bsa.bsa_layout_csr(lay)
+    nnz_eff = _nnz_eff(w, row_ptr, col_idx)
+    flop_qkv = 2 * w.B * w.L * C * 3 * C
+    flop_att = nnz_eff * FLOP_PER_BLOCK
+    flop_out = 2 * w.B * w.L * C * C
+    flop_step = flop_qkv + flop_att + flop_out
+    xd, wqd, bqd, wod, bod = (t.to(dev) for t in (x, wq, bq, wo, bo))
+    kmd = km.to(dev) if km is not None else None
+    q, k, v = (torch.empty((w.B, w.H, w.L, 64), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    y = torch.empty((w.B, w.L, C), dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(bsa.bsa_workspace_bytes(lay, w.B), dtype=torch.uint8, device=dev)
+    launches_per_step = 2 + 1 + (1 if km is not None else 0) + (1 if _has_split_rows(lay) else 0)
+
+    def part_qkv(xs=xd):
+        bsa.bsa_qkv_projection(xs, wqd, bqd, q=q, k=k, v=v, stream=stream)
+
+    def part_att():
+        bsa.bsa_forward(q, k, v, lay, key_mask=kmd, out=o, lse=lse, workspace=ws, stream=stream)
+
+    def part_out():
+        bsa.bsa_out_projection(o, wod, bod, y=y, stream=stream)
+
+    def step(xs=xd):
+        part_qkv(xs)
+        part_att()
+        part_out()
+
+    def timed(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    sampler = ClockSampler(local).start() if rank == 0 else None
+    for _ in range(max(3, args.warmup)):
+        step()
+    _barrier(world)
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error during warm-up")
+    t_settle = time.time()
+    per = max(timed(step, 1), 1e-3)
+    for _ in range(int(min(2000, 1500.0 / per))):
+        step()
+    _barrier(world)
+    t_timed0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    _barrier(world)
+    t_timed1 = time.time()
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error in the timed region")
+    total_ms = sharding.max_over_ranks(start.elapsed_time(end), world)
+    # each part alone, the same number of launches, right after the timed region
+    n_part = max(3, args.steps)
+    ms_parts = {"qkv_projection": timed(part_qkv, n_part), "attention": timed(part_att, n_part),
+                "out_projection": timed(part_out, n_part)}
+    clocks = sampler.summary(t_settle, t_timed1, t_timed0) if sampler else None
+    if sampler:
+        sampler.stop()
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error in the per-part timing")
+
+    # end to end through the public API: x from pinned host memory, the layer, y back
+    e2e_steps = max(3, min(args.steps, 10))
+    xh = x.pin_memory()
+    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    xbuf = torch.empty_like(xd)
+    _barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        xbuf.copy_(xh, non_blocking=True)
+        step(xbuf)
+        yh.copy_(y, non_blocking=True)
+    b.record(stream)
+    _barrier(world)
+    e2e_ms = sharding.max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
+    if bsa.bsa_sync_status(stream) != 0:
+        raise RuntimeError("device status error in the end-to-end run")
+
+    ms_per_step = total_ms / args.steps
+    value = world * flop_step / (ms_per_step * 1e-3) / 1e12
+    peaks, peak_src = _peaks()
+    peak = float(peaks["bf16_tflops"])
+    kern = {}
+    for name, fl in (("qkv_projection", flop_qkv), ("attention", flop_att), ("out_projection", flop_out)):
+        t = ms_parts[name]
+        kern[name] = {"ms": t, "tflops": fl / (t * 1e-3) / 1e12, "frac": fl / (t * 1e-3) / 1e12 / peak,
+                      "share": t / sum(ms_parts.values())}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        lay_o = _oracle_heads(w)
+        budget = float(os.environ.get("BSA_CPU_BUDGET_S", "12"))
+        tot_t = tot_f = 0.0
+        n_blocks, h = min(w.nb, 8), 0
+        while tot_t < budget and h < w.H:
+            dt, fl = _oracle_layer_sample(w, lay_o, x, wq, bq, wo, bo, km, h, n_blocks)
+            tot_t, tot_f, h = tot_t + dt, tot_f + fl, h + 1
+        cpu = {"value": tot_f / tot_t / 1e12, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
+               "sample": f"heads 0..{h - 1} of batch 0: q for query blocks 0..{n_blocks - 1}, k and v for "
+                         f"every row, attention on those blocks, the head's share of the output projection "
+                         f"({tot_t:.1f} s of fp64)"}
+    if rank != 0:
+        return
+    att = kern["attention"]
+    line = {
+        "metric": METRIC_LAYER, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded randn hidden states and weights, see bench._layer_params)",
+        "config": dict(_config(w, nnz_eff, world), **{"pass": "layer", "dim": C}),
+        "pct_of_peak": 100.0 * value / world / peak,
+        "kernels": kern,
+        "roofline": {"bound": "tensor", "achieved": att["tflops"], "peak": peak, "unit": UNIT,
+                     "frac": att["frac"], "traffic": None,
+                     "kernel": "bsa_fwd_kernel (the layer's largest share; the projections are in 'kernels')",
+                     "peak_source": f"{peak_src} bf16 burst"},
+        "e2e": {"value": world * flop_step / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": y.numel() * 2, "ms_per_step": e2e_ms,
+                "pipelining": "none: x in, the layer, y out on one stream"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def _cpu_baseline(w):
     lay = _oracle_heads(w)
     q, k, v = workloads.make_qkv(w, 0)
@@ -696,8 +898,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward"], default="forward",
-                    help="forward (the default benchmark) or the backward pass")
+    ap.add_argument("--pass", dest="pass_", choices=["forward", "backward", "layer"], default="forward",
+                    help="forward (the default benchmark), the backward pass, or the fused layer forward "
+                         "(QKV projection, attention, output projection)")
     ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
                     help="forward over N ranks: each rank its own batch (weak scaling, the default) "
                          "or the heads of one batch split across ranks (strong scaling)")
@@ -713,7 +916,8 @@ def main():
         return
     world, rank, local = _dist_setup(args)
     try:
-        (run_backward if args.pass_ == "backward" else run_ours)(args, w, world, rank, local)
+        runner = {"backward": run_backward, "layer": run_layer}.get(args.pass_, run_ours)
+        runner(args, w, world, rank, local)
     finally:
         if world > 1:
             import torch.distributed as dist
