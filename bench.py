@@ -339,7 +339,16 @@ def run_ours(args, w, world, rank, local):
     layout_build_ms = (time.perf_counter() - t_lay) * 1e3
     row_ptr, col_idx = bsa.bsa_layout_csr(lay)
     heads = args.shard == "heads"
-    if heads:
+    queries = args.shard == "queries"
+    if queries:
+        # strong scaling over query-block ranges: every rank reads the whole q, k, v
+        # of the sequence and computes its own range of query blocks (all heads)
+        q0, q1 = sharding.query_block_shard(row_ptr, w.nb, w.H, rank, world)
+        total_flop = _nnz_eff(w, row_ptr, col_idx) * FLOP_PER_BLOCK
+        row_ptr, col_idx = sharding.query_rows(row_ptr, col_idx, w.nb, w.H, q0, q1)
+        lay = bsa.bsa_layout_from_csr(w.H, w.L, row_ptr, col_idx)
+        q, k, v = workloads.make_qkv(w, data_seed=0)
+    elif heads:
         # strong scaling over heads: every rank takes its heads of the same sequence
         # (the genomic shape has one batch element) and a layout of those heads' rows
         if world > w.H:
@@ -361,7 +370,8 @@ def run_ours(args, w, world, rank, local):
     nnz_eff = _nnz_eff(w, row_ptr, col_idx)
     flop_step = nnz_eff * FLOP_PER_BLOCK
     # work of the whole job per step: every rank's own batch (weak), or one sequence's heads (strong)
-    job_flop = total_flop if heads else world * flop_step
+    strong = heads or queries
+    job_flop = total_flop if strong else world * flop_step
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     kmd = km.to(dev) if km is not None else None
     out = torch.empty_like(qd)
@@ -494,7 +504,7 @@ def run_ours(args, w, world, rank, local):
     peaks, peak_src = _peaks()
     achieved = flop_step / (kernel_ms * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = _traffic_for(w.name) if not heads or world == 1 else None
+    traffic = _traffic_for(w.name) if not strong or world == 1 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = _cpu_baseline(w)
@@ -503,10 +513,10 @@ def run_ours(args, w, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "strong" if heads else "weak", "vs_baseline": None, "dtype": "bf16",
+        "scaling": "strong" if strong else "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded randn, see workloads.py)",
         "config": dict(_config(w, nnz_eff, world),
-                       **({"parallelism": f"heads{world}", "global_batch": w.B} if heads else {})),
+                       **({"parallelism": f"{args.shard}{world}", "global_batch": w.B} if strong else {})),
         "pct_of_peak": 100.0 * value / world / peak,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT,
                      "frac": achieved / peak, "traffic": traffic,
@@ -901,9 +911,10 @@ def main():
     ap.add_argument("--pass", dest="pass_", choices=["forward", "backward", "layer"], default="forward",
                     help="forward (the default benchmark), the backward pass, or the fused layer forward "
                          "(QKV projection, attention, output projection)")
-    ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
+    ap.add_argument("--shard", choices=["batch", "heads", "queries"], default="batch",
                     help="forward over N ranks: each rank its own batch (weak scaling, the default) "
-                         "or the heads of one batch split across ranks (strong scaling)")
+                         "or the heads, or the query-block ranges, of one batch split across ranks "
+                         "(strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -217,3 +217,139 @@ def test_head_sharded_layouts_on_the_gpu_reproduce_the_full_run(world):
     _check(got[0].float().cpu().numpy(), got[1].cpu().numpy(), o_ref, lse_ref)
     dq, dk, dv, mags = OB.attention_backward(qc, kc, vc, doc, ref, key_mask=kmc, with_magnitude=True)
     _check_grads([t.float().cpu().numpy() for t in got[2:]], (dq, dk, dv), mags)
+
+
+# ---------------------------------------------------------------- query-block sharding
+def test_query_block_shard_covers_and_balances():
+    for (H, nb, window, n_global, n_random, seed) in ((3, 40, 1, 2, 3, 5), (2, 64, 2, 4, 2, 1), (1, 9, 0, 1, 0, 2)):
+        lay = OL.build_layout(H, nb * 64, 64, window, n_global, n_random, seed)
+        rp = lay["row_ptr"]
+        per_block = (rp[1:] - rp[:-1]).reshape(H, nb).sum(axis=0)
+        total = int(per_block.sum())
+        for world in range(1, 7):
+            spans = [sharding.query_block_shard(rp, nb, H, r, world) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == nb
+            assert all(a[1] == b[0] and a[0] <= a[1] for a, b in zip(spans, spans[1:]))
+            for a, b in spans:  # no rank exceeds an even share by more than one query block's work
+                assert int(per_block[a:b].sum()) <= -(-total // world) + int(per_block.max())
+
+
+def test_query_rows_keep_exactly_the_range():
+    H, nb = 3, 20
+    lay = OL.build_layout(H, nb * 64, 64, 1, 2, 3, 4)
+    rp, ci = lay["row_ptr"], lay["col_idx"]
+    r2, c2 = sharding.query_rows(rp, ci, nb, H, 4, 11)
+    assert r2.shape == rp.shape and r2[0] == 0
+    for h in range(H):
+        for i in range(nb):
+            x = h * nb + i
+            got = list(c2[r2[x]:r2[x + 1]])
+            assert got == (list(ci[rp[x]:rp[x + 1]]) if 4 <= i < 11 else [])
+
+
+def _worker_queries(rank, world, port, queue):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # one sequence, its query blocks split across the ranks; K and V whole on every rank
+        w = workloads.custom(1, 3, 64 * 12, 1, 2, 2, seed=11, key_pad_tail=30)
+        q, k, v = workloads.make_qkv(w)
+        do = workloads.make_grad(w, seed=5)
+        km = workloads.make_key_mask(w)
+        full = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+        q0, q1 = sharding.query_block_shard(full["row_ptr"], w.nb, w.H, rank, world)
+        rp, ci = sharding.query_rows(full["row_ptr"], full["col_idx"], w.nb, w.H, q0, q1)
+        mine = {"H": w.H, "L": w.L, "block": 64, "nb": w.nb, "row_ptr": rp.astype(np.int64), "col_idx": ci}
+        o, lse = OA.attention(q, k, v, mine, key_mask=km)
+        dq, dk, dv = OB.attention_backward(q, k, v, do, mine, key_mask=km)
+        dkv = torch.from_numpy(np.stack([dk, dv]))
+        sharding.sum_over_ranks(dkv, world)  # the backward's one exchange
+        rows = slice(64 * q0, 64 * q1)
+        shards = [None] * world
+        dist.all_gather_object(shards, (q0, q1, o[:, :, rows], lse[:, :, rows], dq[:, :, rows],
+                                        bool(np.all(o[:, :, :64 * q0] == 0) and np.all(o[:, :, 64 * q1:] == 0))))
+        if rank == 0:
+            queue.put((shards, dkv.numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_query_block_shards_on_two_gloo_ranks_reproduce_single_process():
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_queries, args=(r, 2, port, queue)) for r in range(2)]
+    for pr in procs:
+        pr.start()
+    shards, dkv = queue.get(timeout=120)
+    for pr in procs:
+        pr.join(timeout=120)
+        assert pr.exitcode == 0
+    w = workloads.custom(1, 3, 64 * 12, 1, 2, 2, seed=11, key_pad_tail=30)
+    q, k, v = workloads.make_qkv(w)
+    do = workloads.make_grad(w, seed=5)
+    km = workloads.make_key_mask(w)
+    lay = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    o_ref, lse_ref = OA.attention(q, k, v, lay, key_mask=km)
+    dq_ref, dk_ref, dv_ref = OB.attention_backward(q, k, v, do, lay, key_mask=km)
+    shards = sorted(shards, key=lambda s: s[0])
+    assert shards[0][0] == 0 and shards[-1][1] == w.nb and shards[0][1] == shards[1][0]
+    assert all(s[5] for s in shards)  # rows a rank does not own come out zero there
+    # a row's output and dQ depend on its own layout row alone: bit for bit
+    assert np.array_equal(np.concatenate([s[2] for s in shards], axis=2), o_ref)
+    assert np.array_equal(np.concatenate([s[3] for s in shards], axis=2), lse_ref)
+    assert np.array_equal(np.concatenate([s[4] for s in shards], axis=2), dq_ref)
+    # dK and dV are sums over query rows, added across ranks in another order
+    for got, ref in ((dkv[0], dk_ref), (dkv[1], dv_ref)):
+        assert np.abs(got - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+@pytest.mark.gpu
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+@pytest.mark.parametrize("world", [2, 3])
+def test_query_sharded_layouts_on_the_gpu_match_the_oracle(world):
+    """The work each rank of a query-block-sharded job does, run shard after shard
+    on one GPU: every rank's layout keeps its query blocks' rows
+    (sharding.query_rows -> bsa_layout_from_csr over the full length), the forward
+    and backward read the whole q, k, v.  Each rank's own rows of O, lse and dQ,
+    and dK, dV summed over the ranks in fp32, match the fp64 oracle within the
+    parity tolerances; rows a rank does not own come out as empty rows (O = 0,
+    lse = -inf)."""
+    from block_sparse_attention_bigbird_b200 import bsa
+    from test_backward import _check_grads
+    from test_gpu_parity import _check
+    w = workloads.custom(2, 3, 64 * 64, 1, 2, 3, seed=9, key_pad_tail=30)
+    qc, kc, vc = workloads.make_qkv(w)
+    doc = workloads.make_grad(w, seed=100)
+    kmc = workloads.make_key_mask(w)
+    dev = torch.device("cuda")
+    q, k, v, do, km = (t.to(dev) for t in (qc, kc, vc, doc, kmc))
+    full = bsa.bsa_layout_build(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    rp, ci = bsa.bsa_layout_csr(full)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.L), dtype=torch.float32, device=dev)
+    dq = torch.empty_like(q)
+    dk = torch.zeros(q.shape, dtype=torch.float32, device=dev)
+    dv = torch.zeros_like(dk)
+    for rank in range(world):
+        q0, q1 = sharding.query_block_shard(rp, w.nb, w.H, rank, world)
+        srp, sci = sharding.query_rows(rp, ci, w.nb, w.H, q0, q1)
+        mine = bsa.bsa_layout_from_csr(w.H, w.L, srp, sci)
+        bsa.bsa_layout_upload(mine)
+        o_r, lse_r = bsa.bsa_forward(q, k, v, mine, key_mask=km)
+        dq_r, dk_r, dv_r = bsa.bsa_backward(q, k, v, o_r, do, lse_r, mine, key_mask=km)
+        rows = slice(64 * q0, 64 * q1)
+        o[:, :, rows], lse[:, :, rows], dq[:, :, rows] = o_r[:, :, rows], lse_r[:, :, rows], dq_r[:, :, rows]
+        dk += dk_r.float()
+        dv += dv_r.float()
+        other = torch.ones(w.L, dtype=torch.bool, device=dev)
+        other[rows] = False
+        assert torch.all(o_r[:, :, other] == 0) and torch.all(torch.isneginf(lse_r[:, :, other]))
+    assert bsa.bsa_sync_status() == 0
+    ref = OL.build_layout(w.H, w.L, 64, w.window, w.n_global, w.n_random, w.seed)
+    o_ref, lse_ref = OA.attention(qc, kc, vc, ref, key_mask=kmc)
+    _check(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, lse_ref)
+    dq_o, dk_o, dv_o, mags = OB.attention_backward(qc, kc, vc, doc, ref, key_mask=kmc, with_magnitude=True)
+    _check_grads([dq.float().cpu().numpy(), dk.cpu().numpy(), dv.cpu().numpy()], (dq_o, dk_o, dv_o), mags)
