@@ -14,14 +14,13 @@
 // 64-row query blocks of the same (b, h) over the union of their key-block lists; a
 // chunk is two consecutive union entries (128 keys).
 //   warps 0-3 / 4-7  softmax of slot 0 / 1 (thread r of the slot owns tile row r =
-//               TMEM lane r).  Per chunk: load all of S(g) into registers; p = 2^(s *
-//               scale * log2 e - m) on the ex2 unit with the running max m as it stands;
-//               hand the S columns back; P (bf16) into the P columns once PV(g - 1) has
-//               read them.  m is raised only when a chunk's max exceeds it by more than
-//               2^8 (then l and O are rescaled), so p <= 2^8; the chunk max is taken only
-//               on a row's first chunk or when a row's sum of p passes 2^8 (the chunk is
-//               then redone from S loaded again).  A finished tile's epilogue runs in the
-//               next tile's first chunk.
+//               TMEM lane r).  Per chunk: load all of S(g) into registers and hand the
+//               S columns back at once (S(g + 1) is computed during this chunk's
+//               exponentials); the chunk max; p = 2^(s * scale * log2 e - m) on the ex2
+//               unit; P (bf16) into the P columns once PV(g - 1) has read them.  m is
+//               raised only when a chunk's max exceeds it by more than 8 (log2 units;
+//               then l and O are rescaled), so p <= 2^8.  A finished tile's epilogue runs
+//               in the next tile's first chunk.
 //   warp 8 + s  K producer of slot s: stages the slot's work items; TMA loads of the Q tile
 //               and of K, the chunk's two 64-key blocks per 16 KB stage, 2 stages.
 //   warp 14 + s V producer of slot s: TMA loads of V into 2 stages of 16 KB.
@@ -80,7 +79,6 @@ constexpr uint32_t kTmemO = 0;       // O: 64 fp32 columns
 constexpr uint32_t kTmemS = 64;      // S: 128 fp32 columns
 constexpr uint32_t kTmemP = 192;     // P: 128 keys as 64 bf16 pairs
 constexpr float kRescaleLog2 = 8.0f;  // m is raised when a chunk's max exceeds it by more
-constexpr float kRescaleBound = 256.0f;  // 2^kRescaleLog2
 constexpr uint32_t kOStageBytes = 32 * 128;  // one warp's 32 O rows, staged for a TMA store
 static_assert(kTmemS + 128 <= kTmemP && kTmemP + 64 <= kSlotCols, "TMEM map");
 
@@ -724,18 +722,14 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       }
       ptx::tc_fence_after();
       // All of S(g) into registers (loaded whatever the membership: a load under a
-      // condition makes the compiler keep both versions of the registers alive).
+      // condition makes the compiler keep both versions of the registers alive), then
+      // the S columns go straight back to the S issuer, so that S(g + 1) is computed
+      // while this chunk's exponentials run.
       //
       // The running max m follows one rule: it is raised to the chunk max cm when cm
       // exceeds it by more than kRescaleLog2, so every p = 2^(s - m) stays at or below
-      // 2^kRescaleLog2.  The chunk max itself is needed only on a row's first attended
-      // chunk (m = -inf) or when some p could pass that bound; so a chunk first takes its
-      // exponentials with m as it stands, and only when some row's sum of p exceeds
-      // 2^kRescaleLog2 (the one case where a single p may) is S loaded again, its max
-      // taken and the chunk redone.  m, p and l come out as with the max taken every
-      // time (up to a score within rounding of the bound).  A warp's rows share
-      // membership and key bits, so the branches are warp-uniform.  The S columns go
-      // back to the S issuer once the chunk stands.
+      // 2^kRescaleLog2 and O is rescaled only when m moves that far.  A warp's rows
+      // share membership and key bits, so the branches are warp-uniform.
       const uint32_t sbase = tmem + lane_addr + kTmemS;
       const bool att0 = (att_bits >> e0) & 1ull, att1 = (att_bits >> (e0 + 1)) & 1ull;
       const bool part = ((part_bits >> e0) & 3ull) != 0ull;
@@ -743,42 +737,31 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         if (att0) mask_scores(sbase, entry_mask(st, e0, half));
         if (att1) mask_scores(sbase + 64u, entry_mask(st, e0 + 1, half));
       }
-      float m_new = m_run;
-      bool take_max = __any_sync(0xffffffffu, m_run == -INFINITY);
       // P is written over the scores it came from (a0 and a1 hold P after the
       // exponentials), so that the TMEM stores read the registers the loads wrote
       uint32_t a0[32], b0[32], a1[32], b1[32];
-      float psum;
-      for (;;) {
-        ptx::tmem_ld32(sbase, a0);
-        ptx::tmem_ld32(sbase + 32u, b0);
-        ptx::tmem_ld32(sbase + 64u, a1);
-        ptx::tmem_ld32(sbase + 96u, b1);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence(a0);
-        ptx::reg_fence(b0);
-        ptx::reg_fence(a1);
-        ptx::reg_fence(b1);
-        if (take_max) {  // the chunk max over the keys this row attends (mk != 0 keeps one)
-          const float gm0 = group_max(a0, b0), gm1 = group_max(a1, b1);
-          const float cm = fmaxf(att0 ? gm0 : -INFINITY, att1 ? gm1 : -INFINITY);
-          const float cm2 = cm * sl2;  // scale > 0: the max of the scaled scores
-          m_new = cm2 > m_run + kRescaleLog2 ? cm2 : m_run;
-        }
-        const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
-        psum = 0.f;
-        if (att0) {
-          psum += group_exp(a0, b0, sc2, nm2);
-        }
-        if (att1) {
-          psum += group_exp(a1, b1, sc2, nm2);
-        }
-        // every p <= psum: a sum within the bound keeps m (a NaN sum takes the max path)
-        if (take_max || !__any_sync(0xffffffffu, !(psum <= kRescaleBound))) break;
-        take_max = true;
-      }
+      ptx::tmem_ld32(sbase, a0);
+      ptx::tmem_ld32(sbase + 32u, b0);
+      ptx::tmem_ld32(sbase + 64u, a1);
+      ptx::tmem_ld32(sbase + 96u, b1);
+      ptx::tmem_wait_ld();
+      ptx::reg_fence(a0);
+      ptx::reg_fence(b0);
+      ptx::reg_fence(a1);
+      ptx::reg_fence(b1);
       ptx::tc_fence_before();
       ptx::mbar_arrive(bar(kBarSFree));  // every thread
+      // the chunk max over the keys this row attends (a padded key holds -inf; an
+      // attended block keeps at least one key)
+      float cm = -INFINITY;
+      if (att0) cm = group_max(a0, b0);
+      if (att1) cm = fmaxf(cm, group_max(a1, b1));
+      const float cm2 = cm * sl2;  // scale > 0: the max of the scaled scores
+      const float m_new = cm2 > m_run + kRescaleLog2 ? cm2 : m_run;
+      const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
+      float psum = 0.f;
+      if (att0) psum += group_exp(a0, b0, sc2, nm2);
+      if (att1) psum += group_exp(a1, b1, sc2, nm2);
       const bool grew = m_new != m_run;
       const float alpha = grew ? ptx::ex2_approx(m_run - m_new) : 1.f;  // 2^-inf = 0
       const bool rescale = grew && l_run > 0.f;  // O holds this tile's earlier chunks
