@@ -48,6 +48,8 @@ _SIGNATURES = {
     "bsa_layout_free": (None, [ctypes.c_void_p]),
     "bsa_workspace_bytes": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int,
                                            ctypes.POINTER(ctypes.c_size_t)]),
+    "bsa_forward_workspace_bytes": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.POINTER(ctypes.c_size_t)]),
     "bsa_forward": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                    ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                    ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
@@ -227,21 +229,27 @@ def bsa_workspace_bytes(layout: Layout, B: int) -> int:
     return n.value
 
 
-def _workspace(layout: Layout, B: int, device):
+def bsa_forward_workspace_bytes(layout: Layout, B: int, d: int) -> int:
+    n = ctypes.c_size_t()
+    _check(lib.bsa_forward_workspace_bytes(layout.handle, B, d, ctypes.byref(n)), "bsa_forward_workspace_bytes")
+    return n.value
+
+
+def _workspace(layout: Layout, B: int, device, d: int = 64):
     import torch
-    key = (str(device), B)
+    key = (str(device), B, d)
     ws = layout._workspaces.get(key)
     if ws is None:
-        ws = torch.empty(bsa_workspace_bytes(layout, B), dtype=torch.uint8, device=device)
+        ws = torch.empty(bsa_forward_workspace_bytes(layout, B, d), dtype=torch.uint8, device=device)
         layout._workspaces[key] = ws
     return ws
 
 
 def bsa_forward(q, k, v, layout: Layout, key_mask=None, scale: Optional[float] = None, out=None,
                 lse=None, workspace=None, stream=None):
-    """O (bf16 [B,H,L,64]) and lse (fp32 [B,H,L]) of the block-sparse attention.
+    """O (bf16 [B,H,L,d]) and lse (fp32 [B,H,L]) of the block-sparse attention.
 
-    q, k, v: contiguous bf16 CUDA tensors [B, H, L, 64].  key_mask: optional
+    q, k, v: contiguous bf16 CUDA tensors [B, H, L, d], d = 64 or 128.  key_mask: optional
     uint8 CUDA tensor [B, L] (1 = keep).  workspace: optional uint8 CUDA tensor
     of at least bsa_workspace_bytes(layout, B) bytes, any contents; when
     omitted a cached one of the layout is used (not safe for concurrent calls
@@ -262,7 +270,7 @@ def bsa_forward(q, k, v, layout: Layout, key_mask=None, scale: Optional[float] =
         if key_mask.dtype != torch.uint8 or tuple(key_mask.shape) != (B, L) or not key_mask.is_contiguous():
             raise ValueError("key_mask must be a contiguous uint8 tensor [B, L]")
     if workspace is None:
-        workspace = _workspace(layout, B, q.device)
+        workspace = _workspace(layout, B, q.device, d)
     code = lib.bsa_forward(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, H, L, d, layout.handle,
                            key_mask.data_ptr() if key_mask is not None else None,
                            ctypes.c_float(scale if scale is not None else 0.0), out.data_ptr(),

@@ -47,6 +47,7 @@
 #include <algorithm>
 #include <cmath>
 #include <mutex>
+#include <type_traits>
 
 #include "bsa_internal.h"
 #include "sm100_ptx.cuh"
@@ -55,38 +56,15 @@
 
 namespace bsa {
 
-constexpr int kSlots = 2;
-constexpr int kThreads = 512;
-constexpr int kKProdWarp = 8;  // + slot
-constexpr int kSWarp = 10;     // + slot; warp 10 allocates and frees TMEM
-constexpr int kPvWarp = 12;    // + slot
-constexpr int kVProdWarp = 14;  // + slot
-// Register split: softmax warpgroups 0-1 take kSoftmaxRegs, warpgroups 2-3 (producers
-// and issuers) kOtherRegs; 2 * 128 * (200 + 56) = 65536 = 512 threads x 128.
-constexpr uint32_t kSoftmaxRegs = 200;
-constexpr uint32_t kOtherRegs = 56;
-static_assert(2 * 128 * (kSoftmaxRegs + kOtherRegs) <= 65536, "register split exceeds the launch budget");
 constexpr int kItemRing = 4;  // work items a slot's K producer may publish ahead
 constexpr int kChunkEnt = 2;  // union entries (64-key blocks) per chunk
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
-constexpr uint32_t kBlkBytes = 64 * 128;                 // one 64 x 64 bf16 block
-constexpr uint32_t kQBytes = 2 * kBlkBytes;              // 128-row Q tile
-constexpr uint32_t kStageBytes = kChunkEnt * kBlkBytes;  // one chunk of K (or V)
+constexpr uint32_t kBoxBytes = 64 * 128;  // one TMA box: 64 rows x 64 bf16 columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSlotCols = 256;  // slot s owns columns [256 s, 256 s + 256)
-constexpr uint32_t kTmemO = 0;       // O: 64 fp32 columns
-constexpr uint32_t kTmemS = 64;      // S: 128 fp32 columns
-constexpr uint32_t kTmemP = 192;     // P: 128 keys as 64 bf16 pairs
 constexpr float kRescaleLog2 = 8.0f;  // m is raised when a chunk's max exceeds it by more
-constexpr uint32_t kOStageBytes = 32 * 128;  // one warp's 32 O rows, staged for a TMA store
-static_assert(kTmemS + 128 <= kTmemP && kTmemP + 64 <= kSlotCols, "TMEM map");
+constexpr uint32_t kOStageBytes = 32 * 128;  // one warp's 32 O rows of one 64-column half
 
-// shared memory map of one slot (offsets from its 1024-aligned base)
-constexpr uint32_t kSmemQ = 0;  // 2 Q tiles; a finished tile's buffer also stages its O
-constexpr uint32_t kSmemK = kSmemQ + 2 * kQBytes;
-constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
-constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
 enum : int {
   kBarQFull = 0,                     // [Q stage] the tile's Q landed (TMA)
   kBarQEmpty = kBarQFull + 2,        // [Q stage] 4 softmax warps: the tile's S MMAs and its
@@ -94,18 +72,18 @@ enum : int {
   kBarKFull = kBarQEmpty + 2,        // [K stage] K of the chunk landed (TMA)
   kBarKFree = kBarKFull + kKStages,  // [K stage] MMA commit after the chunk's S
   kBarVFull = kBarKFree + kKStages,  // [V stage] V of the chunk landed (TMA)
-  kBarVFree = kBarVFull + kVStages,  // [V stage] MMA commit after the chunk's PV: the V stage
-                                     // and the P columns are reusable, O holds chunk g
+  kBarVFree = kBarVFull + kVStages,  // [V stage] MMA commits after the chunk's PV (one per
+                                     // PV issuer): the V stage and the P columns are
+                                     // reusable, O holds chunk g
   kBarSFull = kBarVFree + kVStages,  // MMA commit after S: the S columns are readable
   kBarSFree = kBarSFull + 1,         // the 128 softmax threads are done with S
   kBarPFull = kBarSFree + 1,         // the 128 softmax threads have stored P
-  kBarMmaFinal = kBarPFull + 1,      // [2 issuers]
-  kBarItemFull = kBarMmaFinal + 2,   // [item ring] the K producer published a work item
-  kBarItemEmpty = kBarItemFull + kItemRing,  // [item ring] 7 arrivals: V producer, both
-                                             // issuers, the four softmax warps
+  kBarMmaFinal = kBarPFull + 1,      // [S issuer, PV issuers]
+  kBarItemFull = kBarMmaFinal + 3,   // [item ring] the K producer published a work item
+  kBarItemEmpty = kBarItemFull + kItemRing,  // [item ring] one arrival from every reader:
+                                             // V producer, the issuers, the softmax warps
   kNumBars = kBarItemEmpty + kItemRing
 };
-constexpr uint32_t kItemReaders = 7;
 constexpr uint32_t kWarpArrivals = 4;     // Q release: one arrival per softmax warp
 constexpr uint32_t kThreadArrivals = 128;  // S free, P full: every softmax thread arrives
 
@@ -125,13 +103,63 @@ struct ItemStage {
   unsigned long long kb[kMaxItemEntries];  // all ones without a key mask
 };
 static_assert(sizeof(ItemStage) % 16 == 0, "stage alignment");
-constexpr uint32_t kSmemItems = (kSmemBar + 8 * kNumBars + 15) & ~15u;  // ItemStage[kItemRing]
-constexpr uint32_t kSlotBytes = (kSmemItems + sizeof(ItemStage) * kItemRing + 1023) & ~1023u;
-constexpr uint32_t kSmemMisc = kSlots * kSlotBytes;  // u32 TMEM base, int abort flag
-constexpr uint32_t kSmemUsed = kSmemMisc + 16;
-constexpr uint32_t kSmemAlloc = kSmemUsed + 1024;  // slack for 1024-byte alignment
-static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
-static_assert(kQBytes == 4 * kOStageBytes, "a Q buffer stages the four warps' O rows");
+
+// What depends on the head dim d (64 or 128).  Operands in shared memory are kept as
+// d / 64 column halves of 64 bf16 (one 128-byte swizzle atom wide), each half laid
+// out as at d = 64: a Q buffer is [half][128 rows][64], a K or V stage
+// [half][entry][64 keys][64].  TMEM of a slot: O (d columns), S (128), P (64, bf16
+// pairs).
+//   d = 64:  two slots per CTA, 512 threads: softmax warps 0-7 (slot = warp / 4),
+//            K producer 8 + s, S issuer 10 + s, PV issuer 12 + s, V producer 14 + s.
+//   d = 128: one slot (a second would need 256 KB of shared memory), 384 threads:
+//            softmax warps 0-3, K producer 4, S issuer 5, PV issuers 6 and 7 (one per
+//            column half of O, so that each issues eight N = 64 MMAs a chunk), V
+//            producer 8; warps 9-11 only take part in the register split.
+template <int kD>
+struct FwdCfg {
+  static_assert(kD == 64 || kD == 128, "head dim");
+  static constexpr int kHalves = kD / 64;
+  static constexpr int kSlots = kD == 64 ? 2 : 1;
+  static constexpr int kThreads = kD == 64 ? 512 : 384;
+  static constexpr int kPvIssuers = kHalves;  // per slot
+  static constexpr int kKProdWarp = 4 * kSlots;  // + slot
+  static constexpr int kSWarp = kKProdWarp + kSlots;  // + slot; the first allocates and frees TMEM
+  static constexpr int kPvWarp = kSWarp + kSlots;     // + slot * kPvIssuers + half
+  static constexpr int kVProdWarp = kPvWarp + kSlots * kPvIssuers;  // + slot
+  static_assert(kVProdWarp + kSlots <= kThreads / 32, "role warps");
+  // Register split: the softmax warpgroups take kSoftmaxRegs, the other warpgroups
+  // kOtherRegs; the sum stays within the launch's pool (threads x registers a thread).
+  static constexpr uint32_t kSoftmaxRegs = kD == 64 ? 200 : 232;
+  static constexpr uint32_t kOtherRegs = 56;
+  static constexpr uint32_t kLaunchRegs = (65536 / kThreads) & ~7u;
+  static_assert(kSlots * 128 * kSoftmaxRegs + (kThreads - kSlots * 128) * kOtherRegs <= kThreads * kLaunchRegs,
+                "register split exceeds the launch budget");
+  // the noinline wait paths of the two register budgets (one instantiation per budget)
+  static constexpr int kSoftRegion = kD == 64 ? 1 : 3;
+  static constexpr int kRoleRegion = kD == 64 ? 2 : 4;
+  static constexpr uint32_t kItemReaders = 4 + 2 + kPvIssuers;  // softmax warps, V producer, S issuer, PV
+  static constexpr uint32_t kQHalfBytes = 2 * kBoxBytes;          // one column half of the 128-row tile
+  static constexpr uint32_t kQBytes = kHalves * kQHalfBytes;
+  static constexpr uint32_t kStageHalfBytes = kChunkEnt * kBoxBytes;  // one column half of a chunk
+  static constexpr uint32_t kStageBytes = kHalves * kStageHalfBytes;
+  static constexpr uint32_t kTmemO = 0;
+  static constexpr uint32_t kTmemS = kD;
+  static constexpr uint32_t kTmemP = kD + 128;
+  static constexpr uint32_t kSlotCols = 256;  // slot s owns columns from 256 s
+  static_assert(kTmemP + 64 <= (kSlots == 2 ? kSlotCols : kTmemCols), "TMEM map");
+  static constexpr int kRecFloats = rec_floats(kD);
+  // shared memory map of one slot (offsets from its 1024-aligned base)
+  static constexpr uint32_t kSmemQ = 0;  // 2 Q tiles; a finished tile's buffer also stages its O
+  static constexpr uint32_t kSmemK = kSmemQ + 2 * kQBytes;
+  static constexpr uint32_t kSmemV = kSmemK + kKStages * kStageBytes;
+  static constexpr uint32_t kSmemBar = kSmemV + kVStages * kStageBytes;
+  static constexpr uint32_t kSmemItems = (kSmemBar + 8 * kNumBars + 15) & ~15u;  // ItemStage[kItemRing]
+  static constexpr uint32_t kSlotBytes = (kSmemItems + sizeof(ItemStage) * kItemRing + 1023) & ~1023u;
+  static constexpr uint32_t kSmemMisc = kSlots * kSlotBytes;  // u32 TMEM base, int abort flag
+  static constexpr uint32_t kSmemAlloc = kSmemMisc + 16 + 1024;  // + slack for 1024-byte alignment
+  static_assert(kSmemAlloc <= 227 * 1024, "shared memory budget");
+  static_assert(kQHalfBytes == 4 * kOStageBytes, "a Q buffer half stages the four warps' O rows");
+};
 
 // Where one slot's roles find their resources.  Work items are handed out
 // dynamically: the slot's K producer takes the next index from a global counter and
@@ -169,10 +197,11 @@ __device__ __forceinline__ uint32_t bar_at(uint32_t bars, int i) { return bars +
 
 // The slot's k-th work item for an issuer (one thread): its index and entry count.
 // The stage is released at once.
+template <int kRegion>
 __device__ __forceinline__ int take_item_one(const Slot& sl, uint32_t k, int* count, volatile int* abort_flag,
                                              uint64_t timeout_ns) {
   const uint32_t i = k % kItemRing;
-  if (!wait_one<2>(bar_at(sl.bars, kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
+  if (!wait_one<kRegion>(bar_at(sl.bars, kBarItemFull + i), (k / kItemRing) & 1u, abort_flag, timeout_ns))
     return kItemAbort;
   const ItemStage& st = sl.items[i];
   const int t = st.t;
@@ -200,12 +229,13 @@ __device__ __forceinline__ void release_item_warp(const Slot& sl, uint32_t k, in
 
 // Lets every copy a producer thread issued land before the CTA exits (after an abort):
 // the last issue into ring slot s of n issues had index s + R * floor((n - 1 - s) / R).
+template <int kRegion>
 __device__ __forceinline__ void drain_ring(uint32_t bars, int first_bar, uint32_t n, uint32_t ring,
                                            volatile int* abort_flag, uint64_t timeout_ns) {
   for (uint32_t s = 0; s < ring; ++s) {
     if (n > s) {
       const uint32_t last = s + ring * ((n - 1u - s) / ring);
-      wait_force<2>(bar_at(bars, first_bar + static_cast<int>(s)), (last / ring) & 1u, abort_flag, timeout_ns);
+      wait_force<kRegion>(bar_at(bars, first_bar + static_cast<int>(s)), (last / ring) & 1u, abort_flag, timeout_ns);
     }
   }
 }
@@ -237,8 +267,12 @@ __host__ __device__ __forceinline__ int2 item_of(int t, int B, int ns, int nn, i
 // K producer, one warp.  Per work item the warp stages the item, its union entries and
 // their key-padding bits in the slot's item ring; then lane 0 issues the loads: the Q
 // tile into Q buffer (tile % 2) once the tile two back has released it, and for each
-// chunk g its K blocks into K stage g % 2 once S(g - 2) is done.
+// chunk g its K blocks into K stage g % 2 once S(g - 2) is done.  Each 64-row block
+// goes in d / 64 boxes, one per column half.
+template <int kD>
 __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, int lane, volatile int* abort_flag) {
+  using C = FwdCfg<kD>;
+  constexpr int R = C::kRoleRegion;
   const uint32_t sQ = sl.sQ, sK = sl.sK, bars = sl.bars;
   auto bar = [&](int i) { return bar_at(bars, i); };
   const uint64_t pol_q = ptx::policy_evict_first();
@@ -253,7 +287,7 @@ __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, i
     const uint32_t ii = k % kItemRing;
     bool ok = true;
     if (lane == 0)
-      ok = wait_one<2>(bar(kBarItemEmpty + static_cast<int>(ii)), ((k / kItemRing) & 1u) ^ 1u, abort_flag,
+      ok = wait_one<R>(bar(kBarItemEmpty + static_cast<int>(ii)), ((k / kItemRing) & 1u) ^ 1u, abort_flag,
                           p.timeout_ns);
     if (!__shfl_sync(0xffffffffu, ok, 0)) {
       alive = false;
@@ -322,25 +356,33 @@ __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, i
       const int row0 = (st.b * p.H + w.h) * p.L;
       const int qa = st.qa, qb = st.qb;
       const uint32_t qs = nq & 1u;
-      if (!wait_one<2>(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+      if (!wait_one<R>(bar(kBarQEmpty + qs), ((nq >> 1) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
         alive = false;
       } else {
-        ptx::mbar_arrive_expect_tx(bar(kBarQFull + qs), kQBytes);
-        ptx::tma_load_2d(sQ + qs * kQBytes, &p.tm_q, bar(kBarQFull + qs), 0, row0 + qa * 64, pol_q);
-        ptx::tma_load_2d(sQ + qs * kQBytes + kBlkBytes, &p.tm_q, bar(kBarQFull + qs), 0,
-                         row0 + (qb >= 0 ? qb : qa) * 64, pol_q);
+        ptx::mbar_arrive_expect_tx(bar(kBarQFull + qs), C::kQBytes);
+#pragma unroll
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          const uint32_t dst = sQ + qs * C::kQBytes + hf * C::kQHalfBytes;
+          ptx::tma_load_2d(dst, &p.tm_q, bar(kBarQFull + qs), 64 * hf, row0 + qa * 64, pol_q);
+          ptx::tma_load_2d(dst + kBoxBytes, &p.tm_q, bar(kBarQFull + qs), 64 * hf,
+                           row0 + (qb >= 0 ? qb : qa) * 64, pol_q);
+        }
         ++nq;
         for (int e0 = 0; e0 < w.count; e0 += kChunkEnt) {
           const int ne = min(kChunkEnt, w.count - e0);
           const uint32_t ks = nk % kKStages;
-          if (!wait_one<2>(bar(kBarKFree + ks), ((nk / kKStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+          if (!wait_one<R>(bar(kBarKFree + ks), ((nk / kKStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
             alive = false;
             break;
           }
-          ptx::mbar_arrive_expect_tx(bar(kBarKFull + ks), kBlkBytes * ne);
-          for (int x = 0; x < ne; ++x)
-            ptx::tma_load_2d(sK + ks * kStageBytes + x * kBlkBytes, &p.tm_k, bar(kBarKFull + ks), 0,
-                             row0 + static_cast<int>(st.ent[e0 + x] & kEntColMask) * 64, pol_kv);
+          ptx::mbar_arrive_expect_tx(bar(kBarKFull + ks), kBoxBytes * C::kHalves * ne);
+          for (int x = 0; x < ne; ++x) {
+            const int krow = row0 + static_cast<int>(st.ent[e0 + x] & kEntColMask) * 64;
+#pragma unroll
+            for (int hf = 0; hf < C::kHalves; ++hf)
+              ptx::tma_load_2d(sK + ks * C::kStageBytes + hf * C::kStageHalfBytes + x * kBoxBytes, &p.tm_k,
+                               bar(kBarKFull + ks), 64 * hf, krow, pol_kv);
+          }
           ++nk;
         }
       }
@@ -355,26 +397,29 @@ __device__ __forceinline__ void k_producer(const FwdParams& p, const Slot& sl, i
     // Every slot's K producer counts itself out once it has drawn its last index; the
     // last one resets both counters, so the workspace is left as the call found it.
     __threadfence();
-    if (atomicAdd(p.sched + 1, 1) == kSlots * static_cast<int>(gridDim.x) - 1) {
+    if (atomicAdd(p.sched + 1, 1) == C::kSlots * static_cast<int>(gridDim.x) - 1) {
       p.sched[0] = 0;
       p.sched[1] = 0;
     }
   } else {
-    drain_ring(bars, kBarQFull, nq, 2u, abort_flag, p.timeout_ns);
-    drain_ring(bars, kBarKFull, nk, static_cast<uint32_t>(kKStages), abort_flag, p.timeout_ns);
+    drain_ring<R>(bars, kBarQFull, nq, 2u, abort_flag, p.timeout_ns);
+    drain_ring<R>(bars, kBarKFull, nk, static_cast<uint32_t>(kKStages), abort_flag, p.timeout_ns);
   }
 }
 
 // V producer, one warp: follows the item ring and loads V of chunk g into V stage
 // g % 2 once PV(g - 2) is done, releasing each item after its last load.
+template <int kD>
 __device__ __forceinline__ void v_producer(const FwdParams& p, const Slot& sl, int lane, volatile int* abort_flag) {
+  using C = FwdCfg<kD>;
+  constexpr int R = C::kRoleRegion;
   const uint32_t sV = sl.sV, bars = sl.bars;
   auto bar = [&](int i) { return bar_at(bars, i); };
   const uint64_t pol_kv = ptx::policy_evict_last();
   uint32_t nv = 0;
   bool alive = true;
   for (uint32_t k = 0; alive; ++k) {
-    const int t = take_item_warp<2>(sl, k, abort_flag, p.timeout_ns);
+    const int t = take_item_warp<R>(sl, k, abort_flag, p.timeout_ns);
     if (t < 0) {
       if (t == kItemAbort) alive = false;
       break;
@@ -385,27 +430,35 @@ __device__ __forceinline__ void v_producer(const FwdParams& p, const Slot& sl, i
       for (int e0 = 0; e0 < st.w.count; e0 += kChunkEnt) {
         const int ne = min(kChunkEnt, st.w.count - e0);
         const uint32_t vs = nv % kVStages;
-        if (!wait_one<2>(bar(kBarVFree + vs), ((nv / kVStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
+        if (!wait_one<R>(bar(kBarVFree + vs), ((nv / kVStages) & 1u) ^ 1u, abort_flag, p.timeout_ns)) {
           alive = false;
           break;
         }
-        ptx::mbar_arrive_expect_tx(bar(kBarVFull + vs), kBlkBytes * ne);
-        for (int x = 0; x < ne; ++x)
-          ptx::tma_load_2d(sV + vs * kStageBytes + x * kBlkBytes, &p.tm_v, bar(kBarVFull + vs), 0,
-                           row0 + static_cast<int>(st.ent[e0 + x] & kEntColMask) * 64, pol_kv);
+        ptx::mbar_arrive_expect_tx(bar(kBarVFull + vs), kBoxBytes * C::kHalves * ne);
+        for (int x = 0; x < ne; ++x) {
+          const int vrow = row0 + static_cast<int>(st.ent[e0 + x] & kEntColMask) * 64;
+#pragma unroll
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            ptx::tma_load_2d(sV + vs * C::kStageBytes + hf * C::kStageHalfBytes + x * kBoxBytes, &p.tm_v,
+                             bar(kBarVFull + vs), 64 * hf, vrow, pol_kv);
+        }
         ++nv;
       }
     }
     alive = __shfl_sync(0xffffffffu, alive, 0);
     release_item_warp(sl, k, lane);
   }
-  if (lane == 0 && !alive) drain_ring(bars, kBarVFull, nv, static_cast<uint32_t>(kVStages), abort_flag, p.timeout_ns);
+  if (lane == 0 && !alive) drain_ring<R>(bars, kBarVFull, nv, static_cast<uint32_t>(kVStages), abort_flag, p.timeout_ns);
 }
 
 // tcgen05 S issuer, one thread.  S(g) = Q K_g^T (N = 64 per key block of the chunk) into
 // the S columns once K(g) has landed and the softmax has loaded S(g - 1).  Its commits
-// signal S full and release K stage g % 2.
+// signal S full and release K stage g % 2.  The head dim runs in steps of 16: four per
+// 64-column half of Q and K.
+template <int kD>
 __device__ __forceinline__ void s_issuer(const FwdParams& p, const Slot& sl, volatile int* abort_flag) {
+  using C = FwdCfg<kD>;
+  constexpr int R = C::kRoleRegion;
   const uint32_t sQ = sl.sQ, sK = sl.sK, bars = sl.bars, tmem = sl.tmem;
   auto bar = [&](int i) { return bar_at(bars, i); };
   constexpr uint32_t kIdescS2 = ptx::idesc_bf16_f32(128, 128, false);
@@ -417,59 +470,67 @@ __device__ __forceinline__ void s_issuer(const FwdParams& p, const Slot& sl, vol
   bool alive = true;
   for (uint32_t nq = 0; alive; ++nq) {
     int count = 0;
-    if (take_item_one(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
+    if (take_item_one<R>(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
     const uint32_t qs = nq & 1u;
-    if (!wait_one<2>(bar(kBarQFull + qs), (nq >> 1) & 1u, abort_flag, p.timeout_ns)) break;
-    const uint64_t dq = dq0 + qs * (kQBytes >> 4);
+    if (!wait_one<R>(bar(kBarQFull + qs), (nq >> 1) & 1u, abort_flag, p.timeout_ns)) break;
+    const uint64_t dq = dq0 + qs * (C::kQBytes >> 4);
     for (int e0 = 0; e0 < count; e0 += kChunkEnt, ++g) {
       const uint32_t ks = g % kKStages;
-      if (!wait_one<2>(bar(kBarKFull + ks), (g / kKStages) & 1u, abort_flag, p.timeout_ns) ||
-          (g > 0 && !wait_one<2>(bar(kBarSFree), (g - 1u) & 1u, abort_flag, p.timeout_ns))) {
+      if (!wait_one<R>(bar(kBarKFull + ks), (g / kKStages) & 1u, abort_flag, p.timeout_ns) ||
+          (g > 0 && !wait_one<R>(bar(kBarSFree), (g - 1u) & 1u, abort_flag, p.timeout_ns))) {
         alive = false;
         break;
       }
       ptx::tc_fence_after();
-      const uint64_t dk = dk0 + ks * (kStageBytes >> 4);
-      const uint32_t d = tmem + kTmemS;
+      const uint64_t dk = dk0 + ks * (C::kStageBytes >> 4);
+      const uint32_t d = tmem + C::kTmemS;
       const uint32_t idesc = count - e0 >= 2 ? kIdescS2 : kIdescS1;
-      ptx::mma_ss(d, dq, dk, idesc, 0u);  // head dim 64 = 4 x 16: +32 bytes per step
-      ptx::mma_ss(d, dq + 2, dk + 2, idesc, 1u);
-      ptx::mma_ss(d, dq + 4, dk + 4, idesc, 1u);
-      ptx::mma_ss(d, dq + 6, dk + 6, idesc, 1u);
+#pragma unroll
+      for (int hf = 0; hf < C::kHalves; ++hf) {  // 64 columns = 4 steps of 16: +32 bytes a step
+        const uint64_t dqh = dq + hf * (C::kQHalfBytes >> 4), dkh = dk + hf * (C::kStageHalfBytes >> 4);
+        ptx::mma_ss(d, dqh, dkh, idesc, hf > 0 ? 1u : 0u);
+        ptx::mma_ss(d, dqh + 2, dkh + 2, idesc, 1u);
+        ptx::mma_ss(d, dqh + 4, dkh + 4, idesc, 1u);
+        ptx::mma_ss(d, dqh + 6, dkh + 6, idesc, 1u);
+      }
       ptx::mma_commit(bar(kBarSFull));
       ptx::mma_commit(bar(kBarKFree + static_cast<int>(ks)));
     }
   }
   // Every MMA this thread issued must finish before TMEM is released.
   ptx::mma_commit(bar(kBarMmaFinal));
-  wait_force<2>(bar(kBarMmaFinal), 0, abort_flag, p.timeout_ns);
+  wait_force<R>(bar(kBarMmaFinal), 0, abort_flag, p.timeout_ns);
 }
 
-// tcgen05 PV issuer, one thread.  Chunk g: once V(g) has landed and the softmax has
-// written P(g), O (+)= P(g) V_g, 16 keys per MMA (the first MMA of a tile overwrites
-// O), then one commit that frees V stage g % 2 and the P columns and tells the softmax
-// warps that O holds chunk g.
-__device__ __forceinline__ void pv_issuer(const FwdParams& p, const Slot& sl, volatile int* abort_flag) {
-  const uint32_t sV = sl.sV, bars = sl.bars, tmem = sl.tmem;
+// tcgen05 PV issuer, one thread, for the 64 columns of O from 64 hf.  Chunk g: once
+// V(g) has landed and the softmax has written P(g), O (+)= P(g) V_g, 16 keys per MMA
+// (the first MMA of a tile overwrites O), then one commit that (with the other
+// column half's, at d = 128) frees V stage g % 2 and the P columns and tells the
+// softmax warps that O holds chunk g.
+template <int kD>
+__device__ __forceinline__ void pv_issuer(const FwdParams& p, const Slot& sl, int hf, volatile int* abort_flag) {
+  using C = FwdCfg<kD>;
+  constexpr int R = C::kRoleRegion;
+  const uint32_t sV = sl.sV + static_cast<uint32_t>(hf) * C::kStageHalfBytes, bars = sl.bars, tmem = sl.tmem;
   auto bar = [&](int i) { return bar_at(bars, i); };
   constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 64, true);
   const uint64_t dv0 = ptx::smem_desc_sw128(sV, 0);
-  const uint32_t d = tmem + kTmemO;
+  const uint32_t d = tmem + C::kTmemO + 64u * static_cast<uint32_t>(hf);
   uint32_t g = 0;
   bool alive = true;
   for (uint32_t nq = 0; alive; ++nq) {
     int count = 0;
-    if (take_item_one(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
+    if (take_item_one<R>(sl, nq, &count, abort_flag, p.timeout_ns) < 0) break;
     for (int e0 = 0; e0 < count; e0 += kChunkEnt, ++g) {
       const uint32_t vs = g % kVStages;
-      if (!wait_one<2>(bar(kBarVFull + vs), (g / kVStages) & 1u, abort_flag, p.timeout_ns) ||
-          !wait_one<2>(bar(kBarPFull), g & 1u, abort_flag, p.timeout_ns)) {
+      if (!wait_one<R>(bar(kBarVFull + vs), (g / kVStages) & 1u, abort_flag, p.timeout_ns) ||
+          !wait_one<R>(bar(kBarPFull), g & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
       ptx::tc_fence_after();
-      const uint64_t dv = dv0 + vs * (kStageBytes >> 4);
-      const uint32_t a = tmem + kTmemP;
+      const uint64_t dv = dv0 + vs * (C::kStageBytes >> 4);
+      const uint32_t a = tmem + C::kTmemP;
       ptx::mma_ts(d, a, dv, kIdescPV, e0 == 0 ? 0u : 1u);  // 16 keys per MMA
       ptx::mma_ts(d, a + 8u, dv + (2048u >> 4), kIdescPV, 1u);
       ptx::mma_ts(d, a + 16u, dv + (4096u >> 4), kIdescPV, 1u);
@@ -483,8 +544,8 @@ __device__ __forceinline__ void pv_issuer(const FwdParams& p, const Slot& sl, vo
       ptx::mma_commit(bar(kBarVFree + static_cast<int>(vs)));
     }
   }
-  ptx::mma_commit(bar(kBarMmaFinal + 1));
-  wait_force<2>(bar(kBarMmaFinal + 1), 0, abort_flag, p.timeout_ns);
+  ptx::mma_commit(bar(kBarMmaFinal + 1 + hf));
+  wait_force<R>(bar(kBarMmaFinal + 1 + hf), 0, abort_flag, p.timeout_ns);
 }
 
 // What the epilogue of a finished tile needs; it runs in the first chunk of the next
@@ -496,72 +557,90 @@ struct TileDone {
 
 // Epilogue of a finished tile (its last PV is done): normalise O and store it with
 // lse, or, for a chunk of a split tile, its partial record.  O rows go through the
-// tile's own Q buffer (its S MMAs are complete) and one TMA store per warp.  Out of
-// line: it runs once per tile and would otherwise crowd the chunk loop's code and
-// registers (only the softmax warps call it, so it is compiled to their budget).
+// tile's own Q buffer (its S MMAs are complete) and one TMA store per warp and column
+// half.  Out of line: it runs once per tile and would otherwise crowd the chunk loop's
+// code and registers (only the softmax warps call it, so it is compiled to their
+// budget).
+template <int kD>
 __device__ __noinline__ void tile_epilogue(const FwdParams& p, const TileDone& td, const ItemStage& st,
                                               const Slot& sl, uint32_t obase, int warp, int lane) {
+  using C = FwdCfg<kD>;
   const int r = (warp & 3) * 32 + lane;
   const int half = r >> 6;
   const int tb = st.b;
   const WorkItem& tw = st.w;
   const int tqa = st.qa, tqb = st.qb;
   const int tbh = tb * p.H + tw.h;
-  float o[64];
-  {
-    uint32_t raw[2][32];
-    ptx::tmem_ld32(obase, raw[0]);
-    ptx::tmem_ld32(obase + 32u, raw[1]);
-    ptx::tmem_wait_ld();
-    ptx::reg_fence(raw[0]);
-    ptx::reg_fence(raw[1]);
-#pragma unroll
-    for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(raw[c >> 5][c & 31]);
-  }
   const float m = td.m, l = td.l;
   const bool row_active = half == 0 || tqb >= 0;
   const int qblk = half ? tqb : tqa;
   const size_t row = static_cast<size_t>(tbh) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
   if (tw.split < 0) {
     if (row_active) {  // warp-uniform: a warp's 32 rows lie in one half
-      // O rows through this warp's quarter of the tile's Q buffer (128-byte swizzle:
-      // 16-byte chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)), then one TMA store
-      // of the warp's 32 x 64 tile.
+      // O rows through this warp's quarter of each column half of the tile's Q buffer
+      // (128-byte swizzle: 16-byte chunk j of row r at r * 128 + ((j ^ (r % 8)) * 16)),
+      // then one TMA store of the warp's 32 x 64 box per column half.
       const float inv = l > 0.f ? ptx::rcp_approx(l) : 0.f;
       const uint64_t inv2 = ptx::pack2(inv, inv);
       const uint32_t qs = td.k & 1u;
-      uint8_t* stg = sl.q_generic + qs * kQBytes + (warp & 3) * kOStageBytes;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        uint32_t w4[4];
+      for (int hf = 0; hf < C::kHalves; ++hf) {
+        float o[64];
+        {
+          uint32_t raw[2][32];
+          ptx::tmem_ld32(obase + 64u * hf, raw[0]);
+          ptx::tmem_ld32(obase + 64u * hf + 32u, raw[1]);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(raw[0]);
+          ptx::reg_fence(raw[1]);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float y0, y1;
-          ptx::unpack2(ptx::fmul2(ptx::pack2(o[8 * j + 2 * q], o[8 * j + 2 * q + 1]), inv2), y0, y1);
-          w4[q] = pack_bf16x2(y0, y1);
+          for (int c = 0; c < 64; ++c) o[c] = __uint_as_float(raw[c >> 5][c & 31]);
         }
-        const uint4 u = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) = u;
+        const uint32_t off = qs * C::kQBytes + hf * C::kQHalfBytes + (warp & 3) * kOStageBytes;
+        uint8_t* stg = sl.q_generic + off;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float y0, y1;
+            ptx::unpack2(ptx::fmul2(ptx::pack2(o[8 * j + 2 * q], o[8 * j + 2 * q + 1]), inv2), y0, y1);
+            w4[q] = pack_bf16x2(y0, y1);
+          }
+          const uint4 u = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) = u;
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0)
+          ptx::tma_store_2d(&p.tm_o, sl.sQ + off, 64 * hf, static_cast<int>(row - static_cast<size_t>(r & 31)));
       }
-      ptx::fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        ptx::tma_store_2d(&p.tm_o, sl.sQ + qs * kQBytes + (warp & 3) * kOStageBytes, 0,
-                          static_cast<int>(row - static_cast<size_t>(r & 31)));
-        ptx::bulk_commit_group();
-      }
+      if (lane == 0) ptx::bulk_commit_group();
       p.lse[row] = l > 0.f ? (m + ptx::lg2_approx(l)) * kLn2 : -INFINITY;
     }
     return;
   }
   // ---- split chunk: its partial record (unnormalised O, m, l)
-  float* rec = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec) * kRecFloats;
-  float4* orow = reinterpret_cast<float4*>(rec + r * 64);
+  float* rec = p.partials + (static_cast<size_t>(tb) * p.n_records + tw.rec) * C::kRecFloats;
+  float4* orow = reinterpret_cast<float4*>(rec + r * kD);
 #pragma unroll
-  for (int v4 = 0; v4 < 16; ++v4)
-    orow[v4] = make_float4(o[v4 * 4 + 0], o[v4 * 4 + 1], o[v4 * 4 + 2], o[v4 * 4 + 3]);
-  rec[kTileRows * 64 + r] = l > 0.f ? m : -INFINITY;
-  rec[kTileRows * 64 + kTileRows + r] = l;
+  for (int hf = 0; hf < C::kHalves; ++hf) {
+    uint32_t raw[2][32];
+    ptx::tmem_ld32(obase + 64u * hf, raw[0]);
+    ptx::tmem_ld32(obase + 64u * hf + 32u, raw[1]);
+    ptx::tmem_wait_ld();
+    ptx::reg_fence(raw[0]);
+    ptx::reg_fence(raw[1]);
+#pragma unroll
+    for (int v4 = 0; v4 < 16; ++v4) {
+      const int c = v4 * 4;
+      orow[hf * 16 + v4] = make_float4(__uint_as_float(raw[c >> 5][c & 31]), __uint_as_float(raw[c >> 5][(c & 31) + 1]),
+                                       __uint_as_float(raw[c >> 5][(c & 31) + 2]),
+                                       __uint_as_float(raw[c >> 5][(c & 31) + 3]));
+    }
+  }
+  rec[kTileRows * kD + r] = l > 0.f ? m : -INFINITY;
+  rec[kTileRows * kD + kTileRows + r] = l;
 }
 
 // Releases the Q buffer of the tile whose epilogue ran last: its O store (if any)
@@ -582,8 +661,10 @@ __device__ __forceinline__ void mask_group(uint32_t (&a)[32], uint32_t (&b)[32],
   }
 }
 
-// Rare paths, out of line so that the chunk loop's code stays small (softmax warps only).
+// Rare paths, out of line so that the chunk loop's code stays small (softmax warps
+// only; one instantiation per head dim, as the softmax register budget differs).
 // Scores of padded keys of one 64-key group of this warp's rows set to -inf in TMEM.
+template <int kD>
 __device__ __noinline__ void mask_scores(uint32_t taddr, unsigned long long mk) {
   uint32_t a[32], b[32];
   ptx::tmem_ld32(taddr, a);
@@ -597,11 +678,12 @@ __device__ __noinline__ void mask_scores(uint32_t taddr, unsigned long long mk) 
   ptx::tmem_wait_st();
 }
 
-// O (64 columns of this warp's rows) scaled by alpha in TMEM; the caller's next
+// O (d columns of this warp's rows) scaled by alpha in TMEM; the caller's next
 // tcgen05.wait::st covers the stores.
+template <int kD>
 __device__ __noinline__ void rescale_o(uint32_t obase, float alpha) {
 #pragma unroll
-  for (int hlf = 0; hlf < 2; ++hlf) {
+  for (int hlf = 0; hlf < kD / 32; ++hlf) {
     uint32_t o[32];
     ptx::tmem_ld32(obase + 32u * hlf, o);
     ptx::tmem_wait_ld();
@@ -667,20 +749,23 @@ __device__ __forceinline__ unsigned long long entry_mask(const ItemStage& st, in
   return ((st.ent[e] >> (kEntBitsShift + half)) & 1u) ? st.kb[e] : 0ull;
 }
 
+template <int kD>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl, int warp, int lane,
                                              volatile int* abort_flag) {
+  using C = FwdCfg<kD>;
+  constexpr int R = C::kSoftRegion;
   const uint32_t bars = sl.bars, tmem = sl.tmem;
   auto bar = [&](int i) { return bar_at(bars, i); };
   const int r = (warp & 3) * 32 + lane;  // tile row == TMEM lane (warp w reaches lanes 32 (w % 4)..)
   const int half = r >> 6;               // warp-uniform: a warp's 32 rows lie in one half
   const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-  const uint32_t obase = tmem + lane_addr + kTmemO;
+  const uint32_t obase = tmem + lane_addr + C::kTmemO;
   const float sl2 = p.scale_log2;
   uint32_t g = 0;
   bool alive = true;
   // waits for PV(x): its commit freed V stage x % 2
   auto wait_pv = [&](uint32_t x) {
-    return wait_warp<1>(bar(kBarVFree + static_cast<int>(x % kVStages)), (x / kVStages) & 1u, abort_flag,
+    return wait_warp<R>(bar(kBarVFree + static_cast<int>(x % kVStages)), (x / kVStages) & 1u, abort_flag,
                            p.timeout_ns);
   };
 
@@ -689,7 +774,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
   bool q_pending = false;  // the tile of the last epilogue still holds its Q buffer
   uint32_t q_k = 0;
   for (uint32_t k = 0; alive; ++k) {
-    const int t = take_item_warp<1>(sl, k, abort_flag, p.timeout_ns);
+    const int t = take_item_warp<R>(sl, k, abort_flag, p.timeout_ns);
     if (t < 0) {
       if (t == kItemAbort) alive = false;
       break;
@@ -716,7 +801,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
         release_q(sl, q_k, lane);
       }
       const bool two = count - e0 >= 2;
-      if (!wait_warp<1>(bar(kBarSFull), g & 1u, abort_flag, p.timeout_ns)) {
+      if (!wait_warp<R>(bar(kBarSFull), g & 1u, abort_flag, p.timeout_ns)) {
         alive = false;
         break;
       }
@@ -730,12 +815,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       // exceeds it by more than kRescaleLog2, so every p = 2^(s - m) stays at or below
       // 2^kRescaleLog2 and O is rescaled only when m moves that far.  A warp's rows
       // share membership and key bits, so the branches are warp-uniform.
-      const uint32_t sbase = tmem + lane_addr + kTmemS;
+      const uint32_t sbase = tmem + lane_addr + C::kTmemS;
       const bool att0 = (att_bits >> e0) & 1ull, att1 = (att_bits >> (e0 + 1)) & 1ull;
       const bool part = ((part_bits >> e0) & 3ull) != 0ull;
       if (part) {  // an attended key block with some padded keys (rare): -inf in TMEM
-        if (att0) mask_scores(sbase, entry_mask(st, e0, half));
-        if (att1) mask_scores(sbase + 64u, entry_mask(st, e0 + 1, half));
+        if (att0) mask_scores<kD>(sbase, entry_mask(st, e0, half));
+        if (att1) mask_scores<kD>(sbase + 64u, entry_mask(st, e0 + 1, half));
       }
       // P is written over the scores it came from (a0 and a1 hold P after the
       // exponentials), so that the TMEM stores read the registers the loads wrote
@@ -774,13 +859,13 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       ptx::tc_fence_after();
       if (e0 == 0 && have_pend) {  // the previous tile's epilogue
         have_pend = false;
-        tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, obase, warp, lane);
+        tile_epilogue<kD>(p, pend, sl.items[pend.k % kItemRing], sl, obase, warp, lane);
         release_item_warp(sl, pend.k, lane);
         q_pending = true;
         q_k = pend.k;
       }
-      if (__any_sync(0xffffffffu, rescale)) rescale_o(obase, alpha);
-      const uint32_t pbase = tmem + lane_addr + kTmemP;
+      if (__any_sync(0xffffffffu, rescale)) rescale_o<kD>(obase, alpha);
+      const uint32_t pbase = tmem + lane_addr + C::kTmemP;
       if (att0) ptx::tmem_st32(pbase, a0); else tmem_zero32(pbase);
       if (two) {
         if (att1) ptx::tmem_st32(pbase + 32u, a1); else tmem_zero32(pbase + 32u);
@@ -802,41 +887,44 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
   if (alive && have_pend && wait_pv(g - 1)) {
     // the last tile: its last PV is done
     ptx::tc_fence_after();
-    tile_epilogue(p, pend, sl.items[pend.k % kItemRing], sl, obase, warp, lane);
+    tile_epilogue<kD>(p, pend, sl.items[pend.k % kItemRing], sl, obase, warp, lane);
     release_item_warp(sl, pend.k, lane);
   }
   if (lane == 0) ptx::bulk_wait_all();  // O stores complete before the CTA exits
 }
 
-__global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_constant__ FwdParams p) {
+template <int kD>
+__global__ void __launch_bounds__(FwdCfg<kD>::kThreads, 1) bsa_fwd_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<kD>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kSmemMisc);
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + C::kSmemMisc);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      const uint32_t bars = base + s * kSlotBytes + kSmemBar;
+    for (int s = 0; s < C::kSlots; ++s) {
+      const uint32_t bars = base + s * C::kSlotBytes + C::kSmemBar;
       for (int i = 0; i < kNumBars; ++i) {
         uint32_t count = 1;
         if (i >= kBarQEmpty && i < kBarQEmpty + 2) count = kWarpArrivals;
+        if (i >= kBarVFree && i < kBarVFree + kVStages) count = C::kPvIssuers;
         if (i == kBarSFree || i == kBarPFull) count = kThreadArrivals;
-        if (i >= kBarItemEmpty && i < kBarItemEmpty + kItemRing) count = kItemReaders;
+        if (i >= kBarItemEmpty && i < kBarItemEmpty + kItemRing) count = C::kItemReaders;
         ptx::mbar_init(bars + 8u * i, count);
       }
     }
     misc[1] = 0;
     ptx::fence_barrier_init();
   }
-  if (warp == kKProdWarp && lane == 0) {
+  if (warp == C::kKProdWarp && lane == 0) {
     ptx::prefetch_tensormap(&p.tm_q);
     ptx::prefetch_tensormap(&p.tm_k);
     ptx::prefetch_tensormap(&p.tm_v);
     ptx::prefetch_tensormap(&p.tm_o);
   }
-  if (warp == kSWarp) {
+  if (warp == C::kSWarp) {
     ptx::tmem_alloc(ptx::smem_addr(const_cast<uint32_t*>(&misc[0])), kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -845,29 +933,48 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   ptx::tc_fence_after();
   volatile int* abort_flag = reinterpret_cast<volatile int*>(&misc[1]);
 
-  const int slot = warp < 8 ? (warp >> 2) : (warp & 1);
-  Slot sl;
-  sl.sQ = base + slot * kSlotBytes + kSmemQ;
-  sl.sK = base + slot * kSlotBytes + kSmemK;
-  sl.sV = base + slot * kSlotBytes + kSmemV;
-  sl.bars = base + slot * kSlotBytes + kSmemBar;
-  sl.q_generic = smem + slot * kSlotBytes + kSmemQ;
-  sl.items = reinterpret_cast<ItemStage*>(smem + slot * kSlotBytes + kSmemItems);
-  sl.tmem = misc[0] + static_cast<uint32_t>(slot) * kSlotCols;
-
-  if (warp < 8) {
-    ptx::setmaxnreg_inc<kSoftmaxRegs>();
-    softmax_role(p, sl, warp, lane, abort_flag);
+  // the warp's slot: softmax warps 4 s..4 s + 3, then each role's kSlots warps in turn
+  int slot = 0, hf = 0;
+  if constexpr (C::kSlots == 2 && C::kPvIssuers == 1) {
+    static_assert(C::kKProdWarp == 8 && C::kVProdWarp == 14, "two-slot warp map");
+    slot = warp < 8 ? (warp >> 2) : (warp & 1);  // roles alternate slots from warp 8
+  } else if (warp < C::kKProdWarp) {
+    slot = warp >> 2;
+  } else if (warp < C::kPvWarp) {
+    slot = (warp - C::kKProdWarp) % C::kSlots;
+  } else if (warp < C::kVProdWarp) {
+    slot = (warp - C::kPvWarp) / C::kPvIssuers;
+    hf = (warp - C::kPvWarp) % C::kPvIssuers;
   } else {
-    ptx::setmaxnreg_dec<kOtherRegs>();
-    if (warp < kSWarp) {
-      k_producer(p, sl, lane, abort_flag);
-    } else if (warp < kPvWarp) {
-      if (lane == 0) s_issuer(p, sl, abort_flag);
-    } else if (warp < kVProdWarp) {
-      if (lane == 0) pv_issuer(p, sl, abort_flag);
-    } else {
-      v_producer(p, sl, lane, abort_flag);
+    slot = (warp - C::kVProdWarp) % C::kSlots;
+  }
+  Slot sl;
+  sl.sQ = base + slot * C::kSlotBytes + C::kSmemQ;
+  sl.sK = base + slot * C::kSlotBytes + C::kSmemK;
+  sl.sV = base + slot * C::kSlotBytes + C::kSmemV;
+  sl.bars = base + slot * C::kSlotBytes + C::kSmemBar;
+  sl.q_generic = smem + slot * C::kSlotBytes + C::kSmemQ;
+  sl.items = reinterpret_cast<ItemStage*>(smem + slot * C::kSlotBytes + C::kSmemItems);
+  sl.tmem = misc[0] + static_cast<uint32_t>(slot) * C::kSlotCols;
+
+  if (warp < C::kKProdWarp) {
+    ptx::setmaxnreg_inc<C::kSoftmaxRegs>();
+    softmax_role<kD>(p, sl, warp, lane, abort_flag);
+  } else {
+    ptx::setmaxnreg_dec<C::kOtherRegs>();
+    if (warp < C::kSWarp) {
+      k_producer<kD>(p, sl, lane, abort_flag);
+    } else if (warp < C::kPvWarp) {
+      if (lane == 0) s_issuer<kD>(p, sl, abort_flag);
+    } else if (warp < C::kVProdWarp) {
+      if (lane == 0) {
+        if constexpr (C::kPvIssuers == 1)
+          pv_issuer<kD>(p, sl, 0, abort_flag);
+        else
+          pv_issuer<kD>(p, sl, hf, abort_flag);
+      }
+    } else if (warp < C::kVProdWarp + C::kSlots) {
+      v_producer<kD>(p, sl, lane, abort_flag);
     }
     __syncwarp();
   }
@@ -875,7 +982,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == kSWarp) ptx::tmem_dealloc(misc[0], kTmemCols);
+  if (warp == C::kSWarp) ptx::tmem_dealloc(misc[0], kTmemCols);
 }
 
 // Merge of split tiles: one warp per (batch element, split tile, tile row).  The
@@ -885,7 +992,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(const __grid_const
 // largest m_c; lse = (M + log2 of that sum) ln 2.  The records are read in groups
 // of eight with every load of a group in flight at once, and folded into a running
 // (M, sum, O) -- the same rescaling the forward applies between chunks.  Lane x
-// owns output columns 2x, 2x + 1, so each record row is one coalesced 256-byte line.
+// owns output columns (d / 32) x .. (d / 32) x + d / 32 - 1, so each record row is
+// one coalesced line.
 struct MergeParams {
   const float* partials;
   const SplitTile* splits;
@@ -894,12 +1002,16 @@ struct MergeParams {
   int B, H, L, n_split, n_records;
 };
 
+template <int kD>
 __global__ void __launch_bounds__(128) bsa_merge_kernel(const __grid_constant__ MergeParams p) {
   // launched as the forward's programmatic dependent: its launch overlaps the
   // forward's end, and this wait returns once the forward has finished and its
   // records are visible
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int kGroup = 8;
+  constexpr int kCols = kD / 32;  // output columns per lane: kCols * lane ..
+  constexpr int kRec = FwdCfg<kD>::kRecFloats;
+  using Vec = typename std::conditional<kCols == 2, float2, float4>::type;
   const int lane = threadIdx.x & 31;
   const int task = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int per_b = p.n_split * kTileRows;
@@ -910,21 +1022,21 @@ __global__ void __launch_bounds__(128) bsa_merge_kernel(const __grid_constant__ 
   const int qblk = (r >> 6) ? st.qb : st.qa;
   if (qblk < 0) return;  // the unused half of a single-block tile
   const size_t row = static_cast<size_t>(b * p.H + st.h) * p.L + static_cast<size_t>(qblk) * 64 + (r & 63);
-  const float* base = p.partials + (static_cast<size_t>(b) * p.n_records + st.rec_base) * kRecFloats;
-  constexpr int kM = kTileRows * 64, kL = kTileRows * 64 + kTileRows;
+  const float* base = p.partials + (static_cast<size_t>(b) * p.n_records + st.rec_base) * kRec;
+  constexpr int kM = kTileRows * kD, kL = kTileRows * kD + kTileRows;
   const int nc = st.nchunks;
   float M = -INFINITY, lsum = 0.f;
-  float2 acc = make_float2(0.f, 0.f);
+  float acc[kCols] = {};
   for (int x0 = 0; x0 < nc; x0 += kGroup) {
     float mg[kGroup], lg[kGroup];
-    float2 og[kGroup];
+    Vec og[kGroup];
 #pragma unroll
     for (int j = 0; j < kGroup; ++j) {
       const int x = x0 + j < nc ? x0 + j : nc - 1;  // a repeated record gets weight 0 below
-      const float* rc = base + static_cast<size_t>(x) * kRecFloats;
+      const float* rc = base + static_cast<size_t>(x) * kRec;
       mg[j] = __ldcg(rc + kM + r);
       lg[j] = __ldcg(rc + kL + r);
-      og[j] = __ldcg(reinterpret_cast<const float2*>(rc + r * 64) + lane);
+      og[j] = __ldcg(reinterpret_cast<const Vec*>(rc + r * kD) + lane);
     }
     float gm = -INFINITY;
 #pragma unroll
@@ -934,20 +1046,28 @@ __global__ void __launch_bounds__(128) bsa_merge_kernel(const __grid_constant__ 
     const float Mn = fmaxf(M, gm);
     const float a = M == -INFINITY ? 0.f : ptx::ex2_approx(M - Mn);
     lsum *= a;
-    acc.x *= a;
-    acc.y *= a;
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) acc[c] *= a;
 #pragma unroll
     for (int j = 0; j < kGroup; ++j) {
       // a record whose row attended nothing has m = -inf and O = 0: weight 0
       const float f = (x0 + j < nc && mg[j] != -INFINITY) ? ptx::ex2_approx(mg[j] - Mn) : 0.f;
       lsum += f * lg[j];
-      acc.x += f * og[j].x;
-      acc.y += f * og[j].y;
+      const float* ov = reinterpret_cast<const float*>(&og[j]);
+#pragma unroll
+      for (int c = 0; c < kCols; ++c) acc[c] += f * ov[c];
     }
     M = Mn;
   }
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-  reinterpret_cast<uint32_t*>(p.out + row * 64)[lane] = pack_bf16x2(acc.x * inv, acc.y * inv);
+  uint32_t packed[kCols / 2];
+#pragma unroll
+  for (int c = 0; c < kCols / 2; ++c) packed[c] = pack_bf16x2(acc[2 * c] * inv, acc[2 * c + 1] * inv);
+  if constexpr (kCols == 2) {
+    reinterpret_cast<uint32_t*>(p.out + row * kD)[lane] = packed[0];
+  } else {
+    reinterpret_cast<uint2*>(p.out + row * kD)[lane] = make_uint2(packed[0], packed[1]);
+  }
   if (lane == 0) p.lse[row] = lsum > 0.f ? (M + log2f(lsum)) * kLn2 : -INFINITY;
 }
 
@@ -997,12 +1117,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 }  // namespace
 
-// [rows, 64] bf16 row-major tensor, boxes of 64 columns x box_rows rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+// [rows, d] bf16 row-major tensor (d a multiple of 64), boxes of 64 columns x box_rows
+// rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows, int d) {
   auto fn = get_encode_fn();
   if (fn == nullptr) return false;
-  cuuint64_t dims[2] = {64, rows};
-  cuuint64_t strides[1] = {128};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
   cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
@@ -1041,8 +1162,10 @@ int device_setup(int dev, DeviceInfo* out) {
     d.sm100 = (major == 10 && minor == 0);
     d.sms = sms;
     if (d.sm100 &&
-        cudaFuncSetAttribute(bsa_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemAlloc)) != cudaSuccess)
+        (cudaFuncSetAttribute(bsa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(FwdCfg<64>::kSmemAlloc)) != cudaSuccess ||
+         cudaFuncSetAttribute(bsa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(FwdCfg<128>::kSmemAlloc)) != cudaSuccess))
       return BSA_ERR_CUDA;
     d.configured = true;
   }
@@ -1068,13 +1191,13 @@ int validate_forward_args(const void* q, const void* k, const void* v, int B, in
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr || lay == nullptr ||
       B < 1 || H < 1 || L < 1)
     return BSA_ERR_INVALID_ARG;
-  if (d != kHeadDim) return BSA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
   if (H != lay->H || L != lay->L) return BSA_ERR_LAYOUT_MISMATCH;
   if (static_cast<int64_t>(B) * H * L > INT32_MAX - 64) return BSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
     return BSA_ERR_INVALID_ARG;
   if (!(scale == scale) || std::isinf(scale)) return BSA_ERR_INVALID_ARG;
-  c->plan = plan_workspace(*lay, B);
+  c->plan = plan_workspace(*lay, B, d);
   return BSA_OK;
 }
 
@@ -1094,8 +1217,8 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
   const WorkspacePlan& plan = c.plan;
   FwdParams prm{};
   const uint64_t rows = static_cast<uint64_t>(B) * H * L;
-  if (!make_map(&prm.tm_q, q, rows, 64) || !make_map(&prm.tm_k, k, rows, 64) ||
-      !make_map(&prm.tm_v, v, rows, 64) || !make_map(&prm.tm_o, out, rows, 32))
+  if (!make_map(&prm.tm_q, q, rows, 64, d) || !make_map(&prm.tm_k, k, rows, 64, d) ||
+      !make_map(&prm.tm_v, v, rows, 64, d) || !make_map(&prm.tm_o, out, rows, 32, d))
     return BSA_ERR_CUDA;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
@@ -1126,8 +1249,9 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
           cudaSuccess)
     return BSA_ERR_CUDA;
   const int64_t total = static_cast<int64_t>(B) * prm.items_per_batch;
-  // two slots per CTA; items are drawn dynamically
-  const int grid = static_cast<int>(std::min<int64_t>((total + kSlots - 1) / kSlots, c.info.sms));
+  // two slots per CTA at d = 64, one at d = 128; items are drawn dynamically
+  const int slots_per_cta = d == 64 ? FwdCfg<64>::kSlots : FwdCfg<128>::kSlots;
+  const int grid = static_cast<int>(std::min<int64_t>((total + slots_per_cta - 1) / slots_per_cta, c.info.sms));
   if (grid < 1) return BSA_OK;
   // How many batch elements early the split chunks go out: the last element's must
   // start while each slot still has at least one such chunk's length of work ahead.
@@ -1141,14 +1265,17 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
       work += ch;
       if (it.split >= 0) longest = std::max(longest, ch);
     }
-    const int64_t slots = static_cast<int64_t>(kSlots) * grid;
+    const int64_t slots = static_cast<int64_t>(slots_per_cta) * grid;
     while (prm.split_lead < B - 1 && (prm.split_lead + 1) * work < longest * slots) ++prm.split_lead;
     // One head's items are enough work to hand out its split chunks just before its
     // other tiles (the last head's chunks still start early enough): head by head.
     if (prm.split_lead == 0 && work >= static_cast<int64_t>(longest) * slots * H)
       prm.item_order = lay->d_head_order;
   }
-  bsa_fwd_kernel<<<grid, kThreads, kSmemAlloc, s>>>(prm);
+  if (d == 64)
+    bsa_fwd_kernel<64><<<grid, FwdCfg<64>::kThreads, FwdCfg<64>::kSmemAlloc, s>>>(prm);
+  else
+    bsa_fwd_kernel<128><<<grid, FwdCfg<128>::kThreads, FwdCfg<128>::kSmemAlloc, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   if (lay->n_split > 0) {
     MergeParams mp{};
@@ -1172,7 +1299,9 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, bsa_merge_kernel, mp) != cudaSuccess) return BSA_ERR_CUDA;
+    const cudaError_t e = d == 64 ? cudaLaunchKernelEx(&cfg, bsa_merge_kernel<64>, mp)
+                                  : cudaLaunchKernelEx(&cfg, bsa_merge_kernel<128>, mp);
+    if (e != cudaSuccess) return BSA_ERR_CUDA;
   }
   return BSA_OK;
 }

@@ -153,7 +153,7 @@ void build_row(int h, int i, int nb, int window, const std::vector<int32_t>& glo
 
 namespace bsa {
 
-WorkspacePlan plan_workspace(const bsa_layout& lay, int B) {
+WorkspacePlan plan_workspace(const bsa_layout& lay, int B, int d) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   WorkspacePlan p{};
   p.sched_off = 0;
@@ -162,7 +162,7 @@ WorkspacePlan plan_workspace(const bsa_layout& lay, int B) {
   p.keybits_bytes = up(sizeof(uint64_t) * static_cast<size_t>(B) * lay.nb);
   p.partials_off = p.keybits_off + p.keybits_bytes;
   p.partials_bytes =
-      up(sizeof(float) * static_cast<size_t>(kRecFloats) * static_cast<size_t>(B) * lay.n_records);
+      up(sizeof(float) * static_cast<size_t>(rec_floats(d)) * static_cast<size_t>(B) * lay.n_records);
   p.total = p.partials_off + p.partials_bytes;
   return p;
 }
@@ -592,8 +592,13 @@ void bsa_layout_free(bsa_layout* lay) {
 }
 
 int bsa_workspace_bytes(const bsa_layout* lay, int B, size_t* bytes) {
+  return bsa_forward_workspace_bytes(lay, B, bsa::kHeadDim, bytes);
+}
+
+int bsa_forward_workspace_bytes(const bsa_layout* lay, int B, int d, size_t* bytes) {
   if (lay == nullptr || bytes == nullptr || B < 1) return BSA_ERR_INVALID_ARG;
-  *bytes = bsa::plan_workspace(*lay, B).total;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  *bytes = bsa::plan_workspace(*lay, B, d).total;
   return BSA_OK;
 }
 

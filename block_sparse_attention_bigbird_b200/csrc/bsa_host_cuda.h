@@ -9,9 +9,10 @@
 
 namespace bsa {
 
-// TMA map of a [rows, 64] bf16 row-major tensor: boxes of 64 columns x box_rows
-// rows, 128-byte swizzle.  False if the driver entry point or the encode fails.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows);
+// TMA map of a [rows, d] bf16 row-major tensor (d a multiple of 64): boxes of 64
+// columns x box_rows rows, 128-byte swizzle.  False if the driver entry point or the
+// encode fails.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows, int d = 64);
 
 // Enqueues the kernel that packs a [B, L] uint8 key mask into one 64-bit word per
 // (b, key block): bit c set when key 64 j + c is kept.

@@ -24,9 +24,10 @@ constexpr int kTileRows = 128;
 constexpr int kSplitThreshold = BSA_SPLIT_THRESHOLD;
 constexpr int kSplitChunk = BSA_SPLIT_CHUNK;
 
-// Partial record of one split chunk: O[128][64] fp32 (unnormalised, relative to
+// Partial record of one split chunk: O[128][d] fp32 (unnormalised, relative to
 // the chunk's running max), then m[128] (log2 units, scaled) and l[128].
-constexpr int kRecFloats = kTileRows * kHeadDim + 2 * kTileRows;
+constexpr int rec_floats(int d) { return kTileRows * d + 2 * kTileRows; }
+constexpr int kRecFloats = rec_floats(kHeadDim);
 
 // One unit of the static schedule (32 bytes, read with two 16-byte loads).
 struct WorkItem {
@@ -134,7 +135,7 @@ struct WorkspacePlan {
   size_t partials_off, partials_bytes;
   size_t total;
 };
-WorkspacePlan plan_workspace(const bsa_layout& lay, int B);
+WorkspacePlan plan_workspace(const bsa_layout& lay, int B, int d = kHeadDim);
 // Backward workspace for batch size B: key-padding bits, D = rowsum(dO * O) and
 // lse in log2 units per row, and the partial records of split tiles (dQ: 128 x 64
 // floats each; dK and dV: 2 x 128 x 64 floats each).

@@ -46,8 +46,8 @@ extern "C" {
 typedef enum {
   BSA_OK = 0,
   BSA_ERR_INVALID_ARG = -1,     /* null pointer, bad size or range            */
-  BSA_ERR_UNSUPPORTED = -2,     /* block not a multiple of 64, d != 64, not an
-                                   sm_100 device                               */
+  BSA_ERR_UNSUPPORTED = -2,     /* block not a multiple of 64, a head dim the
+                                   call does not take, not an sm_100 device    */
   BSA_ERR_CUDA = -3,            /* a CUDA runtime/driver call failed           */
   BSA_ERR_LAYOUT_MISMATCH = -4, /* layout built for another H/L, or not uploaded
                                    to the current device                       */
@@ -208,9 +208,18 @@ void bsa_layout_free(bsa_layout* layout);
 int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
 
 /*
+ * bsa_forward_workspace_bytes -- the same for head dim d (64 or 128; the partial
+ * results of split rows hold d columns per row): bsa_workspace_bytes is this with
+ * d = 64.  BSA_ERR_UNSUPPORTED for another d.
+ */
+int bsa_forward_workspace_bytes(const bsa_layout* layout, int B, int d, size_t* bytes);
+
+/*
  * bsa_forward -- enqueues the block-sparse attention forward on `stream`.
  *   q, k, v   device, bf16, [B, H, L, d] contiguous, 16-byte aligned.
- *   d         must be 64 (else BSA_ERR_UNSUPPORTED).
+ *   d         64 or 128 (else BSA_ERR_UNSUPPORTED).  At d = 128 the kernel runs
+ *             one pipeline per SM instead of two (its operands take twice the
+ *             shared memory and TMEM).
  *   layout    built for this H and L and uploaded to the current device.
  *   key_mask  device uint8 [B, L] (1 = keep, 0 = drop the key), or NULL.
  *   scale     softmax scale applied to q.k; <= 0 selects 1/sqrt(d).
@@ -218,8 +227,9 @@ int bsa_workspace_bytes(const bsa_layout* layout, int B, size_t* bytes);
  *   lse       device, fp32, [B, H, L]: natural-log sum of exp of the scaled
  *             scores over the attended keys; -inf (with O = 0) for a row whose
  *             attended set is empty.
- *   workspace device, at least bsa_workspace_bytes(layout, B) bytes, 256-byte
- *             aligned, any contents (see above).
+ *   workspace device, at least bsa_forward_workspace_bytes(layout, B, d) bytes
+ *             (bsa_workspace_bytes at d = 64), 256-byte aligned, any contents
+ *             (see above).
  * Enqueues on `stream` a 256-byte memset of the schedule counters and up to
  * three kernels: the key-padding bits (with a key mask), the forward, and the
  * merge of split rows (when the layout has any; it is launched as a

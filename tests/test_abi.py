@@ -72,7 +72,8 @@ def test_forward_argument_errors_before_any_launch():
     assert _fwd(lay, lse=None) == bsa.BSA_ERR_INVALID_ARG
     assert _fwd(lay, use_layout=False) == bsa.BSA_ERR_INVALID_ARG
     assert _fwd(lay, B=0) == bsa.BSA_ERR_INVALID_ARG
-    assert _fwd(lay, d=128) == bsa.BSA_ERR_UNSUPPORTED
+    assert _fwd(lay, d=96) == bsa.BSA_ERR_UNSUPPORTED  # the forward takes d = 64 or 128
+    assert _fwd(lay, d=32) == bsa.BSA_ERR_UNSUPPORTED
     assert _fwd(lay, H=3) == bsa.BSA_ERR_LAYOUT_MISMATCH
     assert _fwd(lay, L=1024) == bsa.BSA_ERR_LAYOUT_MISMATCH
     assert _fwd(lay, q=(1 << 12) + 2) == bsa.BSA_ERR_INVALID_ARG          # misaligned

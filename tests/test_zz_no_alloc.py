@@ -26,7 +26,7 @@ def test_static_entry_rejects_bad_arguments_without_a_gpu():
     fwd = bsa.lib.bsa_forward_static_ws
     a = 1 << 12
     assert fwd(None, a, a, 1, 2, 512, 64, lay.handle, None, ctypes.c_float(0), a, a, None) == bsa.BSA_ERR_INVALID_ARG
-    assert fwd(a, a, a, 1, 2, 512, 128, lay.handle, None, ctypes.c_float(0), a, a, None) == bsa.BSA_ERR_UNSUPPORTED
+    assert fwd(a, a, a, 1, 2, 512, 96, lay.handle, None, ctypes.c_float(0), a, a, None) == bsa.BSA_ERR_UNSUPPORTED
     assert fwd(a, a, a, 1, 3, 512, 64, lay.handle, None, ctypes.c_float(0), a, a, None) == bsa.BSA_ERR_LAYOUT_MISMATCH
 
 
