@@ -8,9 +8,10 @@
 // per-tile list of 64-key blocks ("SQA 稀疏注意力机制详解" 3.1: block-sparse mask,
 // attention only on non-zero blocks).
 //
-// Kernel design: one persistent CTA per SM (512 threads, four warpgroups) running two
-// independent pipelines ("slots"), each with its own work items, shared-memory rings,
-// barriers and 256 TMEM columns: O (64), S (128) and P (64, bf16 pairs).  A tile is two
+// Kernel design (head dim 64; FwdCfg below has what changes at 128): one persistent
+// CTA per SM (512 threads, four warpgroups) running two independent pipelines
+// ("slots"), each with its own work items, shared-memory rings, barriers and 256 TMEM
+// columns: O (64), S (128) and P (64, bf16 pairs).  A tile is two
 // 64-row query blocks of the same (b, h) over the union of their key-block lists; a
 // chunk is two consecutive union entries (128 keys).
 //   warps 0-3 / 4-7  softmax of slot 0 / 1 (thread r of the slot owns tile row r =
