@@ -39,8 +39,12 @@ def _as_f64(x) -> np.ndarray:
 
 
 def token_mask_row(layout: dict, h: int, i: int, L: int) -> np.ndarray:
-    """Boolean [L] mask of the keys attended by query block i of head h."""
+    """Boolean mask of the keys attended by query block i of head h: [L] for a
+    block layout (every token of the block alike), [block, L] for a token-level
+    one (one row per query token, oracle.layout.token_allowed)."""
     block = layout["block"]
+    if "token" in layout:
+        return np.stack([_layout.token_allowed(layout, h, t, L) for t in range(i * block, (i + 1) * block)])
     m = np.zeros(L, dtype=bool)
     for j in _layout.row(layout, h, i):
         m[j * block:(j + 1) * block] = True
@@ -105,7 +109,10 @@ def attention_rows(q, k, v, layout: dict, b: int, h: int, tokens, key_mask=None,
     o = np.zeros((len(tokens), d))
     lse = np.zeros(len(tokens))
     for n, t in enumerate(tokens):
-        allowed = token_mask_row(layout, h, int(t) // block, L)
+        if "token" in layout:
+            allowed = _layout.token_allowed(layout, h, int(t), L)
+        else:
+            allowed = token_mask_row(layout, h, int(t) // block, L)
         if km is not None:
             allowed = allowed & km
         s = (qb[t] @ kb.T) * scale
@@ -126,9 +133,11 @@ def attention_bruteforce(q, k, v, layout: dict, key_mask=None, scale=None):
     for b in range(B):
         for h in range(H):
             for t in range(L):
-                blocks = [int(j) for j in _layout.row(layout, h, t // block)]
-                keys = [p for j in blocks for p in range(j * block, (j + 1) * block)
-                        if key_mask is None or int(key_mask[b][p]) != 0]
+                if "token" in layout:
+                    cand = [int(p) for p in np.nonzero(_layout.token_allowed(layout, h, t, L))[0]]
+                else:
+                    cand = [p for j in _layout.row(layout, h, t // block) for p in range(j * block, (j + 1) * block)]
+                keys = [p for p in cand if key_mask is None or int(key_mask[b][p]) != 0]
                 if not keys:
                     lse[b, h, t] = -math.inf
                     continue

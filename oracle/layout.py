@@ -119,3 +119,86 @@ def block_mask(layout: dict) -> np.ndarray:
         for i in range(nb):
             m[h, i, row(layout, h, i)] = True
     return m
+
+
+# ----------------------------------------------------------------------------- token level
+# Readings for the token-level layout (window and global set in tokens, not whole
+# blocks; [BigBird] 核心实现 gives its window in tokens, w = 64 in its example):
+#   * G: global tokens; explicit, or the linspace rule over tokens:
+#     n_g == 1 -> {0}, n_g >= 2 -> floor(k (L-1) / (n_g-1)).
+#   * allowed(h, i, j) = i in G  or  j in G  or  |i - j| <= w  or
+#     (block(i) holds no global token and block(j) is a random block of block(i)).
+#   * random blocks stay at block granularity (the pages draw blocks): for a query
+#     block I without a global token, n_random blocks drawn as at block level from
+#     the blocks outside the band's blocks {J : |I - J| <= floor((w + 63) / 64)} and
+#     outside the blocks holding a global token, with the same Philox stream.
+#   * blocks are 64 tokens (the kernels' key blocks); L is a multiple of 64.
+
+
+def global_tokens(L: int, n_global: int, explicit=None) -> list[int]:
+    """Sorted distinct global token indices (the linspace rule, over tokens)."""
+    if explicit is not None:
+        g = sorted({int(x) for x in explicit})
+        if g and (g[0] < 0 or g[-1] >= L):
+            raise ValueError("explicit global token out of range")
+        return g
+    if n_global <= 0:
+        return []
+    if n_global == 1:
+        return [0]
+    return sorted({(k * (L - 1)) // (n_global - 1) for k in range(n_global)})
+
+
+def token_random_blocks(h: int, I: int, nb: int, window: int, gblocks: set, n_random: int, seed: int) -> list[int]:
+    """Random key blocks of query block I (none when I holds a global token)."""
+    if I in gblocks:
+        return []
+    wb = (window + 63) // 64
+    band = set(window_blocks(I, nb, wb))
+    cand = [j for j in range(nb) if j not in band and j not in gblocks]
+    take = min(n_random, len(cand))
+    return random_blocks(cand, n_random, philox_stream(seed, I, h, take))
+
+
+def build_token_layout(H: int, L: int, window: int, n_global: int, n_random: int, seed: int,
+                       explicit_globals=None) -> dict:
+    """Token-level layout: the allowed-pair rule above, plus its block CSR (the key
+    blocks holding at least one allowed key of some query token of the block)."""
+    if L % 64:
+        raise ValueError("L must be a multiple of 64")
+    nb = L // 64
+    g = global_tokens(L, n_global, explicit_globals)
+    gblocks = {t // 64 for t in g}
+    rand = [[token_random_blocks(h, I, nb, window, gblocks, n_random, seed) for I in range(nb)] for h in range(H)]
+    gt = np.zeros(L, dtype=bool)
+    gt[g] = True
+    row_ptr = [0]
+    cols: list[int] = []
+    for h in range(H):
+        for I in range(nb):
+            keys = np.zeros(nb, dtype=bool)
+            for i in range(64 * I, 64 * I + 64):
+                keys |= token_allowed(None, h, i, L, _parts=(window, gt, rand)).reshape(nb, 64).any(axis=1)
+            cols.extend(int(j) for j in np.nonzero(keys)[0])
+            row_ptr.append(len(cols))
+    return {"H": H, "L": L, "block": 64, "nb": nb, "globals": sorted(gblocks),
+            "row_ptr": np.asarray(row_ptr, dtype=np.int64), "col_idx": np.asarray(cols, dtype=np.int32),
+            "token": {"window": window, "globals": g, "random": rand}}
+
+
+def token_allowed(layout: dict, h: int, i: int, L: int, _parts=None) -> np.ndarray:
+    """Boolean [L]: the keys query token i of head h attends (the rule above)."""
+    if _parts is None:
+        tk = layout["token"]
+        gt = np.zeros(L, dtype=bool)
+        gt[tk["globals"]] = True
+        window, rand = tk["window"], tk["random"]
+    else:
+        window, gt, rand = _parts
+    if gt[i]:
+        return np.ones(L, dtype=bool)
+    j = np.arange(L)
+    m = gt | (np.abs(j - i) <= window)
+    for J in rand[h][i // 64]:
+        m[64 * J:64 * J + 64] = True
+    return m
