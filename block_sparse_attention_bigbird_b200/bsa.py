@@ -33,6 +33,11 @@ _SIGNATURES = {
                                         ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
                                         ctypes.POINTER(ctypes.c_int32),
                                         ctypes.POINTER(ctypes.c_void_p)]),
+    "bsa_layout_build_tokens": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, ctypes.c_uint64, ctypes.POINTER(ctypes.c_int32),
+                                               ctypes.POINTER(ctypes.c_void_p)]),
+    "bsa_layout_token_masks": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_int),
+                                              ctypes.POINTER(ctypes.c_void_p)]),
     "bsa_layout_from_csr": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                            ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
                                            ctypes.POINTER(ctypes.c_void_p)]),
@@ -152,6 +157,29 @@ def bsa_layout_build(H: int, L: int, block: int = 64, window: int = 1, n_global:
                                 ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), gptr, ctypes.byref(out)),
            "bsa_layout_build")
     return Layout(out.value, H, L)
+
+
+def bsa_layout_build_tokens(H: int, L: int, window: int, n_global: int = 0, n_random: int = 0, seed: int = 0,
+                            global_tokens=None) -> Layout:
+    """A BigBird layout with its window and global set in tokens (see bsa.h)."""
+    out = ctypes.c_void_p()
+    gptr = None
+    if global_tokens is not None:
+        g = np.ascontiguousarray(np.asarray(global_tokens, dtype=np.int32))
+        n_global = int(g.size)
+        gptr = g.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+    _check(lib.bsa_layout_build_tokens(H, L, window, n_global, n_random,
+                                       ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF), gptr, ctypes.byref(out)),
+           "bsa_layout_build_tokens")
+    return Layout(out.value, H, L)
+
+
+def bsa_layout_token_masks(layout: Layout):
+    """(window in tokens, uint64 [L / 64] global-token bits) of a token-level layout."""
+    w, gb = ctypes.c_int(), ctypes.c_void_p()
+    _check(lib.bsa_layout_token_masks(layout.handle, ctypes.byref(w), ctypes.byref(gb)), "bsa_layout_token_masks")
+    bits = np.ctypeslib.as_array(ctypes.cast(gb, ctypes.POINTER(ctypes.c_uint64)), (layout.L // 64,)).copy()
+    return w.value, bits
 
 
 def bsa_layout_from_csr(H: int, L: int, row_ptr, col_idx, block: int = 64) -> Layout:

@@ -626,6 +626,7 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
       dq == nullptr || dk == nullptr || dv == nullptr || lay == nullptr || B < 1 || H < 1 || L < 1)
     return BSA_ERR_INVALID_ARG;
   if (d != kHeadDim) return BSA_ERR_UNSUPPORTED;
+  if (lay->token) return BSA_ERR_UNSUPPORTED;  // per-row masks: the forward only
   if (H != lay->H || L != lay->L) return BSA_ERR_LAYOUT_MISMATCH;
   if (static_cast<int64_t>(B) * H * L > INT32_MAX - 64) return BSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||

@@ -187,6 +187,10 @@ struct FwdParams {
   int split_items;  // the first split_items items of a batch element are split-tile chunks
   int split_lead;   // split chunks are handed out this many batch elements early
   const int32_t* item_order;  // null, or the items of one batch element head by head
+  // token-level layouts (else null): bit c of word j set when token 64 j + c is global;
+  // the window in tokens.  Entries flagged at kEntMaskShift + half get per-row masks.
+  const unsigned long long* tok_gbits;
+  long long tok_window;
   float scale_log2;
   unsigned long long timeout_ns;
 };
@@ -750,7 +754,36 @@ __device__ __forceinline__ unsigned long long entry_mask(const ItemStage& st, in
   return ((st.ent[e] >> (kEntBitsShift + half)) & 1u) ? st.kb[e] : 0ull;
 }
 
+// Token-level layouts: the keys of key block jb that query token i attends by the
+// token rule (i global: all; else the band |i - j| <= w and the global keys).  The
+// random blocks never get here (their entries need no mask).
+__device__ __forceinline__ unsigned long long token_row_mask(const FwdParams& p, long long i, bool row_global,
+                                                             int jb) {
+  if (row_global) return ~0ull;
+  const long long lo = i - p.tok_window - 64ll * jb, hi = i + p.tok_window - 64ll * jb;
+  unsigned long long band = 0ull;
+  if (hi >= 0 && lo <= 63) {
+    const int l = lo < 0 ? 0 : static_cast<int>(lo), h = hi > 63 ? 63 : static_cast<int>(hi);
+    band = (h == 63 ? ~0ull : ((1ull << (h + 1)) - 1ull)) & ~((1ull << l) - 1ull);
+  }
+  return band | p.tok_gbits[jb];
+}
+
+// The -inf mask of one attended 64-key group of this warp's rows (rare path, out of
+// line): the key-padding bits, and at a token-level layout the row's token mask when
+// the entry is flagged for this half.
 template <int kD>
+__device__ __noinline__ void mask_entry(const FwdParams& p, const ItemStage& st, uint32_t taddr, int e, int half,
+                                       long long itok, bool row_global) {
+  unsigned long long mk = entry_mask(st, e, half);
+  if (p.tok_gbits != nullptr && ((st.ent[e] >> (kEntMaskShift + half)) & 1u))
+    mk &= token_row_mask(p, itok, row_global, static_cast<int>(st.ent[e] & kEntColMask));
+  mask_scores<kD>(taddr, mk);
+}
+
+// kTok: the layout is token-level (per-row masks in flagged entries; rows may then see
+// chunks with no allowed key).
+template <int kD, bool kTok>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl, int warp, int lane,
                                              volatile int* abort_flag) {
   using C = FwdCfg<kD>;
@@ -796,6 +829,21 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       part_bits = static_cast<uint64_t>(__ballot_sync(0xffffffffu, k0 + 1ull > 1ull)) |
                   (static_cast<uint64_t>(__ballot_sync(0xffffffffu, k1 + 1ull > 1ull)) << 32);
     }
+    // token-level layouts: entries whose pairs this half's rows mask row by row
+    long long itok = 0;
+    bool row_global = false;
+    if constexpr (kTok) {
+      const uint32_t sh = kEntMaskShift + half;
+      const bool t0 = lane < count && ((st.ent[lane] >> sh) & 1u);
+      const bool t1 = lane + 32 < count && ((st.ent[lane + 32] >> sh) & 1u);
+      part_bits |= static_cast<uint64_t>(__ballot_sync(0xffffffffu, t0)) |
+                   (static_cast<uint64_t>(__ballot_sync(0xffffffffu, t1)) << 32);
+      const int qblk = half ? st.qb : st.qa;
+      if (qblk >= 0) {
+        itok = 64ll * qblk + (r & 63);
+        row_global = (p.tok_gbits[qblk] >> (r & 63)) & 1ull;
+      }
+    }
     for (int e0 = 0; e0 < count; e0 += kChunkEnt, ++g) {
       if (q_pending && e0 > 0) {  // one chunk after the epilogue: its O store has had time
         q_pending = false;
@@ -819,9 +867,14 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       const uint32_t sbase = tmem + lane_addr + C::kTmemS;
       const bool att0 = (att_bits >> e0) & 1ull, att1 = (att_bits >> (e0 + 1)) & 1ull;
       const bool part = ((part_bits >> e0) & 3ull) != 0ull;
-      if (part) {  // an attended key block with some padded keys (rare): -inf in TMEM
-        if (att0) mask_scores<kD>(sbase, entry_mask(st, e0, half));
-        if (att1) mask_scores<kD>(sbase + 64u, entry_mask(st, e0 + 1, half));
+      if (part) {  // some keys of an attended block are padded or masked (rare): -inf in TMEM
+        if constexpr (kTok) {
+          if (att0) mask_entry<kD>(p, st, sbase, e0, half, itok, row_global);
+          if (att1) mask_entry<kD>(p, st, sbase + 64u, e0 + 1, half, itok, row_global);
+        } else {
+          if (att0) mask_scores<kD>(sbase, entry_mask(st, e0, half));
+          if (att1) mask_scores<kD>(sbase + 64u, entry_mask(st, e0 + 1, half));
+        }
       }
       // P is written over the scores it came from (a0 and a1 hold P after the
       // exponentials), so that the TMEM stores read the registers the loads wrote
@@ -844,7 +897,10 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
       if (att1) cm = fmaxf(cm, group_max(a1, b1));
       const float cm2 = cm * sl2;  // scale > 0: the max of the scaled scores
       const float m_new = cm2 > m_run + kRescaleLog2 ? cm2 : m_run;
-      const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_new, -m_new);
+      // token level: a row with no allowed key so far (every score -inf) takes
+      // p = 2^-inf = 0 (at block level an attended block keeps a key)
+      const float m_off = (kTok && m_new == -INFINITY) ? 0.f : m_new;
+      const uint64_t sc2 = ptx::pack2(sl2, sl2), nm2 = ptx::pack2(-m_off, -m_off);
       float psum = 0.f;
       if (att0) psum += group_exp(a0, b0, sc2, nm2);
       if (att1) psum += group_exp(a1, b1, sc2, nm2);
@@ -894,7 +950,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const Slot& sl,
   if (lane == 0) ptx::bulk_wait_all();  // O stores complete before the CTA exits
 }
 
-template <int kD>
+template <int kD, bool kTok>
 __global__ void __launch_bounds__(FwdCfg<kD>::kThreads, 1) bsa_fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<kD>;
   extern __shared__ uint8_t smem_raw[];
@@ -960,7 +1016,7 @@ __global__ void __launch_bounds__(FwdCfg<kD>::kThreads, 1) bsa_fwd_kernel(const 
 
   if (warp < C::kKProdWarp) {
     ptx::setmaxnreg_inc<C::kSoftmaxRegs>();
-    softmax_role<kD>(p, sl, warp, lane, abort_flag);
+    softmax_role<kD, kTok>(p, sl, warp, lane, abort_flag);
   } else {
     ptx::setmaxnreg_dec<C::kOtherRegs>();
     if (warp < C::kSWarp) {
@@ -1163,9 +1219,13 @@ int device_setup(int dev, DeviceInfo* out) {
     d.sm100 = (major == 10 && minor == 0);
     d.sms = sms;
     if (d.sm100 &&
-        (cudaFuncSetAttribute(bsa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        (cudaFuncSetAttribute(bsa_fwd_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(FwdCfg<64>::kSmemAlloc)) != cudaSuccess ||
-         cudaFuncSetAttribute(bsa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+         cudaFuncSetAttribute(bsa_fwd_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(FwdCfg<64>::kSmemAlloc)) != cudaSuccess ||
+         cudaFuncSetAttribute(bsa_fwd_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(FwdCfg<128>::kSmemAlloc)) != cudaSuccess ||
+         cudaFuncSetAttribute(bsa_fwd_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(FwdCfg<128>::kSmemAlloc)) != cudaSuccess))
       return BSA_ERR_CUDA;
     d.configured = true;
@@ -1238,6 +1298,8 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
                                                    [](const WorkItem& it) { return it.split >= 0; }));
   prm.n_split = lay->n_split;
   prm.n_records = lay->n_records;
+  prm.tok_gbits = lay->token ? lay->d_tok_gbits : nullptr;
+  prm.tok_window = lay->tok_window;
   const float sc = scale > 0.f ? scale : 1.f / std::sqrt(static_cast<float>(d));
   prm.scale_log2 = sc * kLog2e;
   prm.timeout_ns = kDefaultTimeoutNs;
@@ -1273,10 +1335,15 @@ int enqueue_forward(const ForwardCall& c, const void* q, const void* k, const vo
     if (prm.split_lead == 0 && work >= static_cast<int64_t>(longest) * slots * H)
       prm.item_order = lay->d_head_order;
   }
-  if (d == 64)
-    bsa_fwd_kernel<64><<<grid, FwdCfg<64>::kThreads, FwdCfg<64>::kSmemAlloc, s>>>(prm);
+  const bool tok = prm.tok_gbits != nullptr;
+  if (d == 64 && !tok)
+    bsa_fwd_kernel<64, false><<<grid, FwdCfg<64>::kThreads, FwdCfg<64>::kSmemAlloc, s>>>(prm);
+  else if (d == 64)
+    bsa_fwd_kernel<64, true><<<grid, FwdCfg<64>::kThreads, FwdCfg<64>::kSmemAlloc, s>>>(prm);
+  else if (!tok)
+    bsa_fwd_kernel<128, false><<<grid, FwdCfg<128>::kThreads, FwdCfg<128>::kSmemAlloc, s>>>(prm);
   else
-    bsa_fwd_kernel<128><<<grid, FwdCfg<128>::kThreads, FwdCfg<128>::kSmemAlloc, s>>>(prm);
+    bsa_fwd_kernel<128, true><<<grid, FwdCfg<128>::kThreads, FwdCfg<128>::kSmemAlloc, s>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   if (lay->n_split > 0) {
     MergeParams mp{};
@@ -1325,6 +1392,7 @@ void free_device(bsa_layout* lay) {
     cudaFree(lay->d_dkv_items);
     cudaFree(lay->d_dq_splits);
     cudaFree(lay->d_dkv_splits);
+    cudaFree(lay->d_tok_gbits);
   }
   if (have_cur) cudaSetDevice(cur);
   lay->d_pair_q = nullptr;
@@ -1338,6 +1406,7 @@ void free_device(bsa_layout* lay) {
   lay->d_dkv_items = nullptr;
   lay->d_dq_splits = nullptr;
   lay->d_dkv_splits = nullptr;
+  lay->d_tok_gbits = nullptr;
   lay->device = -1;
 }
 
@@ -1378,6 +1447,8 @@ int bsa_layout_upload(bsa_layout* lay, void* stream) {
        lay->dq_plan.splits.size() * sizeof(SplitTile)},
       {reinterpret_cast<void**>(&lay->d_dkv_splits), lay->dkv_plan.splits.data(),
        lay->dkv_plan.splits.size() * sizeof(SplitTile)},
+      {reinterpret_cast<void**>(&lay->d_tok_gbits), lay->tok_gbits.data(),
+       lay->tok_gbits.size() * sizeof(uint64_t)},
   };
   lay->device = dev;
   for (const Table& t : tables) {

@@ -5,6 +5,7 @@
 // validates its arguments and returns a bsa_status; no exception crosses the C
 // ABI.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 
@@ -191,10 +192,13 @@ namespace {
 // rows, then the blocks in one row only, alternating first/second, each group
 // ascending.  The order is free (one softmax over the union), and this one keeps
 // the two halves of the tile -- whose warps skip the work of a block their half
-// does not take part in -- doing equal work chunk by chunk.
+// does not take part in -- doing equal work chunk by chunk.  `masked` (optional, one
+// flag per CSR entry) marks block pairs that need a per-row mask; an entry carries the
+// flag of each row it comes from at bit kEntMaskShift + half.
 void make_tiles(int H, int nb, const std::vector<int32_t>& row_ptr, const std::vector<int32_t>& col_idx,
                 const std::vector<uint8_t>& dense, std::vector<int32_t>* pair_q, int* n_pairs,
-                std::vector<int32_t>* pair_ptr, std::vector<uint32_t>* pair_ent) {
+                std::vector<int32_t>* pair_ptr, std::vector<uint32_t>* pair_ent,
+                const std::vector<uint8_t>* masked = nullptr) {
   std::vector<int32_t> gl, ng;
   for (int i = 0; i < nb; ++i) (dense[static_cast<size_t>(i)] ? gl : ng).push_back(i);
   pair_q->clear();
@@ -223,13 +227,22 @@ void make_tiles(int H, int nb, const std::vector<int32_t>& row_ptr, const std::v
       both.clear();
       only_a.clear();
       only_b.clear();
+      // the masked bits of the entry at CSR position x, for half hf
+      auto mbit = [&](const int32_t* x, int hf) -> uint32_t {
+        return (masked != nullptr && (*masked)[static_cast<size_t>(x - col_idx.data())])
+                   ? (1u << (bsa::kEntMaskShift + hf))
+                   : 0u;
+      };
       while (ra != ra_end || rb != rb_end) {
         if (rb == rb_end || (ra != ra_end && *ra < *rb)) {
-          only_a.push_back(static_cast<uint32_t>(*ra++) | (1u << bsa::kEntBitsShift));
+          only_a.push_back(static_cast<uint32_t>(*ra) | (1u << bsa::kEntBitsShift) | mbit(ra, 0));
+          ++ra;
         } else if (ra == ra_end || *rb < *ra) {
-          only_b.push_back(static_cast<uint32_t>(*rb++) | (2u << bsa::kEntBitsShift));
+          only_b.push_back(static_cast<uint32_t>(*rb) | (2u << bsa::kEntBitsShift) | mbit(rb, 1));
+          ++rb;
         } else {
-          both.push_back(static_cast<uint32_t>(*ra++) | (3u << bsa::kEntBitsShift));
+          both.push_back(static_cast<uint32_t>(*ra) | (3u << bsa::kEntBitsShift) | mbit(ra, 0) | mbit(rb, 1));
+          ++ra;
           ++rb;
         }
       }
@@ -284,7 +297,7 @@ void make_bwd_plan(int H, const std::vector<int32_t>& pair_q, int P, const std::
 void build_tiles(bsa_layout* lay, const std::vector<uint8_t>& dense) {
   const int nb = lay->nb, H = lay->H;
   make_tiles(H, nb, lay->row_ptr, lay->col_idx, dense, &lay->pair_q, &lay->n_pairs, &lay->pair_ptr,
-             &lay->pair_ent);
+             &lay->pair_ent, lay->token ? &lay->tok_masked : nullptr);
   const int P = lay->n_pairs;
   // Work items of one batch element: first the chunks of split tiles (the longest
   // items, kept away from the end of the element's run), then the other tiles,
@@ -470,6 +483,105 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
     return BSA_ERR_INVALID_ARG;
   }
   *out = lay;
+  return BSA_OK;
+}
+
+int bsa_layout_build_tokens(int H, int L, int window, int n_global, int n_random, uint64_t seed,
+                            const int32_t* global_tokens, bsa_layout** out) {
+  if (out == nullptr) return BSA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (H < 1 || L < bsa::kBlock || L % bsa::kBlock != 0 || window < 0 || n_global < 0 || n_random < 0)
+    return BSA_ERR_INVALID_ARG;
+  const int nb = L / bsa::kBlock;
+  if (nb > static_cast<int>(bsa::kEntColMask) || static_cast<int64_t>(H) * nb > (1 << 30)) return BSA_ERR_INVALID_ARG;
+  bsa_layout* lay = new (std::nothrow) bsa_layout();
+  if (lay == nullptr) return BSA_ERR_OOM;
+  try {
+    lay->H = H;
+    lay->L = L;
+    lay->block = bsa::kBlock;
+    lay->nb = nb;
+    lay->n_random = n_random;
+    lay->seed = seed;
+    // global tokens: the caller's, or the linspace rule over tokens
+    std::vector<int64_t> g;
+    if (global_tokens != nullptr) {
+      for (int x = 0; x < n_global; ++x) {
+        if (global_tokens[x] < 0 || global_tokens[x] >= L) {
+          delete lay;
+          return BSA_ERR_INVALID_ARG;
+        }
+        g.push_back(global_tokens[x]);
+      }
+    } else if (n_global == 1) {
+      g.push_back(0);
+    } else if (n_global >= 2) {
+      for (int k = 0; k < n_global; ++k) g.push_back((static_cast<int64_t>(k) * (L - 1)) / (n_global - 1));
+    }
+    lay->tok_gbits.assign(static_cast<size_t>(nb), 0ull);
+    for (int64_t t : g) lay->tok_gbits[static_cast<size_t>(t / 64)] |= 1ull << (t % 64);
+    // the blocks holding a global token play the part of global blocks at block level
+    std::vector<int32_t> gblocks;
+    std::vector<uint8_t> is_gb(static_cast<size_t>(nb), 0);
+    for (int j = 0; j < nb; ++j)
+      if (lay->tok_gbits[static_cast<size_t>(j)] != 0) {
+        gblocks.push_back(j);
+        is_gb[static_cast<size_t>(j)] = 1;
+      }
+    lay->globals = gblocks;
+    lay->n_global = static_cast<int>(gblocks.size());
+    // the band's blocks: |I - J| <= floor((w + 63) / 64)
+    const int64_t wb64 = (static_cast<int64_t>(window) + 63) / 64;
+    const int wb = static_cast<int>(std::min<int64_t>(wb64, nb));
+    lay->window = wb;
+    lay->token = true;
+    lay->tok_window = window;
+    std::vector<int32_t> urp, uci, row;
+    urp.reserve(static_cast<size_t>(H) * nb + 1);
+    urp.push_back(0);
+    lay->tok_masked.clear();
+    for (int h = 0; h < H; ++h) {
+      for (int I = 0; I < nb; ++I) {
+        build_row(h, I, nb, wb, gblocks, is_gb, n_random, seed, &row);
+        for (int32_t J : row) {
+          // every pair of the two blocks is allowed: a random block (drawn only for a
+          // block without a global token, outside the band's and the global blocks),
+          // the band covering the whole pair, or a block of global tokens only
+          const int64_t dist = std::abs(static_cast<int64_t>(I) - J);
+          const bool random = !is_gb[static_cast<size_t>(I)] && dist > wb && !is_gb[static_cast<size_t>(J)];
+          const bool full = random || 64 * dist + 63 <= static_cast<int64_t>(window) ||
+                            lay->tok_gbits[static_cast<size_t>(I)] == ~0ull ||
+                            lay->tok_gbits[static_cast<size_t>(J)] == ~0ull;
+          lay->tok_masked.push_back(full ? 0 : 1);
+        }
+        uci.insert(uci.end(), row.begin(), row.end());
+        if (uci.size() > static_cast<size_t>(INT32_MAX)) {
+          delete lay;
+          return BSA_ERR_INVALID_ARG;
+        }
+        urp.push_back(static_cast<int32_t>(uci.size()));
+      }
+    }
+    if (!set_rows(lay, std::move(urp), std::move(uci), is_gb)) {
+      delete lay;
+      return BSA_ERR_INVALID_ARG;
+    }
+  } catch (const std::bad_alloc&) {
+    delete lay;
+    return BSA_ERR_OOM;
+  } catch (...) {
+    delete lay;
+    return BSA_ERR_INVALID_ARG;
+  }
+  *out = lay;
+  return BSA_OK;
+}
+
+int bsa_layout_token_masks(const bsa_layout* lay, int* window, const uint64_t** global_bits) {
+  if (lay == nullptr) return BSA_ERR_INVALID_ARG;
+  if (!lay->token) return BSA_ERR_UNSUPPORTED;
+  if (window != nullptr) *window = static_cast<int>(lay->tok_window);
+  if (global_bits != nullptr) *global_bits = lay->tok_gbits.data();
   return BSA_OK;
 }
 

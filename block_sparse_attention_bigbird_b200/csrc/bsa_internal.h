@@ -77,6 +77,9 @@ struct BwdPlan {
 
 constexpr uint32_t kEntColMask = 0x00FFFFFFu;
 constexpr int kEntBitsShift = 24;
+// Token-level layouts: bit kEntMaskShift + half set when that half's rows need a
+// per-row mask in the entry (not every pair of the two blocks is allowed).
+constexpr int kEntMaskShift = 26;
 
 }  // namespace bsa
 
@@ -93,6 +96,13 @@ struct bsa_layout {
   // its columns); row (h, I) at block 64 m is rows (h, m I .. m I + m - 1) of
   // the tables above, each listing blocks m J .. m J + m - 1 for J in row (h, I)
   std::vector<int32_t> user_row_ptr, user_col_idx;
+  // token-level layouts (bsa_layout_build_tokens): the window in tokens, one bit per
+  // global token (word j: the tokens of block j), and per CSR entry whether the
+  // block pair needs a per-row mask (not every pair of tokens allowed)
+  bool token = false;
+  int64_t tok_window = 0;
+  std::vector<uint64_t> tok_gbits;
+  std::vector<uint8_t> tok_masked;
   std::vector<int32_t> pair_q;      // 2 * n_pairs
   int n_pairs = 0;
   std::vector<int32_t> pair_ptr;    // H*n_pairs + 1
@@ -121,6 +131,7 @@ struct bsa_layout {
   bsa::BwdItem* d_dq_items = nullptr;
   bsa::BwdItem* d_dkv_items = nullptr;
   bsa::SplitTile* d_dq_splits = nullptr;
+  unsigned long long* d_tok_gbits = nullptr;
   bsa::SplitTile* d_dkv_splits = nullptr;
 };
 

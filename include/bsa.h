@@ -98,6 +98,42 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
                      uint64_t seed, const int32_t* globals, bsa_layout** out);
 
 /*
+ * bsa_layout_build_tokens -- host only, no GPU needed.
+ *
+ * A BigBird layout whose window and global set are given in tokens, not whole
+ * blocks ("BigBird 稀疏注意力机制解析", 核心实现 states the window in tokens).
+ * Query token i of head h attends key token j when
+ *     i in G  or  j in G  or  |i - j| <= window
+ *     or  block(j) is a random block of block(i),
+ * with blocks of 64 tokens and
+ *   G        the global tokens: if `global_tokens` is non-NULL, its n_global
+ *            token indices (each in [0, L), any order); otherwise n_global == 0
+ *            -> {}, 1 -> {0}, else floor(k (L-1)/(n_global-1)), k = 0..n_global-1.
+ *   random   for a block I holding no global token, min(n_random, m) blocks
+ *            drawn as in bsa_layout_build (same Philox stream and shuffle) from
+ *            the m blocks outside {J : |I - J| <= floor((window + 63) / 64)} and
+ *            outside the blocks that hold a global token; none for the others.
+ * The layout's block CSR (bsa_layout_csr) is the block layout those rules
+ * touch: bsa_layout_build at block 64 with window floor((window + 63) / 64)
+ * blocks and the blocks holding a global token as its globals.  The forward
+ * applies the token rule inside the block pairs that need it (a per-row mask of
+ * the pair's 64 keys); bsa_backward does not take these layouts
+ * (BSA_ERR_UNSUPPORTED).  L must be a positive multiple of 64; H >= 1;
+ * window, n_global, n_random >= 0 (else BSA_ERR_INVALID_ARG).
+ */
+int bsa_layout_build_tokens(int H, int L, int window, int n_global, int n_random, uint64_t seed,
+                            const int32_t* global_tokens, bsa_layout** out);
+
+/*
+ * bsa_layout_token_masks -- the token-level part of a layout from
+ * bsa_layout_build_tokens: its window in tokens and a host view of L / 64
+ * 64-bit words, bit c of word j set when token 64 j + c is global (valid until
+ * bsa_layout_free).  Either output may be NULL.  BSA_ERR_UNSUPPORTED for a
+ * block layout.
+ */
+int bsa_layout_token_masks(const bsa_layout* layout, int* window, const uint64_t** global_bits);
+
+/*
  * bsa_layout_from_csr -- host only, no GPU needed.
  *
  * Builds a layout from a caller's block mask instead of the BigBird rule.
