@@ -13,6 +13,10 @@ SFree and PFull take one arrival from every softmax thread; a warp's 32 arrivals
 follow its own TMEM accesses in program order, so the model counts one arrival
 per warp.
 
+At head dim 128 the slot has two PV issuers, one per 64-column half of O; both
+commit to the V stage's barrier, which then takes two arrivals, and both read
+the item ring.  The model runs with one PV issuer (d = 64) and with two.
+
 The test replays the roles' sequences under random interleavings, for random
 work lists, with every asynchronous copy and MMA landing at a random later
 moment, and asserts
@@ -31,14 +35,19 @@ import pytest
 from protocol_model import Bar, replay, wait
 
 RING, KST, VST, WARPS = 4, 2, 2, 4
-READERS = 3 + WARPS  # V producer, S issuer, PV issuer, softmax warps
+
+
+def readers(n_pv):
+    return 2 + n_pv + WARPS  # V producer, S issuer, PV issuers, softmax warps
 
 
 class Slot:
     """Contents of one slot's buffers as the replay moves on."""
 
-    def __init__(self, counts):
+    def __init__(self, counts, n_pv=1):
         self.counts = counts
+        self.n_pv = n_pv
+        self.readers = readers(n_pv)
         self.first = [sum(counts[:k]) for k in range(len(counts) + 1)]  # first chunk of tile k
         self.staged = [None] * RING           # item in each ring stage
         self.readers_done = [0] * (len(counts) + 1)
@@ -50,13 +59,20 @@ class Slot:
         self.s_issued, self.s_done = -1, set()
         self.s_loaded = [-1] * WARPS
         self.p_written = [-1] * WARPS
-        self.pv_issued, self.pv_done = 0, set()
+        self.pv_issued = [0] * n_pv            # per column half of O
+        self.pv_done = [set() for _ in range(n_pv)]
 
     def s_complete(self, k):
         return all(x in self.s_done for x in range(self.first[k], self.first[k + 1]))
 
     def pv_complete_to(self, g):
-        return all(x in self.pv_done for x in range(g))
+        return all(x in done for done in self.pv_done for x in range(g))
+
+    def pv_all_done(self, x):
+        return all(x in done for done in self.pv_done)
+
+    def pv_issued_to(self, g):
+        return all(n == g for n in self.pv_issued)
 
 
 def _k_producer(st, n_items, drop=()):
@@ -68,7 +84,7 @@ def _k_producer(st, n_items, drop=()):
         ii = k % RING
 
         def stage(k=k, ii=ii):
-            assert k < RING or st.readers_done[k - RING] == READERS, f"item {k} staged over a read stage"
+            assert k < RING or st.readers_done[k - RING] == st.readers, f"item {k} staged over a read stage"
             st.staged[ii] = k
 
         ops += [wait(f"ItemEmpty{ii}", k // RING - 1), ("do", stage), ("arrive", f"ItemFull{ii}")]
@@ -119,7 +135,7 @@ def _v_producer(st, n_items):
 
             def issue_v(k=k, g=g, vs=vs):
                 assert st.staged[k % RING] == k, "V producer reads a restaged item"
-                assert g < VST or (g - VST) in st.pv_done, f"V({g}) over the stage PV({g - VST}) reads"
+                assert g < VST or st.pv_all_done(g - VST), f"V({g}) over the stage PV({g - VST}) reads"
                 st.v_issued[vs] = g
 
             def land_v(g=g, vs=vs):
@@ -180,9 +196,10 @@ def _s_issuer(st, n_items, drop=()):
     return ops
 
 
-def _pv_issuer(st, n_items):
-    """Per chunk g: O (+)= P(g) V_g once V(g) landed and the four softmax warps
-    wrote P(g); its commit frees the V stage and the P columns."""
+def _pv_issuer(st, n_items, half=0):
+    """Per chunk g: O (+)= P(g) V_g (this issuer's column half of O) once V(g)
+    landed and the four softmax warps wrote P(g); its commit (with the other
+    half's, at d = 128) frees the V stage and the P columns."""
     ops, g = [], 0
     for k in range(n_items + 1):
         ii = k % RING
@@ -195,13 +212,13 @@ def _pv_issuer(st, n_items):
             def issue_pv(g=g, vs=vs):
                 assert st.v_landed[vs] == g and st.v_issued[vs] == g, f"PV({g}) reads a V stage not holding V({g})"
                 assert all(x == g for x in st.p_written), f"PV({g}) before every warp wrote P({g})"
-                assert st.pv_issued == g
-                st.pv_issued = g + 1
+                assert st.pv_issued[half] == g
+                st.pv_issued[half] = g + 1
 
             def land_pv(g=g, vs=vs):
                 assert st.v_issued[vs] == g, f"V stage reloaded while PV({g}) read it"
                 assert all(x == g for x in st.p_written), f"P columns rewritten while PV({g}) read them"
-                st.pv_done.add(g)
+                st.pv_done[half].add(g)
 
             ops += [wait(f"VFull{vs}", g // VST), wait("PFull", g), ("do", issue_pv),
                     ("async", f"VFree{vs}", land_pv)]
@@ -226,7 +243,7 @@ def _softmax_warp(st, n_items, w, drop=()):
     def epilogue(kp, g_now):
         def f():
             assert st.staged[kp % RING] == kp, f"epilogue of tile {kp} reads a restaged item"
-            assert st.pv_complete_to(g_now) and st.pv_issued == g_now, f"O of tile {kp} read with a PV pending"
+            assert st.pv_complete_to(g_now) and st.pv_issued_to(g_now), f"O of tile {kp} read with a PV pending"
             assert st.s_complete(kp), f"O of tile {kp} staged over Q while an S MMA reads it"
             assert st.q_issued[kp & 1] == kp, f"O of tile {kp} staged in a reloaded Q buffer"
             st.readers_done[kp] += 1
@@ -257,7 +274,7 @@ def _softmax_warp(st, n_items, w, drop=()):
                 q_pending, pend = pend, None
 
             def write_p(g=g):
-                assert st.pv_complete_to(g) and st.pv_issued == g, f"P({g}) / O rescale with a PV pending"
+                assert st.pv_complete_to(g) and st.pv_issued_to(g), f"P({g}) / O rescale with a PV pending"
                 st.p_written[w] = g
 
             ops += [("do", write_p), ("arrive", "PFull")]
@@ -271,18 +288,22 @@ def _softmax_warp(st, n_items, w, drop=()):
     return ops
 
 
-def _roles(counts, drop=()):
+def _roles(counts, drop=(), n_pv=1):
     n_items = len(counts)
-    st = Slot(counts)
+    st = Slot(counts, n_pv)
+    vfree = 1 if "VFreeCount" in drop else n_pv
     bars = {}
     for name, count in ([(f"QFull{i}", 1) for i in range(2)] + [(f"QEmpty{i}", WARPS) for i in range(2)] +
                         [(f"KFull{i}", 1) for i in range(KST)] + [(f"KFree{i}", 1) for i in range(KST)] +
-                        [(f"VFull{i}", 1) for i in range(VST)] + [(f"VFree{i}", 1) for i in range(VST)] +
+                        [(f"VFull{i}", 1) for i in range(VST)] + [(f"VFree{i}", vfree) for i in range(VST)] +
                         [("SFull", 1), ("SFree", WARPS), ("PFull", WARPS)] +
-                        [(f"ItemFull{i}", 1) for i in range(RING)] + [(f"ItemEmpty{i}", READERS) for i in range(RING)]):
+                        [(f"ItemFull{i}", 1) for i in range(RING)] +
+                        [(f"ItemEmpty{i}", st.readers) for i in range(RING)]):
         bars[name] = Bar(name, count)
     roles = {"k_producer": _k_producer(st, n_items, drop), "v_producer": _v_producer(st, n_items),
-             "s_issuer": _s_issuer(st, n_items, drop), "pv_issuer": _pv_issuer(st, n_items)}
+             "s_issuer": _s_issuer(st, n_items, drop)}
+    for h in range(n_pv):
+        roles[f"pv_issuer{h}"] = _pv_issuer(st, n_items, h)
     for w in range(WARPS):
         roles[f"softmax{w}"] = _softmax_warp(st, n_items, w, drop)
     return bars, roles, st
@@ -293,15 +314,16 @@ def _work(rnd):
     return [rnd.randint(1, 6) for _ in range(rnd.randint(1, 10))]
 
 
-def test_random_schedules_keep_every_buffer_consistent():
+@pytest.mark.parametrize("n_pv", [1, 2])
+def test_random_schedules_keep_every_buffer_consistent(n_pv):
     for seed in range(400):
         rnd = random.Random(seed)
         counts = _work(rnd)
-        bars, roles, st = _roles(counts)
+        bars, roles, st = _roles(counts, n_pv=n_pv)
         replay(bars, roles, seed)
         total = sum(counts)
-        assert st.pv_done == set(range(total)) and st.s_done == set(range(total))
-        assert st.readers_done[:len(counts)] == [READERS] * len(counts)
+        assert all(done == set(range(total)) for done in st.pv_done) and st.s_done == set(range(total))
+        assert st.readers_done[:len(counts)] == [readers(n_pv)] * len(counts)
 
 
 @pytest.mark.parametrize("missing", ["VFree", "SFree", "QEmpty"])
@@ -314,6 +336,20 @@ def test_the_model_catches_a_missing_wait(missing):
     for seed in range(200):
         rnd = random.Random(seed)
         bars, roles, _ = _roles(_work(rnd), drop=(missing,))
+        try:
+            replay(bars, roles, seed)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+def test_the_model_catches_a_v_barrier_counting_one_of_two_pv_issuers():
+    # planting a mistake: at d = 128 the V stage's barrier initialised for one
+    # arrival lets V(g + 2) or P(g + 1) in while the other half's PV(g) still reads
+    caught = 0
+    for seed in range(200):
+        rnd = random.Random(seed)
+        bars, roles, _ = _roles(_work(rnd), drop=("VFreeCount",), n_pv=2)
         try:
             replay(bars, roles, seed)
         except AssertionError:
