@@ -103,11 +103,25 @@ struct BwdParams {
   const int32_t* pair;       // tile blocks, 2 per tile (second -1: single block)
   const uint32_t* pair_ent;  // entries: block | membership << 24
   const unsigned long long* keybits;  // [B, nb] or null
+  // token-level layouts (else null): bit c of word j set when token 64 j + c is global,
+  // and the window in tokens; entries flagged at kEntMaskShift + half get a mask of
+  // the other block's 64 tokens per row
+  const unsigned long long* tok_gbits;
+  long long tok_window;
   float* records;  // partial sums of split tiles, per batch element n_records of them
   int B, H, L, nb, n_items, n_records;
   float scale, scale_log2;
   unsigned long long timeout_ns;
 };
+
+// The tokens of block `blk` within [c - w, c + w]: the token-level band of token c
+// (its keys for a query, its queries for a key), one bit per token of the block.
+__device__ __forceinline__ unsigned long long band_bits(long long c, long long w, int blk) {
+  const long long lo = c - w - 64ll * blk, hi = c + w - 64ll * blk;
+  if (hi < 0 || lo > 63) return 0ull;
+  const int l = lo < 0 ? 0 : static_cast<int>(lo), h = hi > 63 ? 63 : static_cast<int>(hi);
+  return (h == 63 ? ~0ull : ((1ull << (h + 1)) - 1ull)) & ~((1ull << l) - 1ull);
+}
 
 constexpr uint32_t kIdescQK = ptx::idesc_bf16_f32(128, 64, false);  // B K-major
 constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, 64, true);   // B MN-major
@@ -393,6 +407,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
       const ItemRef t = item_at(p, it);
       const bool active = half == 0 || t.tb >= 0;
       const int blk = half ? t.tb : t.ta;
+      // token-level layouts: this row's token (a query for dQ, a key for dK/dV) and
+      // whether it is global (it then pairs with every token)
+      long long tok_self = 0;
+      bool tok_self_global = false;
+      if (p.tok_gbits != nullptr && active) {
+        tok_self = 64ll * blk + (r & 63);
+        tok_self_global = (p.tok_gbits[blk] >> (r & 63)) & 1ull;
+      }
       // dQ: this row's lse (log2) and D; dKV: whether this key is kept by the padding mask
       float lse2 = INFINITY, drow = 0.f;
       bool key_kept = false;
@@ -430,16 +452,26 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
         ptx::reg_fence(s_raw);
         ptx::reg_fence(dp_raw);
         const bool member = active && ((e >> (kEntBitsShift + half)) & 1u);
+        // the other block's tokens this row pairs with: all, unless the entry is
+        // flagged (token level: global tokens, and the band around this row's token)
+        unsigned long long pair_mask = ~0ull;
+        if (p.tok_gbits != nullptr && ((e >> (kEntMaskShift + half)) & 1u) && !tok_self_global) {
+          const int ob = static_cast<int>(e & kEntColMask);
+          pair_mask = band_bits(tok_self, p.tok_window, ob) | p.tok_gbits[ob];
+        }
         if constexpr (kDkv) {
           const bool take = member && key_kept;
+          // this warp's 32 queries of the entry's block that this key pairs with
+          const uint32_t qh = take ? static_cast<uint32_t>(pair_mask >> (32 * ch)) : 0u;
           const float* vec = reinterpret_cast<const float*>(smem + kSmemVec + es * 2 * kVecBytes) + 32 * ch;
           uint32_t ppk[16], dpk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const float2 l2 = *reinterpret_cast<const float2*>(vec + 2 * c);
             const float2 dd = *reinterpret_cast<const float2*>(vec + 64 + 2 * c);
-            const float p0 = take ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - l2.x) : 0.f;
-            const float p1 = take ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - l2.y) : 0.f;
+            const float p0 = ((qh >> (2 * c)) & 1u) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - l2.x) : 0.f;
+            const float p1 =
+                ((qh >> (2 * c + 1)) & 1u) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - l2.y) : 0.f;
             ppk[c] = pack_bf16x2(p0, p1);
             dpk[c] = pack_bf16x2(p0 * (__uint_as_float(dp_raw[2 * c]) - dd.x),
                                  p1 * (__uint_as_float(dp_raw[2 * c + 1]) - dd.y));
@@ -449,7 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
         } else {
           unsigned long long mk = 0ull;
           if (member)
-            mk = p.keybits != nullptr ? p.keybits[static_cast<size_t>(t.b) * p.nb + (e & kEntColMask)] : ~0ull;
+            mk = (p.keybits != nullptr ? p.keybits[static_cast<size_t>(t.b) * p.nb + (e & kEntColMask)] : ~0ull) &
+                 pair_mask;
           const uint32_t mh = static_cast<uint32_t>(mk >> (32 * ch));  // this warp's 32 keys
           uint32_t pk[16];
 #pragma unroll
@@ -626,7 +659,6 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
       dq == nullptr || dk == nullptr || dv == nullptr || lay == nullptr || B < 1 || H < 1 || L < 1)
     return BSA_ERR_INVALID_ARG;
   if (d != kHeadDim) return BSA_ERR_UNSUPPORTED;
-  if (lay->token) return BSA_ERR_UNSUPPORTED;  // per-row masks: the forward only
   if (H != lay->H || L != lay->L) return BSA_ERR_LAYOUT_MISMATCH;
   if (static_cast<int64_t>(B) * H * L > INT32_MAX - 64) return BSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(dout, 16) ||
@@ -664,6 +696,8 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   prm.dk = static_cast<__nv_bfloat16*>(dk);
   prm.dv = static_cast<__nv_bfloat16*>(dv);
   prm.keybits = key_mask != nullptr ? keybits : nullptr;
+  prm.tok_gbits = lay->token ? lay->d_tok_gbits : nullptr;
+  prm.tok_window = lay->tok_window;
   prm.B = B;
   prm.H = H;
   prm.L = L;

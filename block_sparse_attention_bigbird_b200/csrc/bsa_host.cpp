@@ -350,18 +350,24 @@ void build_tiles(bsa_layout* lay, const std::vector<uint8_t>& dense) {
         ++t_ptr[static_cast<size_t>(h) * nb + lay->col_idx[static_cast<size_t>(x)] + 1];
   for (size_t x = 0; x + 1 < t_ptr.size(); ++x) t_ptr[x + 1] += t_ptr[x];
   std::vector<int32_t> fill(t_ptr.begin(), t_ptr.end() - 1);
+  // a token-level layout's per-pair mask flags follow their entries into the transpose
+  std::vector<uint8_t> t_masked(lay->token ? lay->col_idx.size() : 0);
   for (int h = 0; h < H; ++h)
     for (int i = 0; i < nb; ++i)
       for (int32_t x = lay->row_ptr[static_cast<size_t>(h) * nb + i];
-           x < lay->row_ptr[static_cast<size_t>(h) * nb + i + 1]; ++x)
-        t_col[static_cast<size_t>(fill[static_cast<size_t>(h) * nb + lay->col_idx[static_cast<size_t>(x)]]++)] = i;
+           x < lay->row_ptr[static_cast<size_t>(h) * nb + i + 1]; ++x) {
+        const size_t dst =
+            static_cast<size_t>(fill[static_cast<size_t>(h) * nb + lay->col_idx[static_cast<size_t>(x)]]++);
+        t_col[dst] = i;
+        if (lay->token) t_masked[dst] = lay->tok_masked[static_cast<size_t>(x)];
+      }
   std::vector<uint8_t> kdense(static_cast<size_t>(nb), 1);
   for (int h = 0; h < H; ++h)
     for (int j = 0; j < nb; ++j)
       if (t_ptr[static_cast<size_t>(h) * nb + j + 1] - t_ptr[static_cast<size_t>(h) * nb + j] != nb)
         kdense[static_cast<size_t>(j)] = 0;
   make_tiles(H, nb, t_ptr, t_col, kdense, &lay->ktiles.pair_q, &lay->ktiles.n_pairs, &lay->ktiles.pair_ptr,
-             &lay->ktiles.pair_ent);
+             &lay->ktiles.pair_ent, lay->token ? &t_masked : nullptr);
   make_bwd_plan(H, lay->ktiles.pair_q, lay->ktiles.n_pairs, lay->ktiles.pair_ptr, &lay->dkv_plan);
 }
 

@@ -94,3 +94,31 @@ def test_masked_dense_equals_scalar_loops_with_key_padding():
     assert np.abs(o - o2).max() < 1e-12
     fin = np.isfinite(lse2)
     assert np.array_equal(fin, np.isfinite(lse)) and np.abs(lse[fin] - lse2[fin]).max() < 1e-12
+
+
+def test_backward_oracle_on_a_token_layout_equals_autograd():
+    """oracle.backward with a token-level layout against torch autograd through a
+    dense softmax masked by the token rule written out here per pair."""
+    from oracle import backward as OB
+    B, H, L, d = 1, 2, 64 * 4, 8
+    q, k, v = _qkv(B, H, L, d, seed=11)
+    do = _qkv(B, H, L, d, seed=12)[0]
+    lay = OL.build_token_layout(H, L, 21, 2, 1, 3)
+    g = OL.global_tokens(L, 2)
+    i = torch.arange(L)
+    allowed = torch.zeros(H, L, L, dtype=torch.bool)
+    for h in range(H):
+        gt = torch.zeros(L, dtype=torch.bool)
+        gt[g] = True
+        base = ((i[:, None] - i[None, :]).abs() <= 21) | gt[:, None] | gt[None, :]
+        for I in range(L // 64):
+            for J in lay["token"]["random"][h][I]:
+                base[64 * I:64 * I + 64, 64 * J:64 * J + 64] = True
+        allowed[h] = base
+    qq, kk, vv = (t.clone().requires_grad_() for t in (q, k, v))
+    s = (qq @ kk.transpose(-1, -2)) / math.sqrt(d)
+    o = torch.softmax(s.masked_fill(~allowed[None], -math.inf), -1) @ vv
+    o.backward(do)
+    got = OB.attention_backward(q, k, v, do, lay)
+    for a, b in zip(got, (qq.grad, kk.grad, vv.grad)):
+        assert np.abs(a - b.numpy()).max() < 1e-12

@@ -3,14 +3,15 @@ oracle's rule (CPU), and the forward against the fp64 oracle (GPU).
 
 CPU: the block CSR and the global-token bits equal the oracle's; every tile entry
 the library leaves without its per-row-mask flag for a half joins two blocks whose
-every token pair the oracle's rule allows (the kernel applies no mask there);
-entries with the flag lie in the rows of that half; the backward refuses these
-layouts before any device work.
+every token pair the oracle's rule allows (the kernels apply no mask there);
+entries with the flag lie in the rows of that half.
 GPU: windows below, at and above one block and not multiples of 64, global tokens
 not aligned to blocks (explicit and by the linspace rule, some in one block
 together), random blocks, a partially padded key tail, ragged tiles and split
 global rows, L = 16384 on sampled rows, and d = 128; O max-abs 2e-2, lse max-abs
-1e-3, the parity tolerances.
+1e-3, the parity tolerances.  The backward over token layouts against the oracle's
+gradients at the backward suite's bounds (2^-6 of each element's sum of absolute
+terms plus 2^-8 of its value).
 """
 
 import numpy as np
@@ -73,15 +74,16 @@ def test_tables_match_the_oracle_rule(H, L, w, ng, nr, seed, gt):
                         assert block.all(), (h, I, J)
 
 
-def test_block_layouts_report_no_token_part_and_backward_refuses_token_layouts():
+def test_block_layouts_report_no_token_part_and_bad_arguments_are_refused():
     blk = bsa.bsa_layout_build(1, 64 * 4, 64, 1, 1, 1, 0)
     with pytest.raises(bsa.BsaError):
         bsa.bsa_layout_token_masks(blk)
     lay = bsa.bsa_layout_build_tokens(1, 64 * 4, 10, 1, 1, 0)
     fake = 1 << 20
+    # the backward takes token layouts: argument checks pass, the layout is not uploaded
     code = bsa.lib.bsa_backward(fake, fake, fake, fake, fake, fake, 1, 1, 64 * 4, 64, lay.handle, None, 0.0,
                                 fake, fake, fake, fake, 1 << 20, None)
-    assert code == bsa.BSA_ERR_UNSUPPORTED
+    assert code == bsa.BSA_ERR_LAYOUT_MISMATCH
     for bad in ((0, 64, 1, 0, 0), (1, 100, 1, 0, 0), (1, 64, -1, 0, 0), (1, 64, 1, -1, 0), (1, 64, 1, 0, -1)):
         with pytest.raises(bsa.BsaError):
             bsa.bsa_layout_build_tokens(*bad)
@@ -151,3 +153,34 @@ def test_token_layout_long_sequence_sampled_rows():
         l = lse[b, h].cpu().numpy()[tokens]
         assert np.abs(o - o_ref).max() <= 2e-2
         assert np.abs(l - l_ref).max() <= 1e-3
+
+
+BWD_CASES = [  # name, B, H, L, window, n_global, n_random, seed, global tokens, key pad
+    ("band17_random", 2, 2, 64 * 13, 17, 0, 2, 1, None, 0),
+    ("band100_globals", 1, 3, 64 * 16, 100, 3, 3, 2, None, 0),
+    ("unaligned_globals_padding", 2, 2, 64 * 10, 64, 0, 1, 3, [5, 6, 70, 383, 600], 100),
+    ("globals_split_rows", 1, 2, 64 * 64, 40, 2, 3, 6, [10, 4000], 0),
+]
+
+
+@pytest.mark.parametrize("name,B,H,L,w,ng,nr,seed,gt,pad", BWD_CASES, ids=[c[0] for c in BWD_CASES])
+@pytest.mark.gpu
+@pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
+def test_token_layout_backward_matches_oracle(name, B, H, L, w, ng, nr, seed, gt, pad):
+    from oracle import backward as OB
+    from test_backward import _check_grads
+    wl = workloads.custom(B, H, L, 1, 0, 0, seed=seed, key_pad_tail=pad)
+    q, k, v = workloads.make_qkv(wl, data_seed=seed)
+    do = workloads.make_grad(wl, seed=100 + seed)
+    km = workloads.make_key_mask(wl) if pad else None
+    lay = bsa.bsa_layout_build_tokens(H, L, w, ng, nr, seed, global_tokens=gt)
+    bsa.bsa_layout_upload(lay)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), do.to(dev)
+    kmd = km.to(dev) if km is not None else None
+    out, lse = bsa.bsa_forward(qd, kd, vd, lay, key_mask=kmd)
+    dq, dk, dv = bsa.bsa_backward(qd, kd, vd, out, dod, lse, lay, key_mask=kmd)
+    assert bsa.bsa_sync_status() == 0
+    ref = OL.build_token_layout(H, L, w, ng, nr, seed, explicit_globals=gt)
+    dq_r, dk_r, dv_r, mags = OB.attention_backward(q, k, v, do, ref, key_mask=km, with_magnitude=True)
+    _check_grads([t.float().cpu().numpy() for t in (dq, dk, dv)], (dq_r, dk_r, dv_r), mags)
