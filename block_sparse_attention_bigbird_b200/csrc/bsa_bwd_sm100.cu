@@ -9,8 +9,8 @@
 //   D  = rowsum(dO * O)                               bsa_bwd_prep_kernel
 //   P  = 2^(S * scale * log2 e - lse * log2 e),  S = Q K^T on the attended keys
 //   dP = dO V^T,  dS = P * (dP - D)
-//   dQ = scale * dS K                                 bsa_bwd_kernel<false>
-//   dK = scale * dS^T Q,  dV = P^T dO                 bsa_bwd_kernel<true>
+//   dQ = scale * dS K                                 bsa_bwd_kernel<false, .>
+//   dK = scale * dS^T Q,  dV = P^T dO                 bsa_bwd_kernel<true, .>
 // P is rebuilt from lse, so no softmax statistics are recomputed.
 //
 // bsa_bwd_kernel runs persistent CTAs (one per SM, 352 threads) over a list of
@@ -192,7 +192,9 @@ __device__ __forceinline__ void store32(const float (&v)[32], float f, __nv_bflo
   }
 }
 
-template <bool kDkv>
+// kTok: the layout is token-level (flagged entries get per-row masks); block layouts
+// run the instantiation without that code.
+template <bool kDkv, bool kTok>
 __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_addr(smem_raw);
@@ -411,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
       // whether it is global (it then pairs with every token)
       long long tok_self = 0;
       bool tok_self_global = false;
-      if (p.tok_gbits != nullptr && active) {
+      if (kTok && active) {
         tok_self = 64ll * blk + (r & 63);
         tok_self_global = (p.tok_gbits[blk] >> (r & 63)) & 1ull;
       }
@@ -455,13 +457,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
         // the other block's tokens this row pairs with: all, unless the entry is
         // flagged (token level: global tokens, and the band around this row's token)
         unsigned long long pair_mask = ~0ull;
-        if (p.tok_gbits != nullptr && ((e >> (kEntMaskShift + half)) & 1u) && !tok_self_global) {
+        if (kTok && ((e >> (kEntMaskShift + half)) & 1u) && !tok_self_global) {
           const int ob = static_cast<int>(e & kEntColMask);
           pair_mask = band_bits(tok_self, p.tok_window, ob) | p.tok_gbits[ob];
         }
         if constexpr (kDkv) {
           const bool take = member && key_kept;
-          // this warp's 32 queries of the entry's block that this key pairs with
+          // this warp's 32 queries of the entry's block that this key pairs with (all
+          // of them or none at block level)
           const uint32_t qh = take ? static_cast<uint32_t>(pair_mask >> (32 * ch)) : 0u;
           const float* vec = reinterpret_cast<const float*>(smem + kSmemVec + es * 2 * kVecBytes) + 32 * ch;
           uint32_t ppk[16], dpk[16];
@@ -469,9 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_bwd_kernel(const __grid_const
           for (int c = 0; c < 16; ++c) {
             const float2 l2 = *reinterpret_cast<const float2*>(vec + 2 * c);
             const float2 dd = *reinterpret_cast<const float2*>(vec + 64 + 2 * c);
-            const float p0 = ((qh >> (2 * c)) & 1u) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - l2.x) : 0.f;
-            const float p1 =
-                ((qh >> (2 * c + 1)) & 1u) ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - l2.y) : 0.f;
+            const bool t0 = kTok ? ((qh >> (2 * c)) & 1u) != 0u : take;
+            const bool t1 = kTok ? ((qh >> (2 * c + 1)) & 1u) != 0u : take;
+            const float p0 = t0 ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c]) * sl2 - l2.x) : 0.f;
+            const float p1 = t1 ? ptx::ex2_approx(__uint_as_float(s_raw[2 * c + 1]) * sl2 - l2.y) : 0.f;
             ppk[c] = pack_bf16x2(p0, p1);
             dpk[c] = pack_bf16x2(p0 * (__uint_as_float(dp_raw[2 * c]) - dd.x),
                                  p1 * (__uint_as_float(dp_raw[2 * c + 1]) - dd.y));
@@ -611,9 +615,13 @@ int bwd_device_setup(int dev) {
     }
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaFuncSetAttribute(bsa_bwd_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(bsa_bwd_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemAlloc)) != cudaSuccess ||
-        cudaFuncSetAttribute(bsa_bwd_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(bsa_bwd_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemAlloc)) != cudaSuccess ||
+        cudaFuncSetAttribute(bsa_bwd_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemAlloc)) != cudaSuccess ||
+        cudaFuncSetAttribute(bsa_bwd_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemAlloc)) != cudaSuccess) {
       g_setup_status[dev] = BSA_ERR_CUDA;
       return;
@@ -717,7 +725,10 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   pq.n_items = static_cast<int>(lay->dq_plan.items.size());
   const int64_t gq = std::min<int64_t>(static_cast<int64_t>(B) * pq.n_items, g_sms[dev]);
   if (gq > 0) {
-    bsa_bwd_kernel<false><<<static_cast<unsigned>(gq), kThreads, kSmemAlloc, s>>>(pq);
+    if (lay->token)
+      bsa_bwd_kernel<false, true><<<static_cast<unsigned>(gq), kThreads, kSmemAlloc, s>>>(pq);
+    else
+      bsa_bwd_kernel<false, false><<<static_cast<unsigned>(gq), kThreads, kSmemAlloc, s>>>(pq);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   // dK and dV over the key tiles
@@ -730,7 +741,10 @@ extern "C" int bsa_backward(const void* q, const void* k, const void* v, const v
   pk.n_items = static_cast<int>(lay->dkv_plan.items.size());
   const int64_t gk = std::min<int64_t>(static_cast<int64_t>(B) * pk.n_items, g_sms[dev]);
   if (gk > 0) {
-    bsa_bwd_kernel<true><<<static_cast<unsigned>(gk), kThreads, kSmemAlloc, s>>>(pk);
+    if (lay->token)
+      bsa_bwd_kernel<true, true><<<static_cast<unsigned>(gk), kThreads, kSmemAlloc, s>>>(pk);
+    else
+      bsa_bwd_kernel<true, false><<<static_cast<unsigned>(gk), kThreads, kSmemAlloc, s>>>(pk);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   const int n_dq_split = static_cast<int>(lay->dq_plan.splits.size());
