@@ -117,8 +117,9 @@ int bsa_layout_build(int H, int L, int block, int window, int n_global, int n_ra
  * touch: bsa_layout_build at block 64 with window floor((window + 63) / 64)
  * blocks and the blocks holding a global token as its globals.  The forward
  * applies the token rule inside the block pairs that need it (a per-row mask of
- * the pair's 64 keys); bsa_backward does not take these layouts
- * (BSA_ERR_UNSUPPORTED).  L must be a positive multiple of 64; H >= 1;
+ * the pair's 64 keys), and so does bsa_backward (a mask of the key block's keys
+ * per query row for dQ, of the query block's queries per key row for dK and dV).
+ * L must be a positive multiple of 64; H >= 1;
  * window, n_global, n_random >= 0 (else BSA_ERR_INVALID_ARG).
  */
 int bsa_layout_build_tokens(int H, int L, int window, int n_global, int n_random, uint64_t seed,
