@@ -53,6 +53,42 @@ int main(void) {
   CHECK(memcmp(rp, rp2, sizeof(int32_t) * (size_t)(H * nb + 1)) == 0);
   CHECK(memcmp(ci, ci2, sizeof(int32_t) * (size_t)nnz) == 0);
 
+  /* a token-level layout: window 70 tokens, global tokens 3 and 300 (blocks 0 and 4) */
+  bsa_layout* tok = NULL;
+  const int32_t gtok[2] = {300, 3};
+  CHECK(bsa_layout_build_tokens(2, 512, 70, 2, 1, 7, gtok, &tok) == BSA_OK && tok != NULL);
+  int tw = -1;
+  const uint64_t* gbits = NULL;
+  CHECK(bsa_layout_token_masks(tok, &tw, &gbits) == BSA_OK && tw == 70);
+  CHECK(gbits[0] == (1ull << 3) && gbits[4] == (1ull << (300 - 256)) && gbits[1] == 0);
+  CHECK(bsa_layout_globals(tok, &g, &ng) == BSA_OK && ng == 2 && g[0] == 0 && g[1] == 4);
+  {
+    /* its block CSR is the block layout with window ceil(70 / 64) = 2 blocks and those two blocks global */
+    bsa_layout* blk = NULL;
+    const int32_t gb[2] = {0, 4};
+    CHECK(bsa_layout_build(2, 512, 64, 2, 2, 1, 7, gb, &blk) == BSA_OK);
+    const int32_t *trp = NULL, *tci = NULL, *brp = NULL, *bci = NULL;
+    int64_t tn = 0, bn = 0;
+    CHECK(bsa_layout_csr(tok, &trp, &tci, &tn, NULL, NULL) == BSA_OK);
+    CHECK(bsa_layout_csr(blk, &brp, &bci, &bn, NULL, NULL) == BSA_OK && tn == bn);
+    CHECK(memcmp(trp, brp, sizeof(int32_t) * (size_t)(H * nb + 1)) == 0);
+    CHECK(memcmp(tci, bci, sizeof(int32_t) * (size_t)tn) == 0);
+    bsa_layout_free(blk);
+  }
+  CHECK(bsa_layout_token_masks(lay, &tw, &gbits) == BSA_ERR_UNSUPPORTED);
+  bsa_layout* tbad = NULL;
+  CHECK(bsa_layout_build_tokens(2, 500, 70, 0, 0, 0, NULL, &tbad) == BSA_ERR_INVALID_ARG && tbad == NULL);
+  {
+    const int32_t out_of_range[1] = {512};
+    CHECK(bsa_layout_build_tokens(2, 512, 70, 1, 0, 0, out_of_range, &tbad) == BSA_ERR_INVALID_ARG);
+  }
+  size_t ws128 = 0;
+  CHECK(bsa_forward_workspace_bytes(lay, 2, 128, &ws128) == BSA_OK && ws128 >= ws);
+  CHECK(bsa_forward_workspace_bytes(lay, 2, 96, &ws128) == BSA_ERR_UNSUPPORTED);
+  CHECK(bsa_out_projection(NULL, NULL, NULL, 1, 1, 64, 64, NULL, NULL) == BSA_ERR_INVALID_ARG);
+  CHECK(bsa_qkv_projection(NULL, NULL, NULL, 1, 64, 1, NULL, NULL, NULL, NULL) == BSA_ERR_INVALID_ARG);
+  bsa_layout_free(tok);
+
   /* documented errors, before anything touches a GPU */
   bsa_layout* bad = (bsa_layout*)1;
   CHECK(bsa_layout_build(2, 512, 96, 1, 1, 1, 0, NULL, &bad) == BSA_ERR_UNSUPPORTED && bad == NULL);
