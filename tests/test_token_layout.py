@@ -184,3 +184,35 @@ def test_token_layout_backward_matches_oracle(name, B, H, L, w, ng, nr, seed, gt
     ref = OL.build_token_layout(H, L, w, ng, nr, seed, explicit_globals=gt)
     dq_r, dk_r, dv_r, mags = OB.attention_backward(q, k, v, do, ref, key_mask=km, with_magnitude=True)
     _check_grads([t.float().cpu().numpy() for t in (dq, dk, dv)], (dq_r, dk_r, dv_r), mags)
+
+
+def test_random_token_layouts_equal_the_oracle():
+    """A seeded sweep of token-level layouts: the library's block CSR and global bits
+    equal the oracle's, bit for bit, for windows from 0 to past the sequence, global
+    tokens by rule and explicit (duplicates, neighbours, both ends), and random
+    block counts from 0 to more than there are candidates."""
+    rng = np.random.default_rng(123)
+    for _ in range(40):
+        H = int(rng.integers(1, 4))
+        nb = int(rng.integers(1, 14))
+        L = 64 * nb
+        w = int(rng.choice([0, 1, 31, 63, 64, 65, 127, 200, L + 5]))
+        nr = int(rng.integers(0, 6))
+        seed = int(rng.integers(0, 2 ** 40))
+        if rng.random() < 0.5:
+            gt = None
+            ng = int(rng.integers(0, 5))
+        else:
+            gt = [int(x) for x in rng.integers(0, L, int(rng.integers(0, 6)))]
+            if gt and rng.random() < 0.5:
+                gt += [gt[0], L - 1, 0]
+            ng = len(gt)
+        lay = bsa.bsa_layout_build_tokens(H, L, w, ng, nr, seed, global_tokens=gt)
+        ref = OL.build_token_layout(H, L, w, ng, nr, seed, explicit_globals=gt)
+        rp, ci = bsa.bsa_layout_csr(lay)
+        assert np.array_equal(rp, ref["row_ptr"]) and np.array_equal(ci, ref["col_idx"]), (H, L, w, ng, nr, seed, gt)
+        _, bits = bsa.bsa_layout_token_masks(lay)
+        want = np.zeros(nb, dtype=np.uint64)
+        for t in ref["token"]["globals"]:
+            want[t // 64] |= np.uint64(1) << np.uint64(t % 64)
+        assert np.array_equal(bits, want)
