@@ -38,6 +38,8 @@
 // Long unions (global rows) are cut into chunks run as separate work items; each stores
 // a partial (O, m, l) record, and bsa_merge_kernel, launched after the forward, merges a
 // split tile's records into its output rows.
+// Token-level layouts (window and global tokens not aligned to blocks) run their own
+// instantiation (kTok): flagged entries get a per-row mask of their 64 keys.
 // Every wait is bounded (globaltimer); on expiry the CTA records BSA_ERR_DEVICE_TIMEOUT,
 // drains its own copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
