@@ -331,14 +331,31 @@ bool map_rows(CUtensorMap* m, const void* ptr, uint64_t B, uint64_t rows, uint64
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Per device, once: whether it is an sm_100 part, its SM count, and the kernel's
+// shared-memory attribute set.  A failed setup is not cached (the next call retries).
+constexpr int kMaxProjDevices = 64;
+int g_proj_sms[kMaxProjDevices] = {};
+std::mutex g_proj_mu;
+
 int device_sms() {
-  int dev = -1, major = 0, minor = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxProjDevices) return BSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_proj_mu);
+  if (g_proj_sms[dev] != 0) return g_proj_sms[dev];
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return BSA_ERR_CUDA;
-  if (major != 10 || minor != 0) return BSA_ERR_UNSUPPORTED;
+  if (major != 10 || minor != 0) {
+    g_proj_sms[dev] = BSA_ERR_UNSUPPORTED;
+    return BSA_ERR_UNSUPPORTED;
+  }
+  if (cudaFuncSetAttribute(bsa_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(kPSmemAlloc)) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  g_proj_sms[dev] = sms;
   return sms;
 }
 
@@ -351,9 +368,6 @@ int launch(ProjParams& p, int B, cudaStream_t s) {
   if (tiles > (1ll << 30)) return BSA_ERR_INVALID_ARG;
   p.tiles = static_cast<int>(tiles);
   p.timeout_ns = kDefaultTimeoutNs;
-  if (cudaFuncSetAttribute(bsa_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kPSmemAlloc)) != cudaSuccess)
-    return BSA_ERR_CUDA;
   const int grid = static_cast<int>(std::min<long long>(tiles, sms));
   bsa_proj_kernel<<<grid, kPThreads, kPSmemAlloc, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
